@@ -1,0 +1,299 @@
+"""fp64 CPU oracle for the SeerAttention-R block-sparse decode step.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline / reference leg of ``bench.py`` use it.  It shares no code with the
+CUDA library (no kernels, headers, helpers, tables or constants); it works on
+plain numpy float64 arrays that the caller has already converted from the
+seeded inputs.
+
+What the step computes, and where each part comes from
+------------------------------------------------------
+Sources are the pages this project was specified from, cited by page title and
+section:
+
+* "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning" (paper
+  summary page, Abstract): a self-distilled gate picks KV blocks for each
+  decode query; query pooling is removed for auto-regressive decoding; blocks
+  are large (64 or 128 tokens); accuracy holds at a 4K-token budget; the
+  sparse decoding kernel runs at 90% sparsity.
+* "Sparse Attention Reasoning" (Agent Skill page), Step 1 "Design Sparse
+  Attention Gate": k from a sparsity ratio and a top-k over scores.
+* Same page, Step 4 "Optimized Kernel Implementation": the meaning of sparse
+  attention -- scores Q.K^T / sqrt(head_dim), unselected keys filled with
+  -inf, softmax over keys, weights times V.
+* The step specification this library implements (gate = mean-pooled block
+  keys dotted with the gate-projected query, in fp32 on the GPU; per-KV-head
+  top-k with ties to the lower block index and an optional forced newest
+  block; split-KV partials merged by a log-sum-exp combine).
+
+Readings taken where the pages are silent (each is also listed in the design
+notes): the GQA group's score is the mean of its query heads' scores; the gate
+scale is 1/sqrt(D); k = max(1, ceil((1000 - permille) * NB / 1000)) from a
+sparsity, k = max(1, min(NB, budget // bs)) from a token budget; a forced
+newest block counts toward k; indices come out ascending; NaN scores rank
+below -inf and -0.0 equals +0.0; split s of S covers the selected blocks
+[floor(s*n/S), floor((s+1)*n/S)) of the ascending list.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` to closed
+forms, brute force, library routines or the hand-worked fixtures in
+``tests/golden/``; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from typing import Sequence
+
+import numpy as np
+
+__all__ = [
+    "bf16_bits_to_f64",
+    "num_blocks",
+    "pool_keys",
+    "gate_scores",
+    "k_from_sparsity",
+    "k_from_budget",
+    "select_blocks",
+    "selection_margin",
+    "selection_is_valid",
+    "masked_attention",
+    "split_partials",
+    "combine",
+    "decode_row",
+]
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact bf16 -> float64: a bf16 value is the top 16 bits of a float32."""
+    u = np.asarray(bits).astype(np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def num_blocks(seqlen: int, block_size: int) -> int:
+    """NB = ceil(L / bs): the number of KV blocks of a sequence of length L
+    (the newest one possibly partial).  Block granularity: paper summary page,
+    Abstract ("large sparse attention block sizes (64/128)")."""
+    return -(-int(seqlen) // int(block_size))
+
+
+def pool_keys(K: np.ndarray, seqlen: int, block_size: int) -> np.ndarray:
+    """Mean-pooled block keys of one (sequence, KV head).
+
+    K: [>= seqlen][D] float64 key rows in token order.  Returns kbar [NB][D]
+    where kbar[j] is the plain mean of the valid rows t (t < seqlen) of block
+    j.  Only keys are pooled: the paper summary page's Abstract removes query
+    pooling for decoding, so the query enters the gate unpooled.
+    """
+    L = int(seqlen)
+    nb = num_blocks(L, block_size)
+    D = K.shape[1]
+    kbar = np.zeros((nb, D), dtype=np.float64)
+    for j in range(nb):
+        lo = j * block_size
+        hi = min(lo + block_size, L)
+        kbar[j] = K[lo:hi].sum(axis=0) / float(hi - lo)
+    return kbar
+
+
+def gate_scores(q_group: np.ndarray, W: np.ndarray, kbar: np.ndarray,
+                scale: float) -> np.ndarray:
+    """Gate score of every block for one KV head.
+
+    q_group: [G][D] the GQA group's decode queries; W: [D][D] this KV head's
+    gate projection (g = W q, row-major: g[i] = sum_j W[i][j] q[j]); kbar:
+    [NB][D].  Each query head scores block j as (W q).kbar[j]; the group's
+    score is the mean over its G heads, times ``scale`` (1/sqrt(D)).  Written
+    head by head and averaged last, deliberately not in the order a GPU would
+    use (average the queries first).
+    """
+    per_head = np.empty((q_group.shape[0], kbar.shape[0]), dtype=np.float64)
+    for g in range(q_group.shape[0]):
+        projected = W @ q_group[g]
+        per_head[g] = kbar @ projected
+    return per_head.mean(axis=0) * float(scale)
+
+
+def k_from_sparsity(nb: int, sparsity_permille: int) -> int:
+    """Blocks kept at a sparsity given in permille: the fraction (1 - s) of
+    the NB blocks, rounded up, at least one.  Agent Skill page, Step 1, keeps
+    "the top (1 - sparsity) fraction"; rounding up is the reading that gives
+    13 of 128 and 52 of 512 blocks at 90%."""
+    if not 0 <= sparsity_permille <= 1000:
+        raise ValueError("sparsity_permille must be within [0, 1000]")
+    kept = (1000 - int(sparsity_permille)) * int(nb)
+    return max(1, -(-kept // 1000))
+
+
+def k_from_budget(nb: int, budget_tokens: int, block_size: int) -> int:
+    """Blocks kept under a token budget (paper summary page, Abstract: a 4K
+    token budget): floor(budget / bs) whole blocks, capped at NB, at least
+    one."""
+    return max(1, min(int(nb), int(budget_tokens) // int(block_size)))
+
+
+def _rank_key(score: float, index: int):
+    """Sort key of a block: finite and infinite scores by value descending,
+    then NaN last; equal scores (with -0.0 == +0.0, which Python's == already
+    gives) by lower index first."""
+    if math.isnan(score):
+        return (1, 0.0, index)
+    return (0, -score, index)
+
+
+def select_blocks(scores: Sequence[float], k: int,
+                  force_newest: bool) -> np.ndarray:
+    """Top-k blocks of one KV head, returned in ascending block order.
+
+    scores: [NB] (the valid blocks only).  The newest block NB-1, when
+    forced, is taken first and counts toward k; the other k-1 (or k) places go
+    to the best remaining blocks under (score descending, index ascending).
+    Agent Skill page, Step 1 (top-k over importance scores); the tie rule and
+    the forced block come from the step specification.
+    """
+    s = [float(x) for x in np.asarray(scores, dtype=np.float64)]
+    nb = len(s)
+    k = min(int(k), nb)
+    taken = []
+    candidates = list(range(nb))
+    if force_newest and nb > 0 and k > 0:
+        taken.append(nb - 1)
+        candidates.remove(nb - 1)
+    candidates.sort(key=lambda j: _rank_key(s[j], j))
+    taken.extend(candidates[: max(0, k - len(taken))])
+    return np.array(sorted(taken), dtype=np.int64)
+
+
+def selection_margin(scores: Sequence[float], k: int,
+                     force_newest: bool) -> float:
+    """Gap between the last block taken on merit and the first one left out
+    (forced block excluded from the ranking).  +inf when nothing is left out
+    or nothing is chosen on merit.  Rows whose margin exceeds the gate
+    tolerance must select bit-identically on both sides."""
+    s = np.asarray(scores, dtype=np.float64)
+    nb = len(s)
+    k = min(int(k), nb)
+    pool = list(range(nb))
+    kk = k
+    if force_newest and nb > 0 and k > 0:
+        pool.remove(nb - 1)
+        kk -= 1
+    if kk <= 0 or kk >= len(pool):
+        return math.inf
+    ranked = sorted(pool, key=lambda j: _rank_key(float(s[j]), j))
+    a, b = float(s[ranked[kk - 1]]), float(s[ranked[kk]])
+    if math.isnan(a) or math.isnan(b):
+        return 0.0
+    return float(a - b)
+
+
+def selection_is_valid(scores: Sequence[float], chosen: Sequence[int], k: int,
+                       force_newest: bool, tol: float) -> bool:
+    """Whether an index list is a correct top-k up to ``tol``: right count,
+    ascending, unique, in range, forced block present, and every block chosen
+    on merit scores at least every block left out, minus ``tol``."""
+    s = np.asarray(scores, dtype=np.float64)
+    nb = len(s)
+    k = min(int(k), nb)
+    chosen = [int(c) for c in chosen]
+    if len(chosen) != k or chosen != sorted(set(chosen)):
+        return False
+    if any(c < 0 or c >= nb for c in chosen):
+        return False
+    merit = set(chosen)
+    if force_newest and k > 0:
+        if nb - 1 not in merit:
+            return False
+        merit.discard(nb - 1)
+    left_out = [j for j in range(nb) if j not in chosen]
+    if not merit or not left_out:
+        return True
+    def value(j):  # NaN ranks with -inf here: below every real score
+        return -math.inf if math.isnan(s[j]) else float(s[j])
+    worst_in = min(value(j) for j in merit)
+    best_out = max(value(j) for j in left_out)
+    return bool(worst_in >= best_out - tol)
+
+
+def masked_attention(q_group: np.ndarray, K: np.ndarray, V: np.ndarray,
+                     seqlen: int, blocks: Sequence[int], block_size: int,
+                     scale: float):
+    """Exact softmax attention of G decode queries over the selected blocks.
+
+    Agent Skill page, Step 4: scores = q.K^T * scale over all L cached keys,
+    every key outside the selected blocks (and every tail slot t >= L of a
+    partial block) set to -inf, softmax over keys, weights times V.  The
+    current token's K/V sits at position L-1 already, so no causal mask is
+    needed beyond t < L.  The weighted sum runs over the selected keys only:
+    every other weight is exactly zero, and skipping them keeps garbage (NaN)
+    in unselected or tail slots out of the result.
+
+    Returns (out [G][D], lse [G]) with lse the natural-log log-sum-exp of the
+    scaled scores; an empty selection gives (zeros, -inf).
+    """
+    L = int(seqlen)
+    G, D = q_group.shape
+    keep = np.zeros(L, dtype=bool)
+    for j in blocks:
+        lo = int(j) * block_size
+        keep[lo:min(lo + block_size, L)] = True
+    if not keep.any():
+        return np.zeros((G, V.shape[1])), np.full(G, -np.inf)
+    x = np.full((G, L), -np.inf, dtype=np.float64)
+    x[:, keep] = (q_group @ K[:L][keep].T) * float(scale)
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    total = e.sum(axis=1, keepdims=True)
+    p = e / total
+    out = p[:, keep] @ V[:L][keep]
+    lse = (m + np.log(total))[:, 0]
+    return out, lse
+
+
+def split_partials(q_group, K, V, seqlen, blocks, block_size, scale,
+                   num_splits: int):
+    """Split-KV partials: the ascending block list cut into ``num_splits``
+    contiguous pieces, piece s holding entries [floor(s*n/S), floor((s+1)*n/S)),
+    each attended on its own with ``masked_attention``.  An empty piece gives
+    o = 0 and lse = -inf.  Returns (o [S][G][D], lse [S][G])."""
+    blocks = list(int(b) for b in blocks)
+    n = len(blocks)
+    S = int(num_splits)
+    outs, lses = [], []
+    for s in range(S):
+        piece = blocks[(s * n) // S:((s + 1) * n) // S]
+        o, l = masked_attention(q_group, K, V, seqlen, piece, block_size, scale)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
+def combine(o_parts: np.ndarray, lse_parts: np.ndarray):
+    """Log-sum-exp merge of split partials (the step specification's combine).
+
+    o_parts: [S][G][D] per-piece normalised outputs; lse_parts: [S][G].  The
+    merged lse is log(sum_s exp(lse_s)); the output is sum_s exp(lse_s - lse)
+    * o_s.  Pieces with lse = -inf weigh nothing.
+    """
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    m = lse_parts.max(axis=0)
+    safe_m = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lse_parts - safe_m[None, :])
+    total = w.sum(axis=0)
+    lse = np.where(total > 0, safe_m + np.log(np.where(total > 0, total, 1.0)), -np.inf)
+    weights = np.where(total[None, :] > 0, w / np.where(total > 0, total, 1.0)[None, :], 0.0)
+    out = np.einsum("sg,sgd->gd", weights, np.asarray(o_parts, dtype=np.float64))
+    return out, lse
+
+
+def decode_row(q_group, W, K, V, seqlen, block_size, k, force_newest,
+               gate_scale, softmax_scale):
+    """The whole step for one (sequence, KV head): pool keys, gate scores,
+    top-k selection, then masked softmax attention of the G query heads over
+    the chosen blocks.  Returns a dict with kbar, scores, indices, out, lse."""
+    kbar = pool_keys(K, seqlen, block_size)
+    scores = gate_scores(q_group, W, kbar, gate_scale)
+    idx = select_blocks(scores, k, force_newest)
+    out, lse = masked_attention(q_group, K, V, seqlen, idx, block_size,
+                                softmax_scale)
+    return {"kbar": kbar, "scores": scores, "indices": idx, "out": out,
+            "lse": lse}

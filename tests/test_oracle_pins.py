@@ -1,0 +1,290 @@
+"""Pins of the fp64 oracle to things other than itself: hand-worked fixtures
+(tests/golden/), closed forms, invariants, brute force on tiny inputs and a
+library routine (torch's fp64 scaled_dot_product_attention on the CPU).
+CPU only."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import seer_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _f(x):
+    return float(x) if not isinstance(x, str) else float(x.replace("inf", "inf"))
+
+
+# ---------------------------------------------------------------- fixtures
+
+def test_attention_hand_cases():
+    for case in _load("attention_hand.json")["cases"]:
+        out, lse = O.masked_attention(np.array(case["q"], float), np.array(case["K"], float),
+                                      np.array(case["V"], float), case["seqlen"], case["blocks"],
+                                      case["block_size"], case["scale"])
+        np.testing.assert_allclose(out, np.array(case["out"], float), rtol=0, atol=1e-14,
+                                   err_msg=case["name"])
+        np.testing.assert_allclose(lse, np.array(case["lse"], float), rtol=0, atol=1e-14,
+                                   err_msg=case["name"])
+
+
+def test_gate_hand_case():
+    d = _load("gate_hand.json")
+    s = O.gate_scores(np.array(d["q"], float), np.array(d["W"], float),
+                      np.array(d["kbar"], float), d["scale"])
+    np.testing.assert_allclose(s, d["scores"], rtol=0, atol=1e-14)
+
+
+def test_pool_hand_case():
+    d = _load("pool_hand.json")
+    kbar = O.pool_keys(np.array(d["K"], float), d["seqlen"], d["block_size"])
+    np.testing.assert_array_equal(kbar, np.array(d["kbar"], float))
+
+
+def test_combine_hand_case():
+    d = _load("combine_hand.json")
+    lse = np.array([[_f(v) for v in row] for row in d["lse"]])
+    out, lse_out = O.combine(np.array(d["o"], float), lse)
+    np.testing.assert_allclose(out, d["out"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse_out, d["lse_out"], rtol=0, atol=1e-15)
+
+
+def test_k_rules():
+    d = _load("k_rules.json")
+    for c in d["sparsity"]:
+        assert O.k_from_sparsity(c["nb"], c["permille"]) == c["k"], c
+    for c in d["budget"]:
+        assert O.k_from_budget(c["nb"], c["budget"], c["block_size"]) == c["k"], c
+
+
+def test_select_hand_cases():
+    for c in _load("select_hand.json")["cases"]:
+        scores = [_f(v) for v in c["scores"]]
+        got = O.select_blocks(scores, c["k"], c["force_newest"]).tolist()
+        assert got == c["indices"], c
+
+
+# ---------------------------------------------------------------- selection
+
+def _beats(s, i, j):
+    """Block i outranks block j: higher score, or equal score and lower index;
+    NaN below everything, -0.0 == +0.0."""
+    a, b = s[i], s[j]
+    if math.isnan(a):
+        return math.isnan(b) and i < j
+    if math.isnan(b):
+        return True
+    return a > b or (a == b and i < j)
+
+
+def _brute_select(s, k, force):
+    """Exhaustive: the unique k-subset (holding the forced block) in which
+    every block chosen on merit outranks every block left out."""
+    nb = len(s)
+    k = min(k, nb)
+    found = []
+    for subset in itertools.combinations(range(nb), k):
+        if force and k > 0 and nb - 1 not in subset:
+            continue
+        merit = [i for i in subset if not (force and i == nb - 1)]
+        out = [j for j in range(nb) if j not in subset]
+        if all(_beats(s, i, j) for i in merit for j in out):
+            found.append(list(subset))
+    assert len(found) == 1, (s, k, force, found)
+    return found[0]
+
+
+def test_select_matches_brute_force_with_ties_and_specials():
+    rng = np.random.default_rng(7)
+    specials = [0.0, -0.0, -math.inf, math.inf, math.nan]
+    for trial in range(400):
+        nb = int(rng.integers(1, 9))
+        s = [float(v) for v in rng.integers(-2, 3, nb)]
+        for pos in range(nb):
+            if rng.random() < 0.2:
+                s[pos] = specials[int(rng.integers(0, len(specials)))]
+        k = int(rng.integers(1, nb + 2))
+        force = bool(rng.integers(0, 2))
+        got = O.select_blocks(s, k, force).tolist()
+        assert got == _brute_select(s, k, force), (s, k, force)
+        assert O.selection_is_valid(s, got, k, force, 0.0)
+
+
+def test_selection_margin_and_validity():
+    s = [0.5, 0.9, 0.1, 0.7]
+    assert O.selection_margin(s, 2, False) == pytest.approx(0.2)
+    assert O.selection_margin(s, 4, False) == math.inf
+    # forced newest (0.7) leaves 1 merit slot: 0.9 vs next 0.5
+    assert O.selection_margin(s, 2, True) == pytest.approx(0.4)
+    assert O.selection_is_valid(s, [1, 3], 2, False, 0.0)
+    assert not O.selection_is_valid(s, [0, 1], 2, False, 0.0)
+    assert O.selection_is_valid(s, [0, 1], 2, False, 0.25)
+    assert not O.selection_is_valid(s, [3, 1], 2, False, 0.0)   # not ascending
+    assert not O.selection_is_valid(s, [0, 1], 2, True, 1.0)    # forced block missing
+
+
+# ---------------------------------------------------------------- pooling and gate
+
+def test_pool_closed_forms():
+    rng = np.random.default_rng(1)
+    c = rng.standard_normal(16)
+    K = np.tile(c, (200, 1))
+    kbar = O.pool_keys(K, 200, 64)
+    assert kbar.shape == (4, 16)
+    np.testing.assert_allclose(kbar, np.tile(c, (4, 1)), rtol=1e-15, atol=1e-15)
+    # linear in K; every row of a block moved by the same vector moves the mean by it
+    K2 = rng.standard_normal((130, 16))
+    shift = rng.standard_normal(16)
+    a = O.pool_keys(K2, 130, 64)
+    b = O.pool_keys(K2 + shift, 130, 64)
+    np.testing.assert_allclose(b - a, np.tile(shift, (3, 1)), atol=1e-12)
+    # a single valid token in the newest block is its own mean
+    np.testing.assert_array_equal(a[2], K2[128:130].mean(axis=0))
+
+
+def test_gate_closed_forms():
+    D = 8
+    scale = 1 / math.sqrt(D)
+    eye = np.eye(D)
+    for i in range(D):
+        for j in range(D):
+            s = O.gate_scores(eye[i][None, :], eye, eye[j][None, :], scale)
+            assert s[0] == (scale if i == j else 0.0)
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((5, D))
+    W = rng.standard_normal((D, D))
+    kb = rng.standard_normal((9, D))
+    base = O.gate_scores(q, W, kb, scale)
+    np.testing.assert_allclose(O.gate_scores(2 * q, W, kb, scale), 2 * base, rtol=1e-13)
+    # the group score of G identical heads equals the single-head score
+    np.testing.assert_allclose(O.gate_scores(np.tile(q[:1], (4, 1)), W, kb, scale),
+                               O.gate_scores(q[:1], W, kb, scale), rtol=1e-13)
+    # permuting blocks permutes scores
+    perm = rng.permutation(9)
+    np.testing.assert_allclose(O.gate_scores(q, W, kb[perm], scale), base[perm], rtol=1e-13)
+
+
+# ---------------------------------------------------------------- attention
+
+def _sdpa_dense(q, K, V, scale):
+    """torch's fp64 CPU scaled_dot_product_attention: a library routine."""
+    out = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, :, None, :], torch.from_numpy(K)[None, None].expand(1, q.shape[0], -1, -1),
+        torch.from_numpy(V)[None, None].expand(1, q.shape[0], -1, -1), scale=scale)
+    return out[0, :, 0, :].numpy()
+
+
+@pytest.mark.parametrize("L,bs", [(200, 64), (256, 64), (300, 128), (1, 64), (65, 64)])
+def test_all_blocks_selected_equals_library_dense_attention(L, bs):
+    rng = np.random.default_rng(L)
+    G, D = 5, 32
+    q, K, V = rng.standard_normal((G, D)), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    nb = O.num_blocks(L, bs)
+    out, lse = O.masked_attention(q, K, V, L, range(nb), bs, 1 / math.sqrt(D))
+    np.testing.assert_allclose(out, _sdpa_dense(q, K, V, 1 / math.sqrt(D)), rtol=1e-12, atol=1e-13)
+    x = q @ K.T / math.sqrt(D)
+    from scipy.special import logsumexp
+    np.testing.assert_allclose(lse, logsumexp(x, axis=1), rtol=1e-13)
+
+
+def test_sparse_equals_library_attention_on_the_selected_rows():
+    rng = np.random.default_rng(11)
+    G, D, L, bs = 4, 16, 500, 64
+    q, K, V = rng.standard_normal((G, D)), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    blocks = [1, 4, 7]
+    rows = np.concatenate([np.arange(j * bs, min((j + 1) * bs, L)) for j in blocks])
+    out, _ = O.masked_attention(q, K, V, L, blocks, bs, 0.25)
+    np.testing.assert_allclose(out, _sdpa_dense(q, K[rows], V[rows], 0.25), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_closed_forms_and_invariants():
+    rng = np.random.default_rng(5)
+    G, D, L, bs = 3, 16, 1000, 64
+    q, K, V = rng.standard_normal((G, D)), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    blocks = [0, 3, 15]      # block 15 is partial: rows 960..999
+    # one selected token: output is that V row exactly
+    out, lse = O.masked_attention(q, K, V, 961, [15], bs, 0.3)
+    np.testing.assert_array_equal(out, np.tile(V[960], (G, 1)))
+    np.testing.assert_allclose(lse, q @ K[960] * 0.3, rtol=1e-15)
+    # q = 0: the plain mean of the selected rows
+    out, _ = O.masked_attention(np.zeros((G, D)), K, V, L, blocks, bs, 0.3)
+    rows = np.r_[0:64, 192:256, 960:1000]
+    np.testing.assert_allclose(out, np.tile(V[rows].mean(axis=0), (G, 1)), rtol=1e-12, atol=1e-14)
+    # constant V rows: output is that constant (weights sum to 1)
+    c = rng.standard_normal(D)
+    out, _ = O.masked_attention(q, K, np.tile(c, (L, 1)), L, blocks, bs, 0.3)
+    np.testing.assert_allclose(out, np.tile(c, (G, 1)), rtol=1e-12)
+    # one-hot V (V_t = e_{t mod D}): each output row is a probability vector
+    onehot = np.eye(D)[np.arange(L) % D]
+    out, _ = O.masked_attention(q, K, onehot, L, blocks, bs, 0.3)
+    np.testing.assert_allclose(out.sum(axis=1), 1.0, rtol=1e-13)
+    assert (out >= 0).all()
+    # unselected blocks and tail slots never matter, not even as NaN
+    base, base_lse = O.masked_attention(q, K, V, L - 7, blocks, bs, 0.3)
+    K2, V2 = K.copy(), V.copy()
+    for j in set(range(16)) - set(blocks):
+        K2[j * bs:(j + 1) * bs] = np.nan
+        V2[j * bs:(j + 1) * bs] = 1e30
+    K2[L - 7:] = np.nan
+    V2[L - 7:] = np.nan
+    out2, lse2 = O.masked_attention(q, K2, V2, L - 7, blocks, bs, 0.3)
+    np.testing.assert_array_equal(out2, base)
+    np.testing.assert_array_equal(lse2, base_lse)
+    # the order of the index list does not matter
+    out3, _ = O.masked_attention(q, K, V, L - 7, blocks[::-1], bs, 0.3)
+    np.testing.assert_array_equal(out3, base)
+
+
+@pytest.mark.parametrize("S", [1, 2, 3, 8, 13])
+def test_split_then_combine_equals_unsplit(S):
+    rng = np.random.default_rng(S)
+    G, D, L, bs = 4, 16, 777, 64
+    q, K, V = rng.standard_normal((G, D)), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    blocks = [0, 2, 5, 6, 9, 12]
+    o, l = O.split_partials(q, K, V, L, blocks, bs, 0.25, S)
+    assert o.shape == (S, G, D) and l.shape == (S, G)
+    if S > len(blocks):
+        assert np.isneginf(l).any()
+    out, lse = O.combine(o, l)
+    ref, ref_lse = O.masked_attention(q, K, V, L, blocks, bs, 0.25)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-13)
+    # the pieces are contiguous runs of the ascending list that cover it once
+    n = len(blocks)
+    pieces = [blocks[(s * n) // S:((s + 1) * n) // S] for s in range(S)]
+    assert sum(pieces, []) == blocks
+
+
+def test_decode_row_picks_planted_blocks():
+    """Compose pool -> gate -> select -> attention on a case built so that the
+    answer is known: blocks 2 and 5 carry keys along the gate direction."""
+    rng = np.random.default_rng(9)
+    G, D, bs, L = 2, 16, 8, 60
+    W = np.eye(D)
+    q = np.zeros((G, D)); q[:, 3] = 1.0
+    K = 0.01 * rng.standard_normal((L, D))
+    K[2 * bs:3 * bs, 3] += 2.0
+    K[5 * bs:6 * bs, 3] += 1.0
+    V = rng.standard_normal((L, D))
+    r = O.decode_row(q, W, K, V, L, bs, 2, False, 1 / math.sqrt(D), 1 / math.sqrt(D))
+    assert r["indices"].tolist() == [2, 5]
+    r = O.decode_row(q, W, K, V, L, bs, 2, True, 1 / math.sqrt(D), 1 / math.sqrt(D))
+    assert r["indices"].tolist() == [2, 7]     # newest block 7 (rows 56..59) forced
+    ref, _ = O.masked_attention(q, K, V, L, [2, 7], bs, 1 / math.sqrt(D))
+    np.testing.assert_array_equal(r["out"], ref)
+
+
+def test_bf16_conversion_is_exact():
+    x = torch.randn(1000).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(bits), x.double().numpy())
