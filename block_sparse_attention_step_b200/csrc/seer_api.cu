@@ -1,0 +1,407 @@
+// C ABI of libseer: argument checks, launch geometry, tensor maps and the
+// fused step.  Declared in include/seer.h.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <climits>
+#include <mutex>
+
+#include "seer_kernels.cuh"
+
+using namespace seer;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int num_sms_current() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < kMaxDevices) {
+    const int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Pool tensor map: dims (D, head, token, page) or (D, token, head, page),
+// whichever lists the smaller stride first; box = 64 dims x 64 tokens,
+// 128-byte swizzle (conflict-free ldmatrix rows).
+seer_status make_kv_map(const uint16_t* base, const seer_dims* d, int token_inner, CUtensorMap* map) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return SEER_ERR_CUDA;
+  cuuint64_t dims[4];
+  cuuint64_t strides[3];
+  cuuint32_t box[4];
+  const cuuint32_t elem[4] = {1, 1, 1, 1};
+  dims[0] = (cuuint64_t)d->head_dim;
+  box[0] = 64;
+  if (token_inner) {
+    dims[1] = (cuuint64_t)d->block_size;
+    dims[2] = (cuuint64_t)d->num_kv_heads;
+    strides[0] = (cuuint64_t)d->stride_token * 2;
+    strides[1] = (cuuint64_t)d->stride_head * 2;
+    box[1] = kTileTokens;
+    box[2] = 1;
+  } else {
+    dims[1] = (cuuint64_t)d->num_kv_heads;
+    dims[2] = (cuuint64_t)d->block_size;
+    strides[0] = (cuuint64_t)d->stride_head * 2;
+    strides[1] = (cuuint64_t)d->stride_token * 2;
+    box[1] = 1;
+    box[2] = kTileTokens;
+  }
+  dims[3] = (cuuint64_t)d->num_pages;
+  strides[2] = (cuuint64_t)d->stride_page * 2;
+  box[3] = 1;
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(base), dims,
+                         strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SEER_OK : SEER_ERR_UNSUPPORTED;
+}
+
+seer_status check_dims(const seer_dims* d) {
+  if (d == nullptr) return SEER_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1 || d->max_blocks < 1 ||
+      d->num_pages < 1)
+    return SEER_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return SEER_ERR_INVALID_ARG;
+  if (d->head_dim != kHeadDim) return SEER_ERR_UNSUPPORTED;
+  if (d->num_q_heads / d->num_kv_heads > kMaxGroup) return SEER_ERR_UNSUPPORTED;
+  if (d->block_size != 64 && d->block_size != 128) return SEER_ERR_UNSUPPORTED;
+  if (d->max_blocks > kMaxBlocks) return SEER_ERR_UNSUPPORTED;
+  if (d->batch > 65535 || d->num_kv_heads > 65535 || d->num_q_heads > 65535)
+    return SEER_ERR_UNSUPPORTED;
+  if (d->num_pages > INT_MAX) return SEER_ERR_UNSUPPORTED;
+  return SEER_OK;
+}
+
+seer_status check_pool(const seer_dims* d, const uint16_t* pool) {
+  if (pool == nullptr) return SEER_ERR_INVALID_ARG;
+  if (d->stride_page < 1 || d->stride_token < 1 || d->stride_head < 1) return SEER_ERR_INVALID_ARG;
+  if (!aligned(pool, 16) || d->stride_page % 8 || d->stride_token % 8 || d->stride_head % 8)
+    return SEER_ERR_UNSUPPORTED;
+  return SEER_OK;
+}
+
+#define SEER_TRY(expr)                     \
+  do {                                     \
+    const seer_status st_ = (expr);        \
+    if (st_ != SEER_OK) return st_;        \
+  } while (0)
+
+#define SEER_CUDA(expr)                               \
+  do {                                                \
+    if ((expr) != cudaSuccess) return SEER_ERR_CUDA;  \
+  } while (0)
+
+struct Workspace {
+  float* scores;
+  int32_t* idx;
+  int32_t* n_sel;
+  float* o_part;
+  float* lse_part;
+  size_t bytes;
+};
+
+Workspace carve(const seer_dims* d, int32_t k_max, int32_t S, void* base) {
+  const size_t bh = (size_t)d->batch * d->num_kv_heads;
+  const size_t bq = (size_t)d->batch * d->num_q_heads;
+  size_t off = 0;
+  Workspace w{};
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? static_cast<uint8_t*>(base) + off : nullptr;
+    off += round256(bytes);
+    return p;
+  };
+  w.scores = reinterpret_cast<float*>(take(bh * d->max_blocks * sizeof(float)));
+  w.idx = reinterpret_cast<int32_t*>(take(bh * k_max * sizeof(int32_t)));
+  w.n_sel = reinterpret_cast<int32_t*>(take(bh * sizeof(int32_t)));
+  w.o_part = reinterpret_cast<float*>(take(bq * S * kHeadDim * sizeof(float)));
+  w.lse_part = reinterpret_cast<float*>(take(bq * S * sizeof(float)));
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t seer_version(void) { return 10000; }
+
+const char* seer_status_string(seer_status s) {
+  switch (s) {
+    case SEER_OK: return "ok";
+    case SEER_ERR_INVALID_ARG: return "invalid argument";
+    case SEER_ERR_UNSUPPORTED: return "unsupported shape, layout or alignment";
+    case SEER_ERR_CUDA: return "CUDA error";
+    case SEER_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+seer_status seer_dims_default(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size, int32_t max_blocks,
+                              int64_t num_pages, seer_dims* out) {
+  if (out == nullptr) return SEER_ERR_INVALID_ARG;
+  seer_dims d;
+  d.batch = batch;
+  d.num_q_heads = num_q_heads;
+  d.num_kv_heads = num_kv_heads;
+  d.head_dim = head_dim;
+  d.block_size = block_size;
+  d.max_blocks = max_blocks;
+  d.num_pages = num_pages;
+  d.stride_head = head_dim;
+  d.stride_token = (int64_t)num_kv_heads * head_dim;
+  d.stride_page = (int64_t)block_size * num_kv_heads * head_dim;
+  SEER_TRY(check_dims(&d));
+  *out = d;
+  return SEER_OK;
+}
+
+seer_status seer_k_from_sparsity(int32_t nb, int32_t sparsity_permille, int32_t* k) {
+  if (k == nullptr || nb < 0 || sparsity_permille < 0 || sparsity_permille > 1000)
+    return SEER_ERR_INVALID_ARG;
+  const int64_t kept = ((int64_t)(1000 - sparsity_permille) * nb + 999) / 1000;
+  *k = (int32_t)(kept < 1 ? 1 : kept);
+  return SEER_OK;
+}
+
+seer_status seer_k_from_budget(int32_t nb, int32_t budget_tokens, int32_t block_size, int32_t* k) {
+  if (k == nullptr || nb < 0 || budget_tokens < 0 || block_size < 1) return SEER_ERR_INVALID_ARG;
+  int64_t v = budget_tokens / block_size;
+  if (v > nb) v = nb;
+  *k = (int32_t)(v < 1 ? 1 : v);
+  return SEER_OK;
+}
+
+seer_status seer_fill_k(const seer_dims* d, const int32_t* seqlens, int32_t sparsity_permille,
+                        int32_t budget_tokens, int32_t* k_per_seq, seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (!seqlens || !k_per_seq || budget_tokens < 0 || sparsity_permille < 0 ||
+      sparsity_permille > 1000)
+    return SEER_ERR_INVALID_ARG;
+  SEER_CUDA(run_fill_k(seqlens, d->batch, d->block_size, sparsity_permille, budget_tokens,
+                       k_per_seq, stream));
+  return SEER_OK;
+}
+
+int32_t seer_default_splits(const seer_dims* d, int32_t k_max, int32_t num_sms) {
+  if (check_dims(d) != SEER_OK || k_max < 1) return 1;
+  if (num_sms < 1) num_sms = num_sms_current();
+  const int64_t bh = (int64_t)d->batch * d->num_kv_heads;
+  int64_t s = (4 * (int64_t)num_sms + bh - 1) / bh;
+  int64_t cap = k_max / 2;
+  if (cap < 1) cap = 1;
+  if (cap > kMaxSplits) cap = kMaxSplits;
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  return (int32_t)s;
+}
+
+size_t seer_step_workspace_bytes(const seer_dims* d, int32_t k_max, int32_t num_splits) {
+  if (check_dims(d) != SEER_OK || k_max < 1 || num_splits < 1) return 0;
+  return carve(d, k_max, num_splits, nullptr).bytes;
+}
+
+seer_status seer_pool_keys(const seer_dims* d, const uint16_t* k_pool, const int32_t* page_table,
+                           const int32_t* seqlens, int32_t incremental, float* kbar,
+                           int32_t* dev_status, seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  SEER_TRY(check_pool(d, k_pool));
+  if (!seqlens || !kbar || (incremental != 0 && incremental != 1)) return SEER_ERR_INVALID_ARG;
+  if (!aligned(kbar, 16)) return SEER_ERR_UNSUPPORTED;
+  PoolParams p;
+  p.k_pool = k_pool;
+  p.page_table = page_table;
+  p.seqlens = seqlens;
+  p.kbar = kbar;
+  p.status = dev_status;
+  p.Hkv = d->num_kv_heads;
+  p.bs = d->block_size;
+  p.max_blocks = d->max_blocks;
+  p.incremental = incremental;
+  p.num_pages = d->num_pages;
+  p.stride_page = d->stride_page;
+  p.stride_token = d->stride_token;
+  p.stride_head = d->stride_head;
+  SEER_CUDA(run_pool_keys(p, d->batch, stream));
+  return SEER_OK;
+}
+
+seer_status seer_gate_scores(const seer_dims* d, const uint16_t* q, const float* w_gate,
+                             const float* kbar, const int32_t* seqlens, float gate_scale,
+                             float* scores, int32_t* dev_status, seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (!q || !w_gate || !kbar || !seqlens || !scores) return SEER_ERR_INVALID_ARG;
+  if (!aligned(w_gate, 16) || !aligned(kbar, 16) || !aligned(q, 4)) return SEER_ERR_UNSUPPORTED;
+  GateParams p;
+  p.q = q;
+  p.w_gate = w_gate;
+  p.kbar = kbar;
+  p.seqlens = seqlens;
+  p.scores = scores;
+  p.status = dev_status;
+  p.Hq = d->num_q_heads;
+  p.Hkv = d->num_kv_heads;
+  p.G = d->num_q_heads / d->num_kv_heads;
+  p.bs = d->block_size;
+  p.max_blocks = d->max_blocks;
+  p.gate_scale = gate_scale;
+  // about two CTAs per SM, each with a whole number of 32-row sweeps
+  const int64_t bh = (int64_t)d->batch * d->num_kv_heads;
+  int64_t chunks = (2 * (int64_t)num_sms_current() + bh - 1) / bh;
+  if (chunks < 1) chunks = 1;
+  int64_t per = (d->max_blocks + chunks - 1) / chunks;
+  per = ((per + 31) / 32) * 32;
+  p.blocks_per_cta = (int)per;
+  SEER_CUDA(run_gate_scores(p, d->batch, stream));
+  return SEER_OK;
+}
+
+seer_status seer_block_select(const seer_dims* d, const float* scores, const int32_t* seqlens,
+                              const int32_t* k_per_seq, int32_t force_newest, int32_t k_max,
+                              int32_t* idx, int32_t* n_sel, int32_t* dev_status,
+                              seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (!scores || !seqlens || !k_per_seq || !idx || !n_sel) return SEER_ERR_INVALID_ARG;
+  if (k_max < 1 || k_max > d->max_blocks) return SEER_ERR_INVALID_ARG;
+  SelectParams p;
+  p.scores = scores;
+  p.seqlens = seqlens;
+  p.k_per_seq = k_per_seq;
+  p.idx = idx;
+  p.n_sel = n_sel;
+  p.status = dev_status;
+  p.Hkv = d->num_kv_heads;
+  p.bs = d->block_size;
+  p.max_blocks = d->max_blocks;
+  p.k_max = k_max;
+  p.force_newest = force_newest ? 1 : 0;
+  SEER_CUDA(run_block_select(p, d->batch, stream));
+  return SEER_OK;
+}
+
+seer_status seer_sparse_decode(const seer_dims* d, const uint16_t* q, const uint16_t* k_pool,
+                               const uint16_t* v_pool, const int32_t* page_table,
+                               const int32_t* seqlens, const int32_t* idx, const int32_t* n_sel,
+                               int32_t k_max, int32_t num_splits, float softmax_scale,
+                               float* o_part, float* lse_part, int32_t* dev_status,
+                               seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  SEER_TRY(check_pool(d, k_pool));
+  SEER_TRY(check_pool(d, v_pool));
+  if (!q || !seqlens || !idx || !n_sel || !o_part || !lse_part) return SEER_ERR_INVALID_ARG;
+  if (k_max < 1 || k_max > d->max_blocks || num_splits < 1 || num_splits > kMaxSplits)
+    return SEER_ERR_INVALID_ARG;
+  if (!aligned(q, 4) || !aligned(o_part, 8)) return SEER_ERR_UNSUPPORTED;
+  const int64_t items = (int64_t)d->batch * d->num_kv_heads * num_splits;
+  if (items > INT_MAX) return SEER_ERR_UNSUPPORTED;
+  const int token_inner = d->stride_token < d->stride_head ? 1 : 0;
+  CUtensorMap tk, tv;
+  SEER_TRY(make_kv_map(k_pool, d, token_inner, &tk));
+  SEER_TRY(make_kv_map(v_pool, d, token_inner, &tv));
+  DecodeParams p;
+  p.q = q;
+  p.page_table = page_table;
+  p.seqlens = seqlens;
+  p.idx = idx;
+  p.n_sel = n_sel;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.status = dev_status;
+  p.B = d->batch;
+  p.Hq = d->num_q_heads;
+  p.Hkv = d->num_kv_heads;
+  p.G = d->num_q_heads / d->num_kv_heads;
+  p.bs = d->block_size;
+  p.max_blocks = d->max_blocks;
+  p.k_max = k_max;
+  p.S = num_splits;
+  p.num_items = (int)items;
+  p.token_inner = token_inner;
+  p.num_pages = d->num_pages;
+  p.scale_log2 = softmax_scale * kLog2e;
+  SEER_CUDA(run_sparse_decode(tk, tv, p, num_sms_current(), stream));
+  return SEER_OK;
+}
+
+seer_status seer_combine(const seer_dims* d, const float* o_part, const float* lse_part,
+                         int32_t num_splits, uint16_t* out, float* lse_out, seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (!o_part || !lse_part || !out) return SEER_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > kMaxSplits) return SEER_ERR_INVALID_ARG;
+  CombineParams p;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.out = out;
+  p.lse_out = lse_out;
+  p.S = num_splits;
+  SEER_CUDA(run_combine(p, d->batch, d->num_q_heads, stream));
+  return SEER_OK;
+}
+
+seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (a == nullptr || a->k_per_seq == nullptr || a->kbar == nullptr) return SEER_ERR_INVALID_ARG;
+  if (a->update_kbar < 0 || a->update_kbar > 2) return SEER_ERR_INVALID_ARG;
+  if (a->k_max < 1 || a->num_splits < 1) return SEER_ERR_INVALID_ARG;
+  if (a->workspace == nullptr || !aligned(a->workspace, 256)) return SEER_ERR_WORKSPACE;
+  const Workspace w = carve(d, a->k_max, a->num_splits, a->workspace);
+  if (a->workspace_bytes < w.bytes) return SEER_ERR_WORKSPACE;
+  if (a->update_kbar)
+    SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, a->update_kbar == 1 ? 1 : 0,
+                            a->kbar, a->dev_status, stream));
+  SEER_TRY(seer_gate_scores(d, a->q, a->w_gate, a->kbar, a->seqlens, a->gate_scale, w.scores,
+                            a->dev_status, stream));
+  SEER_TRY(seer_block_select(d, w.scores, a->seqlens, a->k_per_seq, a->force_newest, a->k_max,
+                             w.idx, w.n_sel, a->dev_status, stream));
+  SEER_TRY(seer_sparse_decode(d, a->q, a->k_pool, a->v_pool, a->page_table, a->seqlens, w.idx,
+                              w.n_sel, a->k_max, a->num_splits, a->softmax_scale, w.o_part,
+                              w.lse_part, a->dev_status, stream));
+  SEER_TRY(seer_combine(d, w.o_part, w.lse_part, a->num_splits, a->out, a->lse_out, stream));
+  return SEER_OK;
+}
+
+seer_status seer_decode_step_host(const seer_dims* d, const seer_step_args* a,
+                                  const uint16_t* q_host, uint16_t* q_dev, uint16_t* out_host,
+                                  seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (a == nullptr || q_host == nullptr || q_dev == nullptr || out_host == nullptr ||
+      a->out == nullptr)
+    return SEER_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)d->batch * d->num_q_heads * d->head_dim * sizeof(uint16_t);
+  SEER_CUDA(cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, stream));
+  seer_step_args b = *a;
+  b.q = q_dev;
+  SEER_TRY(seer_decode_step(d, &b, stream));
+  SEER_CUDA(cudaMemcpyAsync(out_host, a->out, bytes, cudaMemcpyDeviceToHost, stream));
+  return SEER_OK;
+}
+
+}  // extern "C"

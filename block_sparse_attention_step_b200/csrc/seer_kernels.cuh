@@ -1,0 +1,72 @@
+// Parameter blocks and launchers of the libseer kernels (internal).
+#pragma once
+
+#include "seer_common.cuh"
+
+namespace seer {
+
+struct PoolParams {
+  const uint16_t* k_pool;
+  const int32_t* page_table;
+  const int32_t* seqlens;
+  float* kbar;
+  int32_t* status;
+  int Hkv, bs, max_blocks, incremental;
+  int64_t num_pages, stride_page, stride_token, stride_head;
+};
+
+struct GateParams {
+  const uint16_t* q;
+  const float* w_gate;
+  const float* kbar;
+  const int32_t* seqlens;
+  float* scores;
+  int32_t* status;
+  int Hq, Hkv, G, bs, max_blocks, blocks_per_cta;
+  float gate_scale;
+};
+
+struct SelectParams {
+  const float* scores;
+  const int32_t* seqlens;
+  const int32_t* k_per_seq;
+  int32_t* idx;
+  int32_t* n_sel;
+  int32_t* status;
+  int Hkv, bs, max_blocks, k_max, force_newest;
+};
+
+struct DecodeParams {
+  const uint16_t* q;
+  const int32_t* page_table;
+  const int32_t* seqlens;
+  const int32_t* idx;
+  const int32_t* n_sel;
+  float* o_part;
+  float* lse_part;
+  int32_t* status;
+  int B, Hq, Hkv, G, bs, max_blocks, k_max, S;
+  int num_items;
+  int token_inner;  // tensor map dims are (D, token, head, page), not (D, head, token, page)
+  int64_t num_pages;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+struct CombineParams {
+  const float* o_part;
+  const float* lse_part;
+  uint16_t* out;
+  float* lse_out;
+  int S;
+};
+
+cudaError_t run_pool_keys(const PoolParams& p, int B, cudaStream_t stream);
+cudaError_t run_gate_scores(const GateParams& p, int B, cudaStream_t stream);
+cudaError_t run_block_select(const SelectParams& p, int B, cudaStream_t stream);
+cudaError_t run_fill_k(const int32_t* seqlens, int B, int bs, int permille, int budget,
+                       int32_t* k_out, cudaStream_t stream);
+cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                              int num_sms, cudaStream_t stream);
+cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream);
+
+}  // namespace seer

@@ -1,0 +1,90 @@
+"""Device buffers for one decode step over a drawn workload (plumbing only).
+
+``StepBuffers`` owns the torch allocations a caller of ``seer_decode_step``
+needs besides the inputs (pooled keys, k per sequence, workspace, output,
+status word) and issues the C-ABI calls through the ctypes binding.  Every
+number it produces comes from the library's kernels.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import seer
+
+
+class StepBuffers:
+    def __init__(self, w, data: dict, num_splits: Optional[int] = None,
+                 sparsity_permille: Optional[int] = None, budget_tokens: Optional[int] = None,
+                 force_newest: Optional[bool] = None, k_max: Optional[int] = None,
+                 device: Optional[torch.device] = None):
+        self.w = w
+        self.data = data
+        dev = device or data["q"].device
+        self.device = dev
+        B, Hkv, D = w.batch, w.kv_heads, w.head_dim
+        self.nb_max = data["nb_max"]
+        self.dims = seer.make_dims(B, w.q_heads, Hkv, D, w.block_size, self.nb_max,
+                                   data["num_pages"])
+        self.budget = w.budget_tokens if budget_tokens is None else budget_tokens
+        self.permille = w.sparsity_permille if sparsity_permille is None else sparsity_permille
+        if self.budget is None and self.permille is None:
+            raise ValueError("workload has neither a budget nor a sparsity")
+        self.force_newest = w.force_newest if force_newest is None else force_newest
+        self.k_per_seq = torch.empty(B, dtype=torch.int32, device=dev)
+        seer.seer_fill_k(self.dims, data["seqlens"], self.permille or 0, self.budget or 0,
+                         self.k_per_seq)
+        self.k_max = int(k_max) if k_max is not None else int(self.k_per_seq.max().item())
+        self.k_max = max(1, min(self.k_max, self.nb_max))
+        if num_splits is None:
+            num_splits = w.num_splits or seer.seer_default_splits(self.dims, self.k_max, 0)
+        self.num_splits = int(num_splits)
+        self.kbar = torch.empty((B, Hkv, self.nb_max, D), dtype=torch.float32, device=dev)
+        ws = seer.seer_step_workspace_bytes(self.dims, self.k_max, self.num_splits)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.out = torch.empty((B, w.q_heads, D), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, w.q_heads), dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.scale = 1.0 / math.sqrt(D)
+
+    # views into the workspace, in the order the library carves it
+    def workspace_views(self):
+        B, Hkv, Hq, S, D = self.w.batch, self.w.kv_heads, self.w.q_heads, self.num_splits, self.w.head_dim
+
+        def r256(x):
+            return (x + 255) // 256 * 256
+        off = 0
+        out = {}
+        for name, n, dt in (("scores", B * Hkv * self.nb_max, torch.float32),
+                            ("idx", B * Hkv * self.k_max, torch.int32),
+                            ("n_sel", B * Hkv, torch.int32),
+                            ("o_part", B * Hq * S * D, torch.float32),
+                            ("lse_part", B * Hq * S, torch.float32)):
+            nbytes = n * 4
+            out[name] = self.workspace[off:off + nbytes].view(dt)
+            off += r256(nbytes)
+        out["scores"] = out["scores"].view(B, Hkv, self.nb_max)
+        out["idx"] = out["idx"].view(B, Hkv, self.k_max)
+        out["n_sel"] = out["n_sel"].view(B, Hkv)
+        out["o_part"] = out["o_part"].view(B, Hq, S, D)
+        out["lse_part"] = out["lse_part"].view(B, Hq, S)
+        return out
+
+    def pool_full(self, stream=None):
+        d = self.data
+        seer.seer_pool_keys(self.dims, d["k_pool"], d["page_table"], d["seqlens"], 0, self.kbar,
+                            self.status, stream)
+
+    def args(self, update_kbar: int = 0, q=None) -> "seer.seer_step_args":
+        d = self.data
+        return seer.step_args(d["q"] if q is None else q, d["k_pool"], d["v_pool"], d["page_table"],
+                              d["seqlens"], d["w_gate"], self.kbar, self.k_per_seq,
+                              update_kbar=update_kbar, force_newest=self.force_newest,
+                              k_max=self.k_max, num_splits=self.num_splits, gate_scale=self.scale,
+                              softmax_scale=self.scale, workspace=self.workspace, out=self.out,
+                              lse_out=self.lse, dev_status=self.status)
+
+    def step(self, update_kbar: int = 0, stream=None, args=None):
+        seer.seer_decode_step(self.dims, args if args is not None else self.args(update_kbar), stream)

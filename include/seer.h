@@ -1,0 +1,248 @@
+/*
+ * seer.h -- C ABI of the block-sparse decode attention step (SeerAttention-R)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What the step computes (one decode token per sequence, one attention layer):
+ *
+ *   kbar[b,h,j]  = mean of the keys of block j of sequence b, KV head h
+ *   g[b,h]       = W[h] . mean over the GQA group's query heads of q
+ *   score[b,h,j] = gate_scale * g[b,h] . kbar[b,h,j]
+ *   idx[b,h,:]   = the top-k blocks by score (ties to the lower block index,
+ *                  the newest block optionally forced in), ascending
+ *   out[b,qh]    = softmax(q[b,qh] . K^T * softmax_scale) V over the tokens of
+ *                  the selected blocks only (t < seqlen), computed as S
+ *                  split-KV partials merged by a log-sum-exp combine.
+ *
+ * Sources, by page and section:
+ *   - "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning",
+ *     Abstract: a self-distilled gate chooses KV blocks for each decode query,
+ *     query pooling removed for decoding, block sizes 64/128, a 4K-token
+ *     budget, a sparse decoding kernel run at 90% sparsity behind a
+ *     FlashAttention-style interface (paged cache, cache_seqlens, num_splits,
+ *     softmax_scale, out + lse).
+ *   - "Sparse Attention Reasoning" (Agent Skill page), Step 1: top-k over gate
+ *     scores, k from a sparsity ratio; Step 4: sparse attention is softmax
+ *     attention with unselected keys filled with -inf, scale 1/sqrt(head_dim).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_host are host memory; every other pointer is device
+ *     memory on the current device.  The caller owns every buffer; the library
+ *     never allocates, frees or synchronises, and keeps no state between calls
+ *     (it caches one driver entry point on first use).
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Host-side checks return an error before anything is enqueued.
+ *     SEER_ERR_CUDA reports a launch error (cudaGetLastError()).
+ *   - Conditions only the device can see are OR-ed into the optional
+ *     `dev_status` word (device int32, may be NULL): see SEER_DEV_*.
+ *     Kernels never trap, assert or spin without a bound.
+ *
+ * Shapes (row-major, innermost last):
+ *   q          [B][Hq][D] bf16; query head qh belongs to KV head qh / (Hq/Hkv)
+ *   k_pool,
+ *   v_pool     [num_pages][block_size][Hkv][D] bf16 by default, or any layout
+ *              given by (stride_page, stride_token, stride_head) in elements
+ *              with the D elements of one row contiguous; all strides and the
+ *              base address 16-byte aligned.  One page holds one KV block.
+ *   page_table [B][max_blocks] int32: page of logical block j of sequence b;
+ *              may be NULL for the identity table page = b * max_blocks + j
+ *              (a contiguous [B][max_blocks * block_size][Hkv][D] cache).
+ *              Entries at j >= NB_b are never read.
+ *   seqlens    [B] int32: tokens in the cache, the current token's K/V
+ *              already appended at position seqlen - 1; 0 <= seqlen <=
+ *              max_blocks * block_size.  NB_b = ceil(seqlen_b / block_size).
+ *   w_gate     [Hkv][D][D] fp32, g[i] = sum_j W[h][i][j] qbar[j]
+ *   kbar       [B][Hkv][max_blocks][D] fp32
+ *   scores     [B][Hkv][max_blocks] fp32 (-inf at j >= NB_b)
+ *   idx        [B][Hkv][k_max] int32, ascending, -1 after the n_sel entries
+ *   n_sel      [B][Hkv] int32
+ *   o_part     [B][Hq][num_splits][D] fp32, lse_part [B][Hq][num_splits] fp32
+ *   out        [B][Hq][D] bf16 (round-to-nearest-even), lse_out [B][Hq] fp32
+ *              natural-log log-sum-exp of the scaled scores (-inf if empty)
+ */
+#ifndef SEER_H_
+#define SEER_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SEER_API __attribute__((visibility("default")))
+#else
+#define SEER_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *seer_stream;
+
+typedef enum seer_status {
+  SEER_OK = 0,
+  SEER_ERR_INVALID_ARG = 1, /* null pointer, negative or inconsistent size */
+  SEER_ERR_UNSUPPORTED = 2, /* D != 128, block_size not 64/128, Hq/Hkv > 16,
+                               misaligned pointer or stride, too many blocks */
+  SEER_ERR_CUDA = 3,        /* a CUDA call or kernel launch failed */
+  SEER_ERR_WORKSPACE = 4    /* workspace missing or smaller than required */
+} seer_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define SEER_DEV_NONFINITE_SCORE 1 /* a gate score was NaN or +-inf */
+#define SEER_DEV_BAD_INDEX 2       /* an idx entry outside [0, NB_b): skipped */
+#define SEER_DEV_BAD_PAGE 4        /* page outside [0, num_pages): page 0 used */
+#define SEER_DEV_K_CLAMPED 8       /* k_per_seq[b] > k_max: clamped to k_max */
+#define SEER_DEV_TIMEOUT 16        /* a pipeline wait gave up after ~1 s */
+
+typedef struct seer_dims {
+  int32_t batch;        /* B >= 1 */
+  int32_t num_q_heads;  /* Hq, a multiple of Hkv, Hq / Hkv <= 16 */
+  int32_t num_kv_heads; /* Hkv >= 1 */
+  int32_t head_dim;     /* D, must be 128 */
+  int32_t block_size;   /* bs, 64 or 128; equal to the page size */
+  int32_t max_blocks;   /* NBmax >= 1: row length of page_table, kbar, scores;
+                           at most 4096 */
+  int64_t num_pages;    /* pages in each pool (>= B * NBmax if table NULL) */
+  int64_t stride_page;  /* element strides of k_pool and v_pool */
+  int64_t stride_token;
+  int64_t stride_head;
+} seer_dims;
+
+/* Library version, as 10000 * major + 100 * minor + patch. */
+SEER_API int32_t seer_version(void);
+
+/* Static text for a status code. */
+SEER_API const char *seer_status_string(seer_status s);
+
+/* Fill a seer_dims for the default pool layout [P][bs][Hkv][D]. */
+SEER_API seer_status seer_dims_default(int32_t batch, int32_t num_q_heads,
+                              int32_t num_kv_heads, int32_t head_dim,
+                              int32_t block_size, int32_t max_blocks,
+                              int64_t num_pages, seer_dims *out);
+
+/* ---------------------------------------------------------------- helpers
+ * k from a sparsity in permille (0..1000): max(1, ceil((1000 - s) * nb / 1000))
+ * -- "keep the top (1 - sparsity) fraction" (Agent Skill page, Step 1),
+ * rounded up.  k from a token budget: max(1, min(nb, budget / block_size))
+ * (paper summary page, Abstract: 4K token budget).  Both in exact integers. */
+SEER_API seer_status seer_k_from_sparsity(int32_t nb, int32_t sparsity_permille,
+                                 int32_t *k);
+SEER_API seer_status seer_k_from_budget(int32_t nb, int32_t budget_tokens,
+                               int32_t block_size, int32_t *k);
+
+/* Device version of the two rules above, one k per sequence from seqlens:
+ * budget mode when budget_tokens > 0, else sparsity mode. */
+SEER_API seer_status seer_fill_k(const seer_dims *d, const int32_t *seqlens,
+                        int32_t sparsity_permille, int32_t budget_tokens,
+                        int32_t *k_per_seq, seer_stream stream);
+
+/* Splits that keep every SM busy for k_max selected blocks per KV head:
+ * enough (b, h, split) items for about four per SM, at least 2 blocks per
+ * split, between 1 and 64. */
+SEER_API int32_t seer_default_splits(const seer_dims *d, int32_t k_max,
+                            int32_t num_sms);
+
+/* Bytes of caller workspace seer_decode_step needs (scores, idx, n_sel,
+ * o_part and lse_part, each 256-byte aligned). */
+SEER_API size_t seer_step_workspace_bytes(const seer_dims *d, int32_t k_max,
+                                 int32_t num_splits);
+
+/* ------------------------------------------------------------- the steps */
+
+/* a0. Mean-pooled block keys.  incremental = 0 rebuilds every block (blocks
+ * j >= NB_b are written as zeros); incremental = 1 recomputes only the
+ * newest block NB_b - 1 of every (b, h), the one the appended token changed.
+ * Pooling keys but not queries follows the Abstract ("removing query
+ * pooling").  fp32 sums in a fixed order. */
+SEER_API seer_status seer_pool_keys(const seer_dims *d, const uint16_t *k_pool,
+                           const int32_t *page_table, const int32_t *seqlens,
+                           int32_t incremental, float *kbar,
+                           int32_t *dev_status, seer_stream stream);
+
+/* a1. Gate scores, fp32: score[b,h,j] = gate_scale * (W[h] qbar) . kbar[j]
+ * with qbar the mean of the G query heads of KV head h (the mean of the
+ * per-head scores, by linearity).  j >= NB_b gets -inf.  Non-finite scores
+ * of valid blocks set SEER_DEV_NONFINITE_SCORE. */
+SEER_API seer_status seer_gate_scores(const seer_dims *d, const uint16_t *q,
+                             const float *w_gate, const float *kbar,
+                             const int32_t *seqlens, float gate_scale,
+                             float *scores, int32_t *dev_status,
+                             seer_stream stream);
+
+/* a2. Top-k block selection per (b, h) (Agent Skill page, Step 1).  k_b =
+ * k_per_seq[b] (values < 1 count as 1, values > k_max are clamped and flag
+ * SEER_DEV_K_CLAMPED), n_sel = min(k_b, NB_b).  Order: score descending,
+ * then lower index; NaN below -inf; -0.0 == +0.0.  force_newest != 0 takes
+ * block NB_b - 1 first, counting toward k.  idx rows are ascending and padded
+ * with -1 to k_max.  Exact: the result depends only on the scores. */
+SEER_API seer_status seer_block_select(const seer_dims *d, const float *scores,
+                              const int32_t *seqlens,
+                              const int32_t *k_per_seq, int32_t force_newest,
+                              int32_t k_max, int32_t *idx, int32_t *n_sel,
+                              int32_t *dev_status, seer_stream stream);
+
+/* a3. Split-KV sparse flash-decoding (Agent Skill page, Step 4: masked
+ * softmax attention, scale softmax_scale).  For each (b, h, split s) the
+ * selected blocks idx[b,h, floor(s*n/S) .. floor((s+1)*n/S)) are staged by
+ * TMA into shared memory; all G query heads of the group attend them with an
+ * online softmax, so each K/V byte is read from HBM once.  Tokens t >=
+ * seqlen_b never enter the math; unselected blocks are never read.  Writes
+ * o_part (normalised per split) and lse_part (natural log); an empty split
+ * writes o = 0, lse = -inf.  1 <= num_splits <= 64. */
+SEER_API seer_status seer_sparse_decode(const seer_dims *d, const uint16_t *q,
+                               const uint16_t *k_pool, const uint16_t *v_pool,
+                               const int32_t *page_table,
+                               const int32_t *seqlens, const int32_t *idx,
+                               const int32_t *n_sel, int32_t k_max,
+                               int32_t num_splits, float softmax_scale,
+                               float *o_part, float *lse_part,
+                               int32_t *dev_status, seer_stream stream);
+
+/* a4. Log-sum-exp combine of the split partials: lse = log sum_s e^{lse_s},
+ * out = sum_s e^{lse_s - lse} o_s, rounded to bf16.  lse_out may be NULL. */
+SEER_API seer_status seer_combine(const seer_dims *d, const float *o_part,
+                         const float *lse_part, int32_t num_splits,
+                         uint16_t *out, float *lse_out, seer_stream stream);
+
+/* The whole step, a0 (optional) .. a4, enqueued back to back on `stream`.
+ * Needs no host synchronisation and can be captured in a CUDA graph. */
+typedef struct seer_step_args {
+  const uint16_t *q;
+  const uint16_t *k_pool;
+  const uint16_t *v_pool;
+  const int32_t *page_table; /* may be NULL (identity) */
+  const int32_t *seqlens;
+  const float *w_gate;
+  float *kbar;               /* read by the gate; written when update_kbar */
+  const int32_t *k_per_seq;
+  int32_t update_kbar;       /* 0: use kbar as is, 1: incremental, 2: full */
+  int32_t force_newest;
+  int32_t k_max;
+  int32_t num_splits;
+  float gate_scale;          /* 1/sqrt(D) */
+  float softmax_scale;       /* 1/sqrt(D) */
+  void *workspace;           /* seer_step_workspace_bytes() bytes, 256-aligned */
+  size_t workspace_bytes;
+  uint16_t *out;
+  float *lse_out;            /* may be NULL */
+  int32_t *dev_status;       /* may be NULL */
+} seer_step_args;
+
+SEER_API seer_status seer_decode_step(const seer_dims *d, const seer_step_args *a,
+                             seer_stream stream);
+
+/* End-to-end form for callers holding q and out in host memory: enqueues the
+ * copy q_host -> q_dev (B*Hq*D bf16), the step with a->q replaced by q_dev,
+ * and the copy a->out -> out_host.  Asynchronous: with pinned host buffers
+ * the copies overlap nothing else on `stream`, and out_host is valid after
+ * the stream is synchronised. */
+SEER_API seer_status seer_decode_step_host(const seer_dims *d, const seer_step_args *a,
+                                  const uint16_t *q_host, uint16_t *q_dev,
+                                  uint16_t *out_host, seer_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEER_H_ */

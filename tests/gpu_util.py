@@ -1,0 +1,59 @@
+"""Shared helpers of the GPU parity tests: copying seeded inputs to the host
+as float64 for the oracle, and the comparison measures with their bounds."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_step_b200 import workloads as W
+
+# Output tolerance of the step against the fp64 oracle (max-abs, rel-L2).
+TOL_MAX_ABS = 2e-2
+TOL_REL_L2 = 1e-2
+# Gate scores closer than this (fp64 margin at the k/k+1 boundary) may
+# legitimately select differently in fp32; such rows get a validity check.
+MARGIN = 1e-4
+
+
+def require_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from block_sparse_attention_step_b200 import seer
+    seer.library()  # raises if the library is missing: no fallback
+    major, minor = torch.cuda.get_device_capability()
+    if (major, minor) != (10, 0):
+        pytest.skip(f"built for sm_100a, device is sm_{major}{minor}")
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").double().numpy()
+
+
+def row_inputs(w, data, b, h):
+    """(q_group [G][D], W [D][D], K [L][D], V [L][D], L) as float64 on the host."""
+    L = int(data["seqlens"][b].item())
+    G = w.group
+    q = f64(data["q"][b, h * G:(h + 1) * G])
+    Wg = f64(data["w_gate"][h])
+    K = f64(W.gather_rows(data["k_pool"], data["page_table"], b, h, L, w.block_size))
+    V = f64(W.gather_rows(data["v_pool"], data["page_table"], b, h, L, w.block_size))
+    return q, Wg, K, V, L
+
+
+def out_errors(got: np.ndarray, ref: np.ndarray):
+    err = got - ref
+    max_abs = float(np.abs(err).max()) if err.size else 0.0
+    denom = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(err) / denom) if denom > 0 else float(np.linalg.norm(err))
+    return max_abs, rel
+
+
+def assert_out_close(got, ref, what=""):
+    max_abs, rel = out_errors(got, ref)
+    assert max_abs <= TOL_MAX_ABS and rel <= TOL_REL_L2, (what, max_abs, rel)
+    return max_abs, rel
+
+
+def scale_of(w):
+    return 1.0 / math.sqrt(w.head_dim)

@@ -1,0 +1,210 @@
+"""End-to-end parity of the fused step (pool -> gate -> select -> sparse
+decode -> combine) against the fp64 oracle: indices bit-exact on every
+(b, h) row whose fp64 gate margin exceeds 1e-4 (validity within 1e-4 on the
+others), outputs within max-abs 2e-2 / rel-L2 1e-2 of the oracle run on the
+GPU's own index set.  Small versions of all five workloads, then the full
+sizes in the launch configuration the benchmark times, checked on sampled
+(b, h) rows."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_step_b200 import seer
+from block_sparse_attention_step_b200 import workloads as W
+from block_sparse_attention_step_b200.runner import StepBuffers
+from oracle import seer_oracle as O
+
+from gpu_util import MARGIN, assert_out_close, f64, require_gpu, row_inputs, scale_of
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def check_rows(w, data, run, rows, report):
+    """Compare the step's outputs on the listed (b, h) rows with the oracle."""
+    views = run.workspace_views()
+    idx = views["idx"].cpu().numpy()
+    n_sel = views["n_sel"].cpu().numpy()
+    scores = f64(views["scores"])
+    kbar = f64(run.kbar)
+    out = f64(run.out)
+    lse = f64(run.lse)
+    k_per_seq = run.k_per_seq.cpu().numpy()
+    G = w.group
+    for (b, h) in rows:
+        q, Wg, K, V, L = row_inputs(w, data, b, h)
+        k = int(k_per_seq[b])
+        ref = O.decode_row(q, Wg, K, V, L, w.block_size, k, run.force_newest, scale_of(w), scale_of(w))
+        nb = ref["kbar"].shape[0]
+        # pooled keys and gate scores
+        np.testing.assert_allclose(kbar[b, h, :nb], ref["kbar"], rtol=1e-5, atol=2e-6)
+        bound = 1e-5 * max(1e-3, float(np.abs(ref["scores"]).max(initial=0)))
+        assert np.abs(scores[b, h, :nb] - ref["scores"]).max(initial=0) <= bound + 2e-6
+        # selection: exact where the oracle's margin is clear, valid otherwise
+        got = idx[b, h, :n_sel[b, h]]
+        margin = O.selection_margin(ref["scores"], k, run.force_newest)
+        if margin > MARGIN:
+            assert got.tolist() == ref["indices"].tolist(), (b, h, margin)
+            report["exact"] += 1
+        else:
+            assert O.selection_is_valid(ref["scores"], got, k, run.force_newest, MARGIN), (b, h)
+            report["near_tie"] += 1
+        assert (idx[b, h, n_sel[b, h]:] == -1).all()
+        # attention on the GPU's own index set
+        o, l = O.masked_attention(q, K, V, L, got, w.block_size, scale_of(w))
+        sl = slice(h * G, (h + 1) * G)
+        assert_out_close(out[b, sl], o, (b, h))
+        fin = np.isfinite(l)
+        np.testing.assert_allclose(lse[b, sl][fin], l[fin], atol=1e-3)
+
+
+SMALL = {
+    "b1_g4_L4k_bs64_budget512": dict(),
+    "b8_h32_L8k_bs64_s90_newest": dict(batch=2, seqlen=2000),
+    "b16_h40_L32k_bs64_s90": dict(batch=2, seqlen=3000),
+    "b16_h40_L32k_bs128_budget4k_newest": dict(batch=2, seqlen=5000, budget_tokens=1024),
+    "b64_ragged_h64_paged_bs64": dict(batch=4, seqlen_range=(1, 3000)),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_step_small_workloads(name):
+    w = W.WORKLOADS[name].replace(**SMALL[name])
+    data = W.generate(w, 100, DEV)
+    run = StepBuffers(w, data)
+    run.step(update_kbar=2)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    rows = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    report = {"exact": 0, "near_tie": 0}
+    check_rows(w, data, run, rows, report)
+    print(name, report)
+    assert report["exact"] >= 1
+
+
+@pytest.mark.parametrize("permille", [0, 500, 950])
+def test_step_ragged_sparsity_sweep_small(permille):
+    w = W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(batch=3, seqlen_range=(64, 2500),
+                                                          sparsity_permille=permille)
+    data = W.generate(w, 7, DEV)
+    run = StepBuffers(w, data)
+    run.step(update_kbar=2)
+    torch.cuda.synchronize()
+    report = {"exact": 0, "near_tie": 0}
+    check_rows(w, data, run, [(b, h) for b in range(3) for h in range(8)], report)
+    if permille == 0:   # every block selected: the step is dense attention
+        n_sel = run.workspace_views()["n_sel"].cpu().numpy()
+        L = data["seqlens"].cpu().numpy()
+        assert (n_sel == (-(-L // 64))[:, None]).all()
+
+
+def test_step_edge_cases_empty_and_single_token():
+    """seqlen 0 (nothing to attend: out 0, lse -inf), seqlen 1, a partial
+    newest block, more splits than blocks."""
+    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=4, q_heads=8, kv_heads=2,
+                                                           seqlen=200)
+    data = W.generate(w, 5, DEV)
+    data["seqlens"] = torch.tensor([0, 1, 65, 200], dtype=torch.int32, device=DEV)
+    run = StepBuffers(w, data, num_splits=16)
+    run.step(update_kbar=2)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    out = f64(run.out)
+    lse = f64(run.lse)
+    assert (out[0] == 0).all() and np.isneginf(lse[0]).all()
+    report = {"exact": 0, "near_tie": 0}
+    check_rows(w, data, run, [(b, h) for b in (1, 2, 3) for h in range(2)], report)
+
+
+def test_step_incremental_kbar_matches_full_rebuild():
+    """Run at L - 1 with a full rebuild, append the token at L - 1 (its K/V
+    rows are already in the pool) with the incremental update, and compare
+    with a full rebuild at L."""
+    w = W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(batch=3, seqlen_range=(100, 2000))
+    data = W.generate(w, 9, DEV)
+    data["seqlens"][0] = 65             # the appended token opens a new block
+    run = StepBuffers(w, data)
+    data["seqlens"] -= 1
+    run.step(update_kbar=2)
+    before = run.kbar.clone()
+    data["seqlens"] += 1
+    run.step(update_kbar=1)
+    inc = run.kbar.clone()
+    inc_out = run.out.clone()
+    run.step(update_kbar=2)
+    torch.cuda.synchronize()
+    assert torch.equal(inc, run.kbar)
+    assert torch.equal(inc_out, run.out)
+    assert not torch.equal(before, run.kbar)
+    assert run.status.item() == 0
+
+
+def test_step_host_entry_point_matches_device_step():
+    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=2, seqlen=1500)
+    data = W.generate(w, 3, DEV)
+    run = StepBuffers(w, data)
+    run.pool_full()
+    run.step()
+    dev_out = run.out.clone()
+    q_host = data["q"].cpu().pin_memory()
+    out_host = torch.empty(dev_out.shape, dtype=torch.bfloat16).pin_memory()
+    q_dev = torch.empty_like(data["q"])
+    run.out.zero_()
+    seer.seer_decode_step_host(run.dims, run.args(0, q=q_dev), q_host, q_dev, out_host)
+    torch.cuda.synchronize()
+    assert torch.equal(out_host, dev_out.cpu())
+
+
+# --------------------------------------------------------- full-size, sampled
+
+FULL = [
+    ("b1_g4_L4k_bs64_budget512", {}),
+    ("b8_h32_L8k_bs64_s90_newest", {}),
+    ("b16_h40_L32k_bs64_s90", {}),
+    ("b16_h40_L32k_bs128_budget4k_newest", {}),
+    ("b64_ragged_h64_paged_bs64", {"sparsity_permille": 900}),
+    ("b64_ragged_h64_paged_bs64", {"sparsity_permille": 0}),
+]
+
+
+@pytest.mark.parametrize("name,over", FULL, ids=[f"{n}-{o}" for n, o in FULL])
+def test_step_full_size_sampled(name, over):
+    w = W.WORKLOADS[name].replace(**over)
+    data = W.generate(w, 1, DEV)
+    run = StepBuffers(w, data)          # the benchmark's launch configuration
+    run.pool_full()
+    run.step(update_kbar=0)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    rng = np.random.default_rng(0)
+    all_rows = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    pick = rng.choice(len(all_rows), size=min(6, len(all_rows)), replace=False)
+    rows = [all_rows[i] for i in sorted(pick)]
+    if len(all_rows) > 1:
+        rows.append(all_rows[-1])
+    report = {"exact": 0, "near_tie": 0}
+    check_rows(w, data, run, rows, report)
+    print(name, over, report)
+    # properties over every row: counts, ascending order, range
+    views = run.workspace_views()
+    idx = views["idx"].cpu().numpy()
+    n_sel = views["n_sel"].cpu().numpy()
+    L = data["seqlens"].cpu().numpy()
+    k = run.k_per_seq.cpu().numpy()
+    for b in range(w.batch):
+        nb = -(-int(L[b]) // w.block_size)
+        for h in range(w.kv_heads):
+            n = n_sel[b, h]
+            assert n == min(int(k[b]), nb)
+            row = idx[b, h, :n]
+            assert (np.diff(row) > 0).all() and row.min() >= 0 and row.max() < nb
+            if run.force_newest:
+                assert row[-1] == nb - 1
+    assert np.isfinite(f64(run.out)).all()
