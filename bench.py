@@ -1,0 +1,486 @@
+"""Benchmark of the block-sparse decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed alone
+
+One step = one pass of the whole hot path over one batch: incremental pooled-
+key update of the newest block, gate scores, top-k block selection, split-KV
+sparse decode and LSE combine (five kernels, one ``seer_decode_step`` call).
+Inputs are seeded synthetic tensors already resident in HBM; the timed loop
+rotates over R independent replicas whose combined footprint exceeds four
+times the L2, so every step reads its K/V, pooled keys and weights from HBM.
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs its own
+replica of the workload (the step has no exchange: "replicas only", weak
+scaling) and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-decode tokens/s and µs/step at 32K ctx, 90% sparsity; HBM GB/s vs roofline"
+UNIT = "tokens/s"
+KERNELS_PER_STEP = 5
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def decode_source_hash():
+    h = hashlib.sha256()
+    for name in ("sparse_decode.cu", "seer_common.cuh", "seer_kernels.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_step_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"sparse_decode_{workload}.traffic.txt")
+    try:
+        kv = dict(line.split(":", 1) for line in open(path) if ":" in line)
+    except OSError:
+        return None
+    kv = {k.strip(): v.strip() for k, v in kv.items()}
+    if kv.get("source_hash") != decode_source_hash():
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            target = str(device_index)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", target], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, loaded, reasons = [], [], [], set()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                s, m, pw = float(parts[1]), float(parts[2]), float(parts[3])
+            except ValueError:
+                continue
+            sm.append(s)
+            smax.append(m)
+            if pw > 200:          # under load
+                loaded.append(s)
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        use = loaded or sm
+        return {"sm_mhz": statistics.median(use) if use else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_rows_timed(w, data, rows, budget_s, k_per_seq, force_newest):
+    """Time the fp64 oracle's whole step on (b, h) rows, one after another,
+    until the row list or the time budget runs out.  Returns (seconds per
+    row, rows timed, threads)."""
+    import numpy as np
+    from block_sparse_attention_step_b200 import workloads as W
+    from oracle import seer_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    scale = 1.0 / math.sqrt(w.head_dim)
+    G = w.group
+    spent, done = 0.0, 0
+    for (b, h) in rows:
+        L = int(data["seqlens"][b])
+        q = data["q"][b, h * G:(h + 1) * G].double().cpu().numpy()
+        Wg = data["w_gate"][h].double().cpu().numpy()
+        K = W.gather_rows(data["k_pool"], data["page_table"], b, h, L, w.block_size).double().numpy()
+        V = W.gather_rows(data["v_pool"], data["page_table"], b, h, L, w.block_size).double().numpy()
+        t0 = time.perf_counter()
+        O.decode_row(q, Wg, K, V, L, w.block_size, int(k_per_seq[b]), force_newest, scale, scale)
+        spent += time.perf_counter() - t0
+        done += 1
+        if spent >= budget_s:
+            break
+    return spent / max(done, 1), done, threads
+
+
+def cpu_k_per_seq(w, seqlens):
+    from oracle import seer_oracle as O
+    out = []
+    for L in seqlens:
+        nb = O.num_blocks(int(L), w.block_size)
+        if w.budget_tokens:
+            out.append(O.k_from_budget(nb, w.budget_tokens, w.block_size))
+        else:
+            out.append(O.k_from_sparsity(nb, w.sparsity_permille))
+    return out
+
+
+def run_reference(args):
+    """The oracle alone on the host cores: each step is a bounded sample of
+    the workload's (b, h) rows, scaled to tokens/s of the whole batch."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import torch
+    from block_sparse_attention_step_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    # rows of a batch-1 draw have the workload's per-row shape (L, G, bs, k)
+    one = w.replace(batch=1) if w.seqlen_range is None else w.replace(batch=2)
+    data = W.generate(one, args.seed, "cpu")
+    kps = cpu_k_per_seq(one, data["seqlens"].tolist())
+    rows = [(b, h) for b in range(one.batch) for h in range(one.kv_heads)]
+    per_step = max(1, min(len(rows), args.ref_rows))
+    times = []
+    for i in range(args.warmup + args.steps):
+        sample = [rows[(i * per_step + r) % len(rows)] for r in range(per_step)]
+        sec, n, threads = oracle_rows_timed(one, data, sample, 1e9, kps, w.force_newest)
+        if i >= args.warmup:
+            times.append(sec)
+    sec_row = sum(times) / len(times)
+    if w.seqlen_range is not None:
+        sec_row *= _ragged_row_scale(w, data)
+    step_s = sec_row * w.batch * w.kv_heads
+    value = w.batch / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, None),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{per_step} (b, kv-head) rows of a batch-{one.batch} draw per "
+                                   f"step, fp64 numpy oracle, scaled to {w.batch}x{w.kv_heads} rows"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _ragged_row_scale(w, data):
+    """Oracle cost grows with L: scale the sampled rows' mean length to the
+    workload's expected mean length."""
+    lo, hi = w.seqlen_range
+    sampled = float(data["seqlens"].double().mean())
+    return ((lo + hi) / 2.0) / sampled
+
+
+def workload_config(w, run, replicas=None, touched=None):
+    cfg = {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+           "head_dim": w.head_dim, "block_size": w.block_size,
+           "seq_len": w.seqlen if w.seqlen else f"U[{w.seqlen_range[0]},{w.seqlen_range[1]}]",
+           "selection": (f"budget {w.budget_tokens} tokens" if w.budget_tokens
+                         else f"sparsity {w.sparsity_permille / 10:g}%"),
+           "force_newest": w.force_newest, "paged": w.paged}
+    if run is not None:
+        cfg["num_splits"] = run.num_splits
+        cfg["k_max"] = run.k_max
+    if replicas is not None:
+        cfg["l2"] = (f"inputs larger than L2: {replicas} rotating replicas, "
+                     f"{touched / 1e6:.0f} MB read per step, L2 126 MB")
+    return cfg
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_step_b200 import seer
+    from block_sparse_attention_step_b200 import workloads as W
+    from block_sparse_attention_step_b200.runner import StepBuffers
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    seer.library()
+    w = W.WORKLOADS[args.workload]
+    if args.sparsity is not None:
+        w = w.replace(sparsity_permille=args.sparsity, budget_tokens=None)
+
+    # replicas: enough that one rotation reads > 4x L2
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    probe = W.generate(w, args.seed + 1000 * rank, dev)
+    run0 = StepBuffers(w, probe, num_splits=args.splits)
+    run0.pool_full()
+    torch.cuda.synchronize()
+    sel_bytes, sel_tokens = selected_bytes(run0, probe, w)
+    kbar_bytes = run0.kbar.numel() * 4
+    touched = sel_bytes + kbar_bytes
+    replicas = max(2, math.ceil(4 * l2 / max(touched, 1)))
+    replicas = min(replicas, args.max_replicas)
+    runs = [run0]
+    for r in range(1, replicas):
+        d = W.generate(w, args.seed + 1000 * rank + r, dev)
+        rr = StepBuffers(w, d, num_splits=run0.num_splits, k_max=run0.k_max)
+        rr.pool_full()
+        runs.append(rr)
+    step_args = [r.args(update_kbar=1) for r in runs]
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    for i in range(args.warmup):
+        seer.seer_decode_step(runs[i % replicas].dims, step_args[i % replicas], stream)
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        seer.seer_decode_step(runs[i % replicas].dims, step_args[i % replicas], stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_total = t0.elapsed_time(t1)
+    ms_max = ms_total
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+
+    # ---- per-stage durations: the same five kernels called one by one with
+    # events between them on the launching stream, K more steps
+    stage = stage_breakdown(runs, args.steps, stream, replicas)
+
+    # ---- end to end through the host entry point: q from pinned host memory
+    # in, out to pinned host memory back, every step
+    e2e = end_to_end(runs, args.steps, stream, replicas, w)
+    clock_info = clocks.stop() if clocks else None
+    status = [int(r.status.item()) for r in runs]
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = measured_peaks()
+    dec_us = stage["sparse_decode"]
+    dec_bytes = decode_bytes(run0, sel_bytes, w)
+    achieved = dec_bytes / (dec_us * 1e-6) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": world * w.batch / (ms_step * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "us_per_step": ms_step * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; random-init gate projection)",
+        "config": workload_config(w, run0, replicas, touched),
+        "selected_kv_bytes_per_step": sel_bytes,
+        "selected_tokens_per_step": sel_tokens,
+        "step_hbm_gbs": (touched / (ms_step * 1e-3)) / 1e9,
+        "selected_kv_gbs": (sel_bytes / (ms_step * 1e-3)) / 1e9,
+        "stage_us": stage,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": recorded_traffic(w.name), "kernel": "sparse_decode_kernel",
+                     "bytes_per_launch": dec_bytes, "peak_source": f"{peak_kind} hbm_gbs"},
+        "e2e": e2e,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clock_info,
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, runs[0], args)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def selected_bytes(run, data, w):
+    """Bytes of K and V the selection makes the decode kernel read (valid
+    tokens of the selected blocks x D x 2 bytes x 2 tensors), from the
+    selection this input actually produces."""
+    import torch
+    run.step(update_kbar=0)
+    torch.cuda.synchronize()
+    v = run.workspace_views()
+    idx = v["idx"].long()
+    n = v["n_sel"].long()
+    L = data["seqlens"].long()
+    bs = w.block_size
+    pos = torch.arange(idx.shape[-1], device=idx.device)
+    live = pos[None, None, :] < n[:, :, None]
+    start = idx.clamp(min=0) * bs
+    valid = (L[:, None, None] - start).clamp(min=0, max=bs) * live
+    tokens = int(valid.sum().item())
+    return tokens * w.head_dim * 2 * 2, tokens
+
+
+def decode_bytes(run, sel_bytes, w):
+    """Algorithmic bytes of one decode launch: selected K/V, q, the index
+    rows, and the split partials written."""
+    B, Hq, Hkv, S, D = w.batch, w.q_heads, w.kv_heads, run.num_splits, w.head_dim
+    return (sel_bytes + B * Hq * D * 2 + B * Hkv * (run.k_max + 1) * 4 + B * Hq * S * (D + 1) * 4)
+
+
+def stage_breakdown(runs, steps, stream, replicas):
+    import torch
+    from block_sparse_attention_step_b200 import seer
+    names = ("pool_keys", "gate_scores", "block_select", "sparse_decode", "combine")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for i in range(steps):
+        r = runs[i % replicas]
+        v = r.views_cache if hasattr(r, "views_cache") else r.workspace_views()
+        r.views_cache = v
+        d, data = r.dims, r.data
+        e = ev[i]
+        e[0].record(stream)
+        seer.seer_pool_keys(d, data["k_pool"], data["page_table"], data["seqlens"], 1, r.kbar,
+                            r.status, stream)
+        e[1].record(stream)
+        seer.seer_gate_scores(d, data["q"], data["w_gate"], r.kbar, data["seqlens"], r.scale,
+                              v["scores"], r.status, stream)
+        e[2].record(stream)
+        seer.seer_block_select(d, v["scores"], data["seqlens"], r.k_per_seq, r.force_newest,
+                               r.k_max, v["idx"], v["n_sel"], r.status, stream)
+        e[3].record(stream)
+        seer.seer_sparse_decode(d, data["q"], data["k_pool"], data["v_pool"], data["page_table"],
+                                data["seqlens"], v["idx"], v["n_sel"], r.k_max, r.num_splits,
+                                r.scale, v["o_part"], v["lse_part"], r.status, stream)
+        e[4].record(stream)
+        seer.seer_combine(d, v["o_part"], v["lse_part"], r.num_splits, r.out, r.lse, stream)
+        e[5].record(stream)
+    torch.cuda.synchronize()
+    out = {}
+    for k, name in enumerate(names):
+        out[name] = sum(ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(steps)) / steps * 1e3
+    out["sum"] = sum(out[n] for n in names)
+    return out
+
+
+def end_to_end(runs, steps, stream, replicas, w):
+    import torch
+    from block_sparse_attention_step_b200 import seer
+    q_host = [r.data["q"].cpu().pin_memory() for r in runs]
+    out_host = [torch.empty(r.out.shape, dtype=torch.bfloat16).pin_memory() for r in runs]
+    q_dev = [torch.empty_like(r.data["q"]) for r in runs]
+    args = [r.args(update_kbar=1, q=q_dev[i]) for i, r in enumerate(runs)]
+    for i in range(3):
+        seer.seer_decode_step_host(runs[i % replicas].dims, args[i % replicas], q_host[i % replicas],
+                                   q_dev[i % replicas], out_host[i % replicas], stream)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        k = i % replicas
+        seer.seer_decode_step_host(runs[k].dims, args[k], q_host[k], q_dev[k], out_host[k], stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    ms = a.elapsed_time(b) / steps
+    qbytes = runs[0].data["q"].numel() * 2
+    return {"value": w.batch / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": qbytes,
+            "d2h_bytes_per_step": runs[0].out.numel() * 2, "ms_per_step": ms,
+            "host_wall_ms_per_step": wall / steps * 1e3,
+            "path": "seer_decode_step_host: pinned q H2D, step, out D2H, device-timed"}
+
+
+def cpu_baseline(w, run, args):
+    rows = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    import random
+    random.Random(0).shuffle(rows)
+    k = run.k_per_seq.cpu().tolist()
+    sec_row, n, threads = oracle_rows_timed(w, run.data, rows, args.cpu_budget, k, run.force_newest)
+    step_s = sec_row * len(rows)
+    return {"value": w.batch / step_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {len(rows)} (b, kv-head) rows of this workload, fp64 numpy oracle "
+                      f"(pool, gate, select, masked attention), {sec_row * 1e3:.1f} ms/row, scaled "
+                      f"to the whole batch"}
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    from block_sparse_attention_step_b200 import workloads as W
+    p.add_argument("--workload", choices=sorted(W.WORKLOADS), default=W.HEADLINE)
+    p.add_argument("--sparsity", type=int, default=None, help="override: sparsity in permille")
+    p.add_argument("--splits", type=int, default=None)
+    p.add_argument("--seed", type=int, default=1)
+    p.add_argument("--max-replicas", type=int, default=8)
+    p.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time")
+    p.add_argument("--ref-rows", type=int, default=4, help="oracle rows per reference step")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        p.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

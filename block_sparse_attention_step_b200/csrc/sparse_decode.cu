@@ -18,7 +18,8 @@
 //     warp owns 16 tokens of the tile and computes S = Q K^T and O += P V with
 //     mma.sync m16n8k16 (the group's G <= 16 query heads are the 16 rows, so
 //     each K/V byte is read from HBM once for all G heads), online softmax in
-//     the exp2 domain with warp-quad shuffles;
+//     the exp2 domain with warp-quad shuffles, P fed to the tensor cores as a
+//     bf16 hi + lo pair so the weights keep ~16 bits;
 //   * at the end of an item the 4*NGROUPS warps merge their (m, l, O) through
 //     shared memory and write o_part / lse_part.
 // Every mbarrier wait is bounded (SEER_DEV_TIMEOUT); nothing traps.
@@ -261,11 +262,14 @@ __global__ void __launch_bounds__(DecodeShape<NGROUPS, NSTAGES>::kThreads, 1)
             o[nd][2] *= a1;
             o[nd][3] *= a1;
           }
-          uint32_t pa[4];
-          pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
-          pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
-          pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
-          pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+          // P as a bf16 pair hi + lo (hi = RNE(p), lo = RNE(p - hi)): the
+          // product P V then carries p to ~2^-16 instead of bf16's 2^-9, so
+          // heavy-tailed V rows do not amplify the rounding of the weights.
+          uint32_t pa[4], pl[4];
+          split_bf16x2(pr[0][0], pr[0][1], pa[0], pl[0]);
+          split_bf16x2(pr[0][2], pr[0][3], pa[1], pl[1]);
+          split_bf16x2(pr[1][0], pr[1][1], pa[2], pl[2]);
+          split_bf16x2(pr[1][2], pr[1][3], pa[3], pl[3]);
 
           // ---- O += P V (V tile rows past the end are zeroed in registers:
           // their P is 0 but the slot may hold anything, NaN included)
@@ -285,8 +289,14 @@ __global__ void __launch_bounds__(DecodeShape<NGROUPS, NSTAGES>::kThreads, 1)
                                   ((chunk ^ (vtok & 7)) << 4);
             uint32_t b0, b1, b2, b3;
             ldmatrix_x4_trans(addr, b0, b1, b2, b3);
-            mma_bf16_16816(o[2 * dp], pa, b0 & vmask_lo, b1 & vmask_hi);
-            mma_bf16_16816(o[2 * dp + 1], pa, b2 & vmask_lo, b3 & vmask_hi);
+            b0 &= vmask_lo;
+            b1 &= vmask_hi;
+            b2 &= vmask_lo;
+            b3 &= vmask_hi;
+            mma_bf16_16816(o[2 * dp], pa, b0, b1);
+            mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+            mma_bf16_16816(o[2 * dp], pl, b0, b1);
+            mma_bf16_16816(o[2 * dp + 1], pl, b2, b3);
           }
         }
         __syncwarp();
