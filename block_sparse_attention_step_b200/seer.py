@@ -31,8 +31,9 @@ EXPORTS = (
     "seer_version", "seer_status_string", "seer_dims_default", "seer_k_from_sparsity",
     "seer_k_from_budget", "seer_fill_k", "seer_default_splits", "seer_step_workspace_bytes",
     "seer_pool_keys", "seer_gate_scores", "seer_block_select", "seer_sparse_decode",
-    "seer_combine", "seer_decode_step", "seer_decode_step_host",
+    "seer_combine", "seer_decode_step", "seer_decode_step_host", "seer_decode_step_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class SeerError(RuntimeError):
@@ -82,6 +83,7 @@ _SIGS = {
     "seer_combine": (_I, [_D, _P, _P, _I, _P, _P, _P]),
     "seer_decode_step": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_decode_step_host": (_I, [_D, ctypes.POINTER(seer_step_args), _P, _P, _P, _P]),
+    "seer_decode_step_noalloc": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
 }
 
 _lib_handle = None
@@ -255,3 +257,10 @@ def seer_decode_step_host(d, args: seer_step_args, q_host, q_dev, out_host, stre
         ctypes.byref(d), ctypes.byref(args), _ptr(q_host, torch.bfloat16, "q_host", device=False),
         _ptr(q_dev, torch.bfloat16, "q_dev"), _ptr(out_host, torch.bfloat16, "out_host", device=False),
         _stream(stream)))
+
+
+def seer_decode_step_noalloc(d, args: seer_step_args, stream=None):
+    """The step with the library's own fixed 16 MiB device scratch instead of
+    ``args.workspace`` (for callers that cannot allocate device memory)."""
+    _check("seer_decode_step_noalloc", _lib().seer_decode_step_noalloc(
+        ctypes.byref(d), ctypes.byref(args), _stream(stream)))

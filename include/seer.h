@@ -241,6 +241,37 @@ SEER_API seer_status seer_decode_step_host(const seer_dims *d, const seer_step_a
                                   const uint16_t *q_host, uint16_t *q_dev,
                                   uint16_t *out_host, seer_stream stream);
 
+/* ------------------------------------------------------ no-allocation step
+ * No counterpart in the paper: this entry point exists for callers that
+ * cannot allocate device memory themselves -- a host framework or serving
+ * runtime that owns every byte of GPU memory through its own pool (a
+ * separate allocation would escape its accounting, or fail), or a decode loop
+ * that must never enter the CUDA allocator (cudaMalloc can serialise against
+ * other work and can fail under memory pressure mid-generation).
+ *
+ * It runs exactly seer_decode_step, but its workspace is a file-scope device
+ * array of SEER_NOALLOC_SCRATCH_BYTES (16 MiB) inside this library: every GPU
+ * that loads the library holds those 16 MiB until the process exits.
+ * a->workspace and a->workspace_bytes are ignored; the caller still passes
+ * every input and output.  Nothing is allocated or freed, by this call or by
+ * anything it calls.
+ *   - Limit: when seer_step_workspace_bytes(d, a->k_max, a->num_splits)
+ *     exceeds SEER_NOALLOC_SCRATCH_BYTES the call returns SEER_ERR_WORKSPACE
+ *     before anything is enqueued.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current and caches it;
+ *     make that first call before any stream capture begins.
+ *   - Sharing: all calls on a device use the same array, which keeps the last
+ *     call's contents.  Nothing in it has to start at zero (every byte the
+ *     step reads there is written earlier by the same call), but calls whose
+ *     work can overlap on the GPU -- two streams, or two host threads -- race
+ *     on it: order them on one stream or serialise them. */
+#define SEER_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+SEER_API seer_status seer_decode_step_noalloc(const seer_dims *d,
+                                              const seer_step_args *a,
+                                              seer_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

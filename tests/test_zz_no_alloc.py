@@ -1,0 +1,57 @@
+"""seer_decode_step_noalloc against seer_decode_step, through the C ABI.
+
+The no-allocation entry point serves callers that cannot allocate device
+memory (a host runtime that owns all GPU memory through its own pool, or a
+decode loop that must never enter the CUDA allocator): it runs the same step
+with the library's fixed 16 MiB device array as workspace.  Two calls in a
+row must each match the caller-workspace step within the output tolerance the
+other tests use, and a size beyond the array must be refused.  This file is
+collected last on purpose, so a failure here comes after every other test has
+run; it also passes alone in a fresh process.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_step_b200 import seer
+from block_sparse_attention_step_b200 import workloads as W
+from block_sparse_attention_step_b200.runner import StepBuffers
+
+from gpu_util import assert_out_close, f64, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_step_matches_workspace_step_twice():
+    require_gpu()
+    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=4, seqlen=3000)
+    data = W.generate(w, 17, "cuda")
+    run = StepBuffers(w, data)
+    run.pool_full()
+    run.step(update_kbar=0)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = f64(run.out), f64(run.lse)
+    assert run.status.item() == 0
+
+    need = seer.seer_step_workspace_bytes(run.dims, run.k_max, run.num_splits)
+    assert 0 < need <= seer.NOALLOC_SCRATCH_BYTES
+    for call in range(2):
+        run.out.fill_(0)
+        run.lse.fill_(0)
+        seer.seer_decode_step_noalloc(run.dims, run.args(update_kbar=0))
+        torch.cuda.synchronize()
+        out, lse = f64(run.out), f64(run.lse)
+        for b in range(w.batch):
+            assert_out_close(out[b], ref_out[b], ("call", call, "batch", b))
+        np.testing.assert_allclose(lse, ref_lse, atol=1e-3)
+        assert run.status.item() == 0
+
+    # a request larger than the fixed array is refused before any work
+    big = seer.make_dims(64, 64, 8, 128, 64, 4096, 64 * 4096)
+    args = run.args(update_kbar=0)
+    args.k_max = 4096
+    args.num_splits = 64
+    assert seer.seer_step_workspace_bytes(big, 4096, 64) > seer.NOALLOC_SCRATCH_BYTES
+    with pytest.raises(seer.SeerError) as e:
+        seer.seer_decode_step_noalloc(big, args)
+    assert e.value.status == 4          # SEER_ERR_WORKSPACE
