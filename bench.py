@@ -5,7 +5,8 @@
 
 One step = one pass of the whole hot path over one batch: incremental pooled-
 key update of the newest block, gate scores, top-k block selection, split-KV
-sparse decode and LSE combine (five kernels, one ``seer_decode_step`` call).
+sparse decode and LSE combine (one ``seer_decode_step`` call: the fused
+pool+gate+select kernel, the decode kernel and the combine kernel).
 Inputs are seeded synthetic tensors already resident in HBM; the timed loop
 rotates over R independent replicas whose combined footprint exceeds four
 times the L2, so every step reads its K/V, pooled keys and weights from HBM.
@@ -31,7 +32,7 @@ if ROOT not in sys.path:
 
 METRIC = "sparse-decode tokens/s and µs/step at 32K ctx, 90% sparsity; HBM GB/s vs roofline"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 5
+KERNELS_PER_STEP = 3   # gate+select (with the incremental pooled-key update), decode, combine
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -144,8 +145,8 @@ def oracle_rows_timed(w, data, rows, budget_s, k_per_seq, force_newest):
         L = int(data["seqlens"][b])
         q = data["q"][b, h * G:(h + 1) * G].double().cpu().numpy()
         Wg = data["w_gate"][h].double().cpu().numpy()
-        K = W.gather_rows(data["k_pool"], data["page_table"], b, h, L, w.block_size).double().numpy()
-        V = W.gather_rows(data["v_pool"], data["page_table"], b, h, L, w.block_size).double().numpy()
+        K = W.gather_rows(data["k_pool"], data["page_table"], b, h, L, w.block_size, data.get("layout", "nhd")).double().numpy()
+        V = W.gather_rows(data["v_pool"], data["page_table"], b, h, L, w.block_size, data.get("layout", "nhd")).double().numpy()
         t0 = time.perf_counter()
         O.decode_row(q, Wg, K, V, L, w.block_size, int(k_per_seq[b]), force_newest, scale, scale)
         spent += time.perf_counter() - t0
@@ -214,13 +215,15 @@ def _ragged_row_scale(w, data):
     return ((lo + hi) / 2.0) / sampled
 
 
-def workload_config(w, run, replicas=None, touched=None):
+def workload_config(w, run, replicas=None, touched=None, layout=None):
     cfg = {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
            "head_dim": w.head_dim, "block_size": w.block_size,
            "seq_len": w.seqlen if w.seqlen else f"U[{w.seqlen_range[0]},{w.seqlen_range[1]}]",
            "selection": (f"budget {w.budget_tokens} tokens" if w.budget_tokens
                          else f"sparsity {w.sparsity_permille / 10:g}%"),
            "force_newest": w.force_newest, "paged": w.paged}
+    if layout is not None:
+        cfg["kv_layout"] = layout
     if run is not None:
         cfg["num_splits"] = run.num_splits
         cfg["k_max"] = run.k_max
@@ -255,7 +258,7 @@ def run_ours(args):
 
     # replicas: enough that one rotation reads > 4x L2
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
-    probe = W.generate(w, args.seed + 1000 * rank, dev)
+    probe = W.generate(w, args.seed + 1000 * rank, dev, layout=args.layout)
     run0 = StepBuffers(w, probe, num_splits=args.splits)
     run0.pool_full()
     torch.cuda.synchronize()
@@ -266,7 +269,7 @@ def run_ours(args):
     replicas = min(replicas, args.max_replicas)
     runs = [run0]
     for r in range(1, replicas):
-        d = W.generate(w, args.seed + 1000 * rank + r, dev)
+        d = W.generate(w, args.seed + 1000 * rank + r, dev, layout=args.layout)
         rr = StepBuffers(w, d, num_splits=run0.num_splits, k_max=run0.k_max)
         rr.pool_full()
         runs.append(rr)
@@ -301,9 +304,8 @@ def run_ours(args):
         ms_max = float(t.item())
     ms_step = ms_max / args.steps
 
-    # ---- per-stage durations: the same five kernels called one by one with
-    # events between them on the launching stream, K more steps
-    stage = stage_breakdown(runs, args.steps, stream, replicas)
+    # ---- the dominant kernel alone (roofline), K more launches
+    dec_us = decode_alone(runs, args.steps, stream, replicas)
 
     # ---- end to end through the host entry point: q from pinned host memory
     # in, out to pinned host memory back, every step
@@ -318,7 +320,6 @@ def run_ours(args):
         return 0
 
     peaks, peak_kind = measured_peaks()
-    dec_us = stage["sparse_decode"]
     dec_bytes = decode_bytes(run0, sel_bytes, w)
     achieved = dec_bytes / (dec_us * 1e-6) / 1e9
     line = {
@@ -335,12 +336,13 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; random-init gate projection)",
-        "config": workload_config(w, run0, replicas, touched),
+        "config": workload_config(w, run0, replicas, touched, args.layout),
         "selected_kv_bytes_per_step": sel_bytes,
         "selected_tokens_per_step": sel_tokens,
         "step_hbm_gbs": (touched / (ms_step * 1e-3)) / 1e9,
         "selected_kv_gbs": (sel_bytes / (ms_step * 1e-3)) / 1e9,
-        "stage_us": stage,
+        "stage_us": {"step": ms_step * 1e3, "sparse_decode_alone": dec_us,
+                     "rest_of_step": ms_step * 1e3 - dec_us},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": recorded_traffic(w.name), "kernel": "sparse_decode_kernel",
@@ -383,39 +385,30 @@ def decode_bytes(run, sel_bytes, w):
     return (sel_bytes + B * Hq * D * 2 + B * Hkv * (run.k_max + 1) * 4 + B * Hq * S * (D + 1) * 4)
 
 
-def stage_breakdown(runs, steps, stream, replicas):
+def decode_alone(runs, steps, stream, replicas):
+    """Mean duration of the dominant kernel, sparse decode, launched alone K
+    times over the rotating replicas (each replica's index rows are those its
+    last step selected), CUDA events on the launching stream."""
     import torch
     from block_sparse_attention_step_b200 import seer
-    names = ("pool_keys", "gate_scores", "block_select", "sparse_decode", "combine")
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
-    for i in range(steps):
-        r = runs[i % replicas]
-        v = r.views_cache if hasattr(r, "views_cache") else r.workspace_views()
-        r.views_cache = v
-        d, data = r.dims, r.data
-        e = ev[i]
-        e[0].record(stream)
-        seer.seer_pool_keys(d, data["k_pool"], data["page_table"], data["seqlens"], 1, r.kbar,
-                            r.status, stream)
-        e[1].record(stream)
-        seer.seer_gate_scores(d, data["q"], data["w_gate"], r.kbar, data["seqlens"], r.scale,
-                              v["scores"], r.status, stream)
-        e[2].record(stream)
-        seer.seer_block_select(d, v["scores"], data["seqlens"], r.k_per_seq, r.force_newest,
-                               r.k_max, v["idx"], v["n_sel"], r.status, stream)
-        e[3].record(stream)
-        seer.seer_sparse_decode(d, data["q"], data["k_pool"], data["v_pool"], data["page_table"],
-                                data["seqlens"], v["idx"], v["n_sel"], r.k_max, r.num_splits,
+    views = [r.workspace_views() for r in runs]
+
+    def launch(i):
+        r, v = runs[i % replicas], views[i % replicas]
+        d = r.data
+        seer.seer_sparse_decode(r.dims, d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                d["seqlens"], v["idx"], v["n_sel"], r.k_max, r.num_splits,
                                 r.scale, v["o_part"], v["lse_part"], r.status, stream)
-        e[4].record(stream)
-        seer.seer_combine(d, v["o_part"], v["lse_part"], r.num_splits, r.out, r.lse, stream)
-        e[5].record(stream)
+    for i in range(3):
+        launch(i)
     torch.cuda.synchronize()
-    out = {}
-    for k, name in enumerate(names):
-        out[name] = sum(ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(steps)) / steps * 1e3
-    out["sum"] = sum(out[n] for n in names)
-    return out
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        launch(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps * 1e3
 
 
 def end_to_end(runs, steps, stream, replicas, w):
@@ -469,6 +462,8 @@ def main(argv=None):
     p.add_argument("--workload", choices=sorted(W.WORKLOADS), default=W.HEADLINE)
     p.add_argument("--sparsity", type=int, default=None, help="override: sparsity in permille")
     p.add_argument("--splits", type=int, default=None)
+    p.add_argument("--layout", choices=("nhd", "hnd"), default="nhd",
+                   help="KV pool page layout: token-major [P][bs][Hkv][D] or head-major [P][Hkv][bs][D]")
     p.add_argument("--seed", type=int, default=1)
     p.add_argument("--max-replicas", type=int, default=8)
     p.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time")

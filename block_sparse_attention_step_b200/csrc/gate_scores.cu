@@ -9,15 +9,10 @@
 // then streams its chunk of kbar rows, one warp per row, 4 rows in flight per
 // warp, a 32-lane float4 dot product and a shuffle reduction per row.  The
 // kbar stream is the HBM cost: NB * D * 4 bytes per (b, h).
+#include "block_mean.cuh"
 #include "seer_kernels.cuh"
 
 namespace seer {
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 __global__ void __launch_bounds__(256) gate_scores_kernel(const GateParams p) {
   __shared__ __align__(16) float qbar[kHeadDim];
@@ -48,7 +43,7 @@ __global__ void __launch_bounds__(256) gate_scores_kernel(const GateParams p) {
 #pragma unroll 4
     for (int row = warp; row < kHeadDim; row += 8) {
       const float4 w = __ldg(reinterpret_cast<const float4*>(W + row * kHeadDim + 4 * lane));
-      const float v = warp_sum(w.x * qv.x + w.y * qv.y + w.z * qv.z + w.w * qv.w);
+      const float v = warp_dot4(w, qv);
       if (lane == 0) gvec[row] = v * p.gate_scale;
     }
   }
@@ -67,7 +62,7 @@ __global__ void __launch_bounds__(256) gate_scores_kernel(const GateParams p) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = jb + u;
-      const float sc = warp_sum(v[u].x * gv.x + v[u].y * gv.y + v[u].z * gv.z + v[u].w * gv.w);
+      const float sc = warp_dot4(v[u], gv);
       if (lane == 0 && j < j1) {
         if (j < nb) {
           out[j] = sc;

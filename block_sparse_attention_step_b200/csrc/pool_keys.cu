@@ -9,12 +9,13 @@
 // order through shared memory (deterministic).  The incremental form runs one
 // CTA per (b, h) on the newest block NB_b - 1 only: the block the appended
 // token changed.
+#include "block_mean.cuh"
 #include "seer_kernels.cuh"
 
 namespace seer {
 
 __global__ void __launch_bounds__(256) pool_keys_kernel(const PoolParams p) {
-  __shared__ float part[8][kHeadDim];
+  __shared__ __align__(16) float part[kPoolWarps][kHeadDim];
   const int b = blockIdx.z, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int L = __ldg(p.seqlens + b);
@@ -35,23 +36,10 @@ __global__ void __launch_bounds__(256) pool_keys_kernel(const PoolParams p) {
     return;
   }
   const uint16_t* base = p.k_pool + page * p.stride_page + (int64_t)h * p.stride_head + 4 * lane;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-  for (int t = warp; t < valid; t += 8) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(base + (int64_t)t * p.stride_token));
-    a0 += __uint_as_float(v.x << 16);
-    a1 += __uint_as_float(v.x & 0xffff0000u);
-    a2 += __uint_as_float(v.y << 16);
-    a3 += __uint_as_float(v.y & 0xffff0000u);
-  }
-  *reinterpret_cast<float4*>(&part[warp][4 * lane]) = make_float4(a0, a1, a2, a3);
+  const float4 a = pool_warp_partial(base, p.stride_token, valid, warp);
+  *reinterpret_cast<float4*>(&part[warp][4 * lane]) = a;
   __syncthreads();
-  if (threadIdx.x < kHeadDim) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
-    dst[threadIdx.x] = s / (float)valid;
-  }
+  if (threadIdx.x < kHeadDim) dst[threadIdx.x] = pool_finish(&part[0][0], threadIdx.x, valid);
 }
 
 cudaError_t run_pool_keys(const PoolParams& p, int B, cudaStream_t stream) {

@@ -374,13 +374,43 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   if (a->workspace == nullptr || !aligned(a->workspace, 256)) return SEER_ERR_WORKSPACE;
   const Workspace w = carve(d, a->k_max, a->num_splits, a->workspace);
   if (a->workspace_bytes < w.bytes) return SEER_ERR_WORKSPACE;
-  if (a->update_kbar)
-    SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, a->update_kbar == 1 ? 1 : 0,
-                            a->kbar, a->dev_status, stream));
-  SEER_TRY(seer_gate_scores(d, a->q, a->w_gate, a->kbar, a->seqlens, a->gate_scale, w.scores,
-                            a->dev_status, stream));
-  SEER_TRY(seer_block_select(d, w.scores, a->seqlens, a->k_per_seq, a->force_newest, a->k_max,
-                             w.idx, w.n_sel, a->dev_status, stream));
+  if (a->update_kbar == 2)
+    SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
+                            stream));
+  // a0 (incremental) + a1 + a2 in one kernel; same results as the three calls
+  SEER_TRY(check_pool(d, a->k_pool));
+  if (!a->q || !a->w_gate || !a->seqlens) return SEER_ERR_INVALID_ARG;
+  if (a->k_max > d->max_blocks) return SEER_ERR_INVALID_ARG;
+  if (!aligned(a->w_gate, 16) || !aligned(a->kbar, 16) || !aligned(a->q, 4))
+    return SEER_ERR_UNSUPPORTED;
+  {
+    GateSelectParams g;
+    g.q = a->q;
+    g.w_gate = a->w_gate;
+    g.kbar = a->kbar;
+    g.seqlens = a->seqlens;
+    g.k_per_seq = a->k_per_seq;
+    g.scores = w.scores;
+    g.idx = w.idx;
+    g.n_sel = w.n_sel;
+    g.status = a->dev_status;
+    g.k_pool = a->k_pool;
+    g.page_table = a->page_table;
+    g.incremental = a->update_kbar == 1 ? 1 : 0;
+    g.num_pages = d->num_pages;
+    g.stride_page = d->stride_page;
+    g.stride_token = d->stride_token;
+    g.stride_head = d->stride_head;
+    g.Hq = d->num_q_heads;
+    g.Hkv = d->num_kv_heads;
+    g.G = d->num_q_heads / d->num_kv_heads;
+    g.bs = d->block_size;
+    g.max_blocks = d->max_blocks;
+    g.k_max = a->k_max;
+    g.force_newest = a->force_newest ? 1 : 0;
+    g.gate_scale = a->gate_scale;
+    SEER_CUDA(run_gate_select(g, d->batch, stream));
+  }
   SEER_TRY(seer_sparse_decode(d, a->q, a->k_pool, a->v_pool, a->page_table, a->seqlens, w.idx,
                               w.n_sel, a->k_max, a->num_splits, a->softmax_scale, w.o_part,
                               w.lse_part, a->dev_status, stream));

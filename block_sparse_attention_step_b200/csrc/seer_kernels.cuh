@@ -36,6 +36,24 @@ struct SelectParams {
   int Hkv, bs, max_blocks, k_max, force_newest;
 };
 
+struct GateSelectParams {
+  const uint16_t* q;
+  const float* w_gate;
+  float* kbar;
+  const int32_t* seqlens;
+  const int32_t* k_per_seq;
+  float* scores;
+  int32_t* idx;
+  int32_t* n_sel;
+  int32_t* status;
+  const uint16_t* k_pool;     // for the incremental pooled-key refresh
+  const int32_t* page_table;
+  int incremental;
+  int64_t num_pages, stride_page, stride_token, stride_head;
+  int Hq, Hkv, G, bs, max_blocks, k_max, force_newest;
+  float gate_scale;
+};
+
 struct DecodeParams {
   const uint16_t* q;
   const int32_t* page_table;
@@ -63,6 +81,7 @@ struct CombineParams {
 cudaError_t run_pool_keys(const PoolParams& p, int B, cudaStream_t stream);
 cudaError_t run_gate_scores(const GateParams& p, int B, cudaStream_t stream);
 cudaError_t run_block_select(const SelectParams& p, int B, cudaStream_t stream);
+cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream);
 cudaError_t run_fill_k(const int32_t* seqlens, int B, int bs, int permille, int budget,
                        int32_t* k_out, cudaStream_t stream);
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,

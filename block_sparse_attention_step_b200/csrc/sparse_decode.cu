@@ -6,22 +6,29 @@
 // blocks idx[b,h, floor(s*n/S) .. floor((s+1)*n/S)); the result is one
 // normalised partial output and its log-sum-exp per query head.
 //
-// How it runs on sm_100a:
-//   * persistent CTAs (one per SM) walk a static list of (b, h, s) items;
-//   * one producer thread streams 64-token tiles of the selected K and V
-//     blocks (4 boxes of 64 tokens x 64 dims, 128-byte swizzled) with 4-D
-//     TMA loads into an NSTAGES-deep shared-memory ring guarded by mbarriers;
-//     page lookup, block index and stride handling all live in the tensor
-//     map coordinates, so the gather costs no address arithmetic in the math
-//     warps;
-//   * NGROUPS groups of 4 math warps take alternate tiles; inside a group each
-//     warp owns 16 tokens of the tile and computes S = Q K^T and O += P V with
-//     mma.sync m16n8k16 (the group's G <= 16 query heads are the 16 rows, so
-//     each K/V byte is read from HBM once for all G heads), online softmax in
-//     the exp2 domain with warp-quad shuffles, P fed to the tensor cores as a
-//     bf16 hi + lo pair so the weights keep ~16 bits;
-//   * at the end of an item the 4*NGROUPS warps merge their (m, l, O) through
-//     shared memory and write o_part / lse_part.
+// How it runs on sm_100a (one persistent CTA per SM, static item list):
+//   * scheduler warp: for each (b, h, s) item it reads the item's index slice
+//     and page numbers lane-parallel (the dependent global loads stay off the
+//     copy path), publishes an item record (the G query rows, copied into
+//     shared memory by a bulk copy, and the number of 64-token stages) in a
+//     small ring, and appends one (page, head, sub-tile, valid tokens) entry
+//     per stage to an entry ring;
+//   * copy thread: pops entries and streams the selected K and V tiles with
+//     4-D TMA loads (64 tokens x 64 dims per box, 128-byte swizzle, L2
+//     evict-first, no multicast) into an NSTAGES-deep ring of 32 KB stages
+//     whose per-stage metadata (valid tokens) rides along;
+//   * two groups of four math warps take alternate stages; each warp owns 16
+//     tokens of a stage and never touches global memory in the loop.  The
+//     tensor-core tile is "swap-AB": S^T = K q^T with the 16 tokens as M and
+//     the query heads as N (8 per n-tile), O^T += V^T P^T with head_dim as M,
+//     so a GQA group of G <= 8 heads costs one n-tile.  K and V fragments are
+//     read with ldmatrix (conflict-free thanks to the swizzle) and the stage is
+//     handed back to the copy thread before the softmax and P.V math;
+//   * online softmax per head column in the exp2 domain; P^T enters the
+//     tensor cores through movmatrix as a bf16 hi + lo pair (weights kept to
+//     ~16 bits); tail tokens past seqlen are masked in registers;
+//   * at the end of an item the 8 warps merge (m, l, O) through shared memory
+//     and write o_part / lse_part.
 // Every mbarrier wait is bounded (SEER_DEV_TIMEOUT); nothing traps.
 #include "seer_kernels.cuh"
 
@@ -29,342 +36,575 @@ namespace seer {
 
 constexpr int kHalfTileBytes = kTileTokens * 64 * 2;  // 64 tokens x 64 dims bf16
 constexpr int kStageBytes = 4 * kHalfTileBytes;       // K lo, K hi, V lo, V hi
+constexpr int kItemSlots = 3;
+constexpr int kOStride = kHeadDim + 4;                 // padded merge row (floats)
+constexpr int kEntries = 256;                          // stage entries in flight (power of 2)
 
-template <int NGROUPS, int NSTAGES>
+template <int NT, int STAGES>
 struct DecodeShape {
-  static constexpr int kMathWarps = 4 * NGROUPS;
-  static constexpr int kThreads = (kMathWarps + 1) * 32;
-  static size_t smem_bytes(int G) {
-    return 1024 /* alignment slack */ + (size_t)NSTAGES * kStageBytes +
-           2 * NSTAGES * sizeof(uint64_t) + (size_t)kMathWarps * 2 * kMaxGroup * sizeof(float) +
-           (size_t)kMathWarps * G * kHeadDim * sizeof(float);
-  }
+  static constexpr int kMathWarps = 8;
+  static constexpr int kThreads = (kMathWarps + 2) * 32;  // + copy warp + scheduler warp
+  static constexpr int kGroups = 2;
+  // Stage k goes to group k % kGroups and slot k % kStages.  The ring depth
+  // must be a multiple of the group count so that every slot is always
+  // consumed by the same group: a group then never waits on a slot two
+  // phases ahead of it (a parity wait cannot tell phase k from k + 2).
+  static constexpr int kStages = STAGES;
+  static_assert(kStages % kGroups == 0, "each ring slot must belong to one group");
+  static constexpr int kQSlotBytes = NT * 8 * kHeadDim * 2;  // the group's query rows
+  // shared memory carve (offsets from the 1024-aligned base)
+  static constexpr size_t kRing = 0;
+  static constexpr size_t kQBuf = kRing + (size_t)kStages * kStageBytes;
+  static constexpr size_t kBars = kQBuf + (size_t)kItemSlots * kQSlotBytes;
+  static constexpr size_t kMeta = kBars + 8 * (2 * kStages + 2 * kItemSlots);
+  static constexpr size_t kRec = (kMeta + 4 * kStages + 15) & ~size_t(15);
+  static constexpr size_t kEnt = (kRec + 8 * kItemSlots + 15) & ~size_t(15);
+  static constexpr size_t kEntCtl = kEnt + 8 * kEntries;  // tail, head
+  static constexpr size_t kML = kEntCtl + 16;
+  static constexpr size_t kO = kML + (size_t)kMathWarps * 2 * kMaxGroup * 4;
+  static size_t smem_bytes(int G) { return 1024 + kO + (size_t)kMathWarps * G * kOStride * 4; }
+  static_assert(kRing % 1024 == 0 && kStageBytes % 1024 == 0, "swizzled TMA tiles need 1 KB");
+  static_assert(kQBuf % 16 == 0 && kQSlotBytes % 16 == 0, "bulk copy destinations need 16 B");
+  static_assert(kBars % 8 == 0 && kRec % 8 == 0 && kEnt % 16 == 0 && kML % 16 == 0 &&
+                    kO % 16 == 0,
+                "shared-memory carve alignment");
 };
 
-// One work item: (b, h, split s) and the slice [lo, hi) of its index row.
-struct Item {
+__device__ __forceinline__ uint32_t ld_volatile(const uint32_t* p) {
+  return *reinterpret_cast<const volatile uint32_t*>(p);
+}
+
+__device__ __forceinline__ void st_volatile(uint32_t* p, uint32_t v) {
+  *reinterpret_cast<volatile uint32_t*>(p) = v;
+}
+
+struct ItemCoord {
   int b, h, s, L, nb, lo, hi;
+  int64_t row;  // offset of the (b, h) index row
 };
 
-__device__ __forceinline__ Item decode_item(const DecodeParams& p, int item) {
-  Item it;
+__device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item, int L, int n) {
+  ItemCoord c;
   const int bh = item / p.S;
-  it.s = item - bh * p.S;
-  it.b = bh / p.Hkv;
-  it.h = bh - it.b * p.Hkv;
-  int L = __ldg(p.seqlens + it.b);
-  L = max(0, min(L, p.max_blocks * p.bs));
-  it.L = L;
-  it.nb = ceil_div_i(L, p.bs);
-  int n = __ldg(p.n_sel + bh);
+  c.s = item - bh * p.S;
+  c.b = bh / p.Hkv;
+  c.h = bh - c.b * p.Hkv;
+  c.L = max(0, min(L, p.max_blocks * p.bs));
+  c.nb = ceil_div_i(c.L, p.bs);
   n = max(0, min(n, p.k_max));
-  it.lo = (int)(((long long)it.s * n) / p.S);
-  it.hi = (int)(((long long)(it.s + 1) * n) / p.S);
-  return it;
+  c.lo = (int)(((long long)c.s * n) / p.S);
+  c.hi = (int)(((long long)(c.s + 1) * n) / p.S);
+  c.row = (int64_t)bh * p.k_max;
+  return c;
 }
 
-// Block index i of the item's row, or -1 if it is not a valid block.
-__device__ __forceinline__ int block_at(const DecodeParams& p, const Item& it, int i) {
-  const int j = __ldg(p.idx + (int64_t)(it.b * p.Hkv + it.h) * p.k_max + i);
-  return (j >= 0 && j < it.nb) ? j : -1;
-}
-
-template <int NGROUPS, int NSTAGES>
-__global__ void __launch_bounds__(DecodeShape<NGROUPS, NSTAGES>::kThreads, 1)
+template <int NT, int STAGES>
+__global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  using Shape = DecodeShape<NGROUPS, NSTAGES>;
+  using Shape = DecodeShape<NT, STAGES>;
+  constexpr int kStages = Shape::kStages;
+  constexpr int kQSlotBytes = Shape::kQSlotBytes;
   constexpr int kMathWarps = Shape::kMathWarps;
   constexpr int kMathThreads = kMathWarps * 32;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(ring + NSTAGES * kStageBytes);
-  uint64_t* empty_bar = full_bar + NSTAGES;
-  float* m_sh = reinterpret_cast<float*>(empty_bar + NSTAGES);  // [warps][16]
-  float* l_sh = m_sh + kMathWarps * kMaxGroup;                   // [warps][16]
-  float* o_sh = l_sh + kMathWarps * kMaxGroup;                   // [warps][G][128]
+  uint8_t* ring = smem + Shape::kRing;
+  uint8_t* qbuf = smem + Shape::kQBuf;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Shape::kBars);
+  uint64_t* empty_bar = full_bar + kStages;
+  uint64_t* item_full = empty_bar + kStages;
+  uint64_t* item_empty = item_full + kItemSlots;
+  int* stage_valid = reinterpret_cast<int*>(smem + Shape::kMeta);
+  int2* item_rec = reinterpret_cast<int2*>(smem + Shape::kRec);  // (item, stages)
+  int2* ent = reinterpret_cast<int2*>(smem + Shape::kEnt);  // (page, h | sub | valid)
+  uint32_t* ent_tail = reinterpret_cast<uint32_t*>(smem + Shape::kEntCtl);
+  uint32_t* ent_head = ent_tail + 1;
+  float* m_sh = reinterpret_cast<float*>(smem + Shape::kML);  // [warps][16]
+  float* l_sh = m_sh + kMathWarps * kMaxGroup;                 // [warps][16]
+  float* o_sh = reinterpret_cast<float*>(smem + Shape::kO);    // [warps][G][kOStride]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int G = p.G;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NSTAGES; ++i) {
+    *ent_tail = 0;
+    *ent_head = 0;
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&full_bar[i], 1);
       mbar_init(&empty_bar[i], 4);
+    }
+    for (int i = 0; i < kItemSlots; ++i) {
+      mbar_init(&item_full[i], 1);
+      mbar_init(&item_empty[i], kMathWarps);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kMathWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane != 0) return;
-    prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
-    const uint64_t policy = policy_evict_first();
-    uint32_t issued = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < p.num_items && ok; item += gridDim.x) {
-      const Item it = decode_item(p, item);
-      for (int i = it.lo; i < it.hi && ok; ++i) {
-        const int j = block_at(p, it, i);
-        if (j < 0) {
-          flag_status(p.status, SEER_DEV_BAD_INDEX);
-          continue;
+  if (warp == kMathWarps + 1) {
+    // =============================================================== scheduler
+    // Runs ahead of the copies: resolves each item's block indices and pages
+    // (lane-parallel, dependent global loads off the copy path), publishes
+    // the item record + query rows, and appends one entry per 64-token stage
+    // to the entry ring read by the copy thread.
+    int ok = 1;
+    uint32_t tail = 0;
+    int item = blockIdx.x;
+    int L_cur = 0, n_cur = 0;
+    if (item < p.num_items) {
+      const int bh = item / p.S;
+      L_cur = __ldg(p.seqlens + bh / p.Hkv);
+      n_cur = __ldg(p.n_sel + bh);
+    }
+    for (int it_no = 0; item < p.num_items && ok; item += gridDim.x, ++it_no) {
+      const int nxt = item + gridDim.x;  // next item's length and count, in flight
+      int L_nxt = 0, n_nxt = 0;
+      if (nxt < p.num_items) {
+        const int bh = nxt / p.S;
+        L_nxt = __ldg(p.seqlens + bh / p.Hkv);
+        n_nxt = __ldg(p.n_sel + bh);
+      }
+      const ItemCoord ic = item_coord(p, item, L_cur, n_cur);
+
+      // stages of this item (the first 32 indices stay in registers)
+      int j0 = -1, nst = 0;
+      for (int base = ic.lo; base < ic.hi; base += 32) {
+        const int i = base + lane;
+        int cnt = 0;
+        if (i < ic.hi) {
+          const int j = __ldg(p.idx + ic.row + i);
+          if (j >= 0 && j < ic.nb) cnt = ceil_div_i(min(p.bs, ic.L - j * p.bs), kTileTokens);
+          if (base == ic.lo) j0 = j;
         }
-        int64_t page = page_of(p.page_table, it.b, j, p.max_blocks);
-        if (page < 0 || page >= p.num_pages) {
-          flag_status(p.status, SEER_DEV_BAD_PAGE);
-          page = 0;  // keep the copy inside the pool; the result is flagged
-        }
-        for (int sub = 0; sub < p.bs / kTileTokens; ++sub) {
-          const int tok0 = j * p.bs + sub * kTileTokens;
-          if (tok0 >= it.L) break;
-          const int slot = issued % NSTAGES;
-          const uint32_t phase = (issued / NSTAGES) & 1;
-          if (!mbar_wait(&empty_bar[slot], phase ^ 1)) {
-            flag_status(p.status, SEER_DEV_TIMEOUT);
-            ok = false;
-            break;
-          }
-          uint8_t* st = ring + slot * kStageBytes;
-          mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
-          const int t = sub * kTileTokens;
-          const int c1 = p.token_inner ? t : it.h;
-          const int c2 = p.token_inner ? it.h : t;
-          const int pg = (int)page;
-          tma_load_4d(st + 0 * kHalfTileBytes, &tm_k, 0, c1, c2, pg, &full_bar[slot], policy);
-          tma_load_4d(st + 1 * kHalfTileBytes, &tm_k, 64, c1, c2, pg, &full_bar[slot], policy);
-          tma_load_4d(st + 2 * kHalfTileBytes, &tm_v, 0, c1, c2, pg, &full_bar[slot], policy);
-          tma_load_4d(st + 3 * kHalfTileBytes, &tm_v, 64, c1, c2, pg, &full_bar[slot], policy);
-          ++issued;
+        nst += __reduce_add_sync(0xffffffffu, cnt);
+      }
+
+      // item record + query rows
+      const int islot = it_no % kItemSlots;
+      const uint32_t iphase = (it_no / kItemSlots) & 1;
+      if (lane == 0) {
+        if (!mbar_wait(&item_empty[islot], iphase ^ 1)) {
+          flag_status(p.status, SEER_DEV_TIMEOUT);
+          ok = 0;
+        } else {
+          item_rec[islot] = make_int2(item, nst);
+          const uint32_t qbytes = (uint32_t)(G * kHeadDim * 2);
+          mbar_arrive_expect_tx(&item_full[islot], qbytes);
+          bulk_copy_g2s(qbuf + islot * kQSlotBytes,
+                        p.q + ((int64_t)ic.b * p.Hq + (int64_t)ic.h * G) * kHeadDim, qbytes,
+                        &item_full[islot]);
         }
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+
+      // one entry per stage: (page, h | sub-tile | valid tokens)
+      for (int base = ic.lo; base < ic.hi && ok; base += 32) {
+        const int i = base + lane;
+        int j = -1, pg = 0, ne = 0;
+        if (i < ic.hi) {
+          j = (base == ic.lo) ? j0 : __ldg(p.idx + ic.row + i);
+          if (j < 0 || j >= ic.nb) {
+            flag_status(p.status, SEER_DEV_BAD_INDEX);
+            j = -1;
+          } else {
+            const int64_t page = page_of(p.page_table, ic.b, j, p.max_blocks);
+            if (page < 0 || page >= p.num_pages) {
+              flag_status(p.status, SEER_DEV_BAD_PAGE);
+              pg = 0;  // keep the copy inside the pool; the result is flagged
+            } else {
+              pg = (int)page;
+            }
+            ne = ceil_div_i(min(p.bs, ic.L - j * p.bs), kTileTokens);
+          }
+        }
+        int incl = ne;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (lane == 0) {  // wait for room in the entry ring
+          const long long t0 = clock64();
+          while (tail + (uint32_t)total - ld_volatile(ent_head) > (uint32_t)kEntries) {
+            if (clock64() - t0 > (1ll << 31)) {
+              flag_status(p.status, SEER_DEV_TIMEOUT);
+              ok = 0;
+              break;
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        for (int e = 0; e < ne; ++e) {
+          const int t = e * kTileTokens;
+          const int valid = min(kTileTokens, ic.L - (j * p.bs + t));
+          ent[(tail + incl - ne + e) & (kEntries - 1)] =
+              make_int2(pg, (ic.h << 16) | (e << 8) | valid);
+        }
+        tail += (uint32_t)total;
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          st_volatile(ent_tail, tail);
+        }
+        __syncwarp();
+      }
+      L_cur = L_nxt;
+      n_cur = n_nxt;
     }
-    // Let every copy this CTA started land before the CTA can retire.
-    for (uint32_t k = 0; k < NSTAGES && k < issued; ++k) {
-      const uint32_t s_it = issued - 1 - k;
-      mbar_wait(&full_bar[s_it % NSTAGES], (s_it / NSTAGES) & 1);
+    // terminator (the copy thread stops on a negative page)
+    if (lane == 0) {
+      const long long t0 = clock64();
+      bool room = true;
+      while (tail + 1u - ld_volatile(ent_head) > (uint32_t)kEntries) {
+        if (clock64() - t0 > (1ll << 31)) {
+          flag_status(p.status, SEER_DEV_TIMEOUT);
+          room = false;
+          break;
+        }
+      }
+      if (room) {
+        ent[tail & (kEntries - 1)] = make_int2(-1, 0);
+        __threadfence_block();
+        st_volatile(ent_tail, tail + 1u);
+      }
     }
     return;
   }
 
-  // -------------------------------------------------------------- math warps
-  const int group = warp / 4;
-  const int wq = warp % 4;         // which 16 tokens of a tile
-  const int r = lane >> 2;         // fragment row (query head) r and r + 8
-  const int c = lane & 3;          // fragment column pair
-  const int G = p.G;
-  uint32_t stage_iter = 0;
+  if (warp == kMathWarps) {
+    // ============================================================ copy thread
+    if (lane != 0) return;
+    const uint64_t policy = policy_evict_first();
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    uint32_t head = 0, issued = 0;
+    for (;;) {
+      if (ld_volatile(ent_tail) == head) {  // wait for the scheduler
+        const long long t0 = clock64();
+        bool timed_out = false;
+        while (ld_volatile(ent_tail) == head) {
+          __nanosleep(32);
+          if (clock64() - t0 > (1ll << 31)) {
+            timed_out = true;
+            break;
+          }
+        }
+        if (timed_out) {
+          flag_status(p.status, SEER_DEV_TIMEOUT);
+          break;
+        }
+      }
+      __threadfence_block();
+      const int2 e = ent[head & (kEntries - 1)];
+      __threadfence_block();
+      st_volatile(ent_head, ++head);
+      if (e.x < 0) break;
+      const int slot = issued % kStages;
+      const uint32_t phase = (issued / kStages) & 1;
+      if (!mbar_wait(&empty_bar[slot], phase ^ 1)) {
+        flag_status(p.status, SEER_DEV_TIMEOUT);
+        break;
+      }
+      const int h = (int)((uint32_t)e.y >> 16);
+      const int t = ((e.y >> 8) & 0xff) * kTileTokens;
+      stage_valid[slot] = e.y & 0xff;
+      uint8_t* st = ring + slot * kStageBytes;
+      mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
+      const int c1 = p.token_inner ? t : h;
+      const int c2 = p.token_inner ? h : t;
+      tma_load_4d(st + 0 * kHalfTileBytes, &tm_k, 0, c1, c2, e.x, &full_bar[slot], policy);
+      tma_load_4d(st + 1 * kHalfTileBytes, &tm_k, 64, c1, c2, e.x, &full_bar[slot], policy);
+      tma_load_4d(st + 2 * kHalfTileBytes, &tm_v, 0, c1, c2, e.x, &full_bar[slot], policy);
+      tma_load_4d(st + 3 * kHalfTileBytes, &tm_v, 64, c1, c2, e.x, &full_bar[slot], policy);
+      ++issued;
+    }
+    // Let every copy this CTA started land before the CTA can retire.
+    for (uint32_t k = 0; k < kStages && k < issued; ++k) {
+      const uint32_t s_it = issued - 1 - k;
+      mbar_wait(&full_bar[s_it % kStages], (s_it / kStages) & 1);
+    }
+    return;
+  }
+
+  // ================================================================== math
+  const int group = warp >> 2;  // kMathWarps / 4 == kGroups
+  const int wq = warp & 3;   // which 16 tokens of a stage
+  const int r = lane >> 2;   // fragment row group
+  const int c = lane & 3;    // fragment column pair
+  const int mi = lane >> 3;  // ldmatrix sub-matrix this lane addresses
+  uint32_t stage_base = 0;
   bool ok = true;
 
-  for (int item = blockIdx.x; item < p.num_items; item += gridDim.x) {
-    const Item it = decode_item(p, item);
+  for (int item = blockIdx.x, it_no = 0; item < p.num_items; item += gridDim.x, ++it_no) {
+    const int islot = it_no % kItemSlots;
+    const uint32_t iphase = (it_no / kItemSlots) & 1;
+    if (ok && !mbar_wait(&item_full[islot], iphase)) {
+      flag_status(p.status, SEER_DEV_TIMEOUT);
+      ok = false;
+    }
+    const int nst = ok ? item_rec[islot].y : 0;
 
-    // Q fragments: rows = the group's query heads (zero past G), 8 k-steps.
-    uint32_t qa[8][4];
+    // q^T fragments (B operand of S^T = K q^T): n = head, k = dim.
+    uint32_t qb[NT][8][2];
     {
-      const uint16_t* qrow0 = p.q + ((int64_t)it.b * p.Hq + (int64_t)it.h * G + r) * kHeadDim;
-      const uint16_t* qrow1 = qrow0 + 8 * kHeadDim;
+      const uint32_t qs = smem_u32(qbuf + islot * kQSlotBytes);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int d0 = kk * 16 + 2 * c;
-        qa[kk][0] = (r < G) ? __ldg(reinterpret_cast<const uint32_t*>(qrow0 + d0)) : 0u;
-        qa[kk][1] = (r + 8 < G) ? __ldg(reinterpret_cast<const uint32_t*>(qrow1 + d0)) : 0u;
-        qa[kk][2] = (r < G) ? __ldg(reinterpret_cast<const uint32_t*>(qrow0 + d0 + 8)) : 0u;
-        qa[kk][3] = (r + 8 < G) ? __ldg(reinterpret_cast<const uint32_t*>(qrow1 + d0 + 8)) : 0u;
+      for (int nt = 0; nt < NT; ++nt) {
+        const int head = nt * 8 + (lane & 7);
+        const bool live = nt * 8 + r < G;
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp) {
+          // 4 matrices: 8 head rows x dim chunks 4kp .. 4kp+3 (two k-steps)
+          const uint32_t addr = qs + head * (kHeadDim * 2) + (4 * kp + mi) * 16;
+          uint32_t x0, x1, x2, x3;
+          ldmatrix_x4(addr, x0, x1, x2, x3);
+          qb[nt][2 * kp][0] = live ? x0 : 0u;
+          qb[nt][2 * kp][1] = live ? x1 : 0u;
+          qb[nt][2 * kp + 1][0] = live ? x2 : 0u;
+          qb[nt][2 * kp + 1][1] = live ? x3 : 0u;
+        }
       }
     }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[islot]);
 
-    float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 domain) of rows r, r+8
-    float l0 = 0.f, l1 = 0.f;              // this thread's share of the row sums
-    float o[16][4];
+    float m[NT][2], l[NT][2];
+    float o[8][NT][4];
 #pragma unroll
-    for (int nd = 0; nd < 16; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+    }
 
-    for (int i = it.lo; i < it.hi; ++i) {
-      const int j = block_at(p, it, i);
-      if (j < 0) continue;
-      for (int sub = 0; sub < p.bs / kTileTokens; ++sub) {
-        const int tok0 = j * p.bs + sub * kTileTokens;
-        if (tok0 >= it.L) break;
-        const uint32_t my_iter = stage_iter++;
-        if ((int)(my_iter % NGROUPS) != group) continue;
-        const int slot = my_iter % NSTAGES;
-        const uint32_t phase = (my_iter / NSTAGES) & 1;
-        if (ok && !mbar_wait(&full_bar[slot], phase)) {
-          flag_status(p.status, SEER_DEV_TIMEOUT);
-          ok = false;
-        }
-        if (ok) {
-          const uint32_t k_base = smem_u32(ring + slot * kStageBytes);
-          const uint32_t v_base = k_base + 2 * kHalfTileBytes;
-          const int valid = it.L - tok0;  // >= 1; < 64 only on the newest tile
-
-          // ---- S = Q K^T for this warp's 16 tokens (2 n-tiles of 8)
-          float s[2][4];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-            const int tok = wq * 16 + nt * 8 + (lane & 7);
-            const int mi = lane >> 3;
-#pragma unroll
-            for (int kp = 0; kp < 4; ++kp) {
-              const int half = kp >> 1;
-              const int chunk = (kp & 1) * 4 + mi;
-              const uint32_t addr = k_base + half * kHalfTileBytes + tok * 128 +
-                                    ((chunk ^ (tok & 7)) << 4);
-              uint32_t b0, b1, b2, b3;
-              ldmatrix_x4(addr, b0, b1, b2, b3);
-              mma_bf16_16816(s[nt], qa[2 * kp], b0, b1);
-              mma_bf16_16816(s[nt], qa[2 * kp + 1], b2, b3);
-            }
-          }
-          // ---- scale, mask tokens past the sequence end, online softmax
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            const int t_rel = wq * 16 + nt * 8 + 2 * c;
-            const bool v0 = t_rel < valid, v1 = t_rel + 1 < valid;
-            s[nt][0] = v0 ? s[nt][0] * p.scale_log2 : -INFINITY;
-            s[nt][1] = v1 ? s[nt][1] * p.scale_log2 : -INFINITY;
-            s[nt][2] = v0 ? s[nt][2] * p.scale_log2 : -INFINITY;
-            s[nt][3] = v1 ? s[nt][3] * p.scale_log2 : -INFINITY;
-          }
-          float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-          float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-          const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
-          const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-          const float a0 = fast_exp2(m0 - mu0), a1 = fast_exp2(m1 - mu1);
-          m0 = mn0;
-          m1 = mn1;
-          float pr[2][4];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            pr[nt][0] = fast_exp2(s[nt][0] - mu0);
-            pr[nt][1] = fast_exp2(s[nt][1] - mu0);
-            pr[nt][2] = fast_exp2(s[nt][2] - mu1);
-            pr[nt][3] = fast_exp2(s[nt][3] - mu1);
-          }
-          l0 = l0 * a0 + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
-          l1 = l1 * a1 + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
-#pragma unroll
-          for (int nd = 0; nd < 16; ++nd) {
-            o[nd][0] *= a0;
-            o[nd][1] *= a0;
-            o[nd][2] *= a1;
-            o[nd][3] *= a1;
-          }
-          // P as a bf16 pair hi + lo (hi = RNE(p), lo = RNE(p - hi)): the
-          // product P V then carries p to ~2^-16 instead of bf16's 2^-9, so
-          // heavy-tailed V rows do not amplify the rounding of the weights.
-          uint32_t pa[4], pl[4];
-          split_bf16x2(pr[0][0], pr[0][1], pa[0], pl[0]);
-          split_bf16x2(pr[0][2], pr[0][3], pa[1], pl[1]);
-          split_bf16x2(pr[1][0], pr[1][1], pa[2], pl[2]);
-          split_bf16x2(pr[1][2], pr[1][3], pa[3], pl[3]);
-
-          // ---- O += P V (V tile rows past the end are zeroed in registers:
-          // their P is 0 but the slot may hold anything, NaN included)
-          uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
-          if (valid < kTileTokens) {
-            const int t0 = wq * 16 + 2 * c, t1 = t0 + 8;
-            vmask_lo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
-            vmask_hi = (t1 < valid ? 0x0000ffffu : 0u) | (t1 + 1 < valid ? 0xffff0000u : 0u);
-          }
-          const int mi = lane >> 3;
-          const int vtok = wq * 16 + (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-          for (int dp = 0; dp < 8; ++dp) {
-            const int half = dp >> 2;
-            const int chunk = (dp & 3) * 2 + (mi >> 1);
-            const uint32_t addr = v_base + half * kHalfTileBytes + vtok * 128 +
-                                  ((chunk ^ (vtok & 7)) << 4);
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4_trans(addr, b0, b1, b2, b3);
-            b0 &= vmask_lo;
-            b1 &= vmask_hi;
-            b2 &= vmask_lo;
-            b3 &= vmask_hi;
-            mma_bf16_16816(o[2 * dp], pa, b0, b1);
-            mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
-            mma_bf16_16816(o[2 * dp], pl, b0, b1);
-            mma_bf16_16816(o[2 * dp + 1], pl, b2, b3);
-          }
-        }
+    for (int k = 0; k < nst; ++k) {
+      const uint32_t gi = stage_base + k;
+      if ((int)(gi % Shape::kGroups) != group) continue;
+      const int slot = gi % kStages;
+      const uint32_t phase = (gi / kStages) & 1;
+      if (ok && !mbar_wait(&full_bar[slot], phase)) {
+        flag_status(p.status, SEER_DEV_TIMEOUT);
+        ok = false;
+      }
+      if (!ok) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[slot]);
-      }
-    }
-
-    // ---- merge the math warps' partial softmax states for this item
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    if (c == 0) {
-      m_sh[warp * kMaxGroup + r] = m0;
-      l_sh[warp * kMaxGroup + r] = l0;
-      m_sh[warp * kMaxGroup + r + 8] = m1;
-      l_sh[warp * kMaxGroup + r + 8] = l1;
-    }
-    float* ow = o_sh + (size_t)warp * G * kHeadDim;
-#pragma unroll
-    for (int nd = 0; nd < 16; ++nd) {
-      const int d = nd * 8 + 2 * c;
-      if (r < G) *reinterpret_cast<float2*>(ow + r * kHeadDim + d) = make_float2(o[nd][0], o[nd][1]);
-      if (r + 8 < G)
-        *reinterpret_cast<float2*>(ow + (r + 8) * kHeadDim + d) = make_float2(o[nd][2], o[nd][3]);
-    }
-    named_barrier_sync(1, kMathThreads);
-    for (int e = threadIdx.x; e < G * kHeadDim; e += kMathThreads) {
-      const int g = e / kHeadDim, d = e - g * kHeadDim;
-      float mt = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kMathWarps; ++w) mt = fmaxf(mt, m_sh[w * kMaxGroup + g]);
-      const int64_t row = ((int64_t)it.b * p.Hq + (int64_t)it.h * G + g) * p.S + it.s;
-      if (mt == -INFINITY) {
-        p.o_part[row * kHeadDim + d] = 0.f;
-        if (d == 0) p.lse_part[row] = -INFINITY;
         continue;
       }
-      float lt = 0.f, acc = 0.f;
+      const int valid = stage_valid[slot];
+      const uint32_t k_base = smem_u32(ring + slot * kStageBytes);
+      const uint32_t v_base = k_base + 2 * kHalfTileBytes;
+
+      // ---- S^T = K q^T over this warp's 16 tokens (two chains of 4 k-steps)
+      float sacc[NT][2][4];
 #pragma unroll
-      for (int w = 0; w < kMathWarps; ++w) {
-        const float f = fast_exp2(m_sh[w * kMaxGroup + g] - mt);
-        lt += l_sh[w * kMaxGroup + g] * f;
-        acc += o_sh[((size_t)w * G + g) * kHeadDim + d] * f;
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+          sacc[nt][a][0] = sacc[nt][a][1] = sacc[nt][a][2] = sacc[nt][a][3] = 0.f;
+      {
+        const int tok = wq * 16 + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int chunk = 2 * kk + (mi >> 1);  // 16-byte chunk of the 128 dims
+          const uint32_t addr = k_base + (chunk >> 3) * kHalfTileBytes + tok * 128 +
+                                (((chunk & 7) ^ (tok & 7)) << 4);
+          uint32_t a[4];
+          ldmatrix_x4(addr, a[0], a[1], a[2], a[3]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_bf16_16816(sacc[nt][kk & 1], a, qb[nt][kk][0], qb[nt][kk][1]);
+        }
       }
-      p.o_part[row * kHeadDim + d] = acc / lt;
-      if (d == 0) p.lse_part[row] = (mt + log2f(lt)) * kLn2;
+      // ---- V^T fragments (A operand of O^T += V^T P^T), then hand the stage back
+      uint32_t va[8][4];
+      {
+        const int tok = wq * 16 + (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int chunk = 2 * mt + (mi & 1);
+          const uint32_t addr = v_base + (chunk >> 3) * kHalfTileBytes + tok * 128 +
+                                (((chunk & 7) ^ (tok & 7)) << 4);
+          ldmatrix_x4_trans(addr, va[mt][0], va[mt][1], va[mt][2], va[mt][3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[slot]);
+
+      // ---- tokens past the sequence end (only on the newest tile)
+      const int t0 = wq * 16 + r;  // token of S^T rows r and r + 8
+      const bool in0 = t0 < valid, in1 = t0 + 8 < valid;
+      if (valid < kTileTokens) {
+        const int u = wq * 16 + 2 * c;  // tokens of the V^T fragment columns
+        const uint32_t mlo = (u < valid ? 0x0000ffffu : 0u) | (u + 1 < valid ? 0xffff0000u : 0u);
+        const uint32_t mhi =
+            (u + 8 < valid ? 0x0000ffffu : 0u) | (u + 9 < valid ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          va[mt][0] &= mlo;
+          va[mt][1] &= mlo;
+          va[mt][2] &= mhi;
+          va[mt][3] &= mhi;
+        }
+      }
+
+      // ---- online softmax per head column, P^T fragments via movmatrix
+      uint32_t pb[NT][4];  // hi b0, hi b1, lo b0, lo b1
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = sacc[nt][0][e] + sacc[nt][1][e];
+        x[0] = in0 ? x[0] * p.scale_log2 : -INFINITY;
+        x[1] = in0 ? x[1] * p.scale_log2 : -INFINITY;
+        x[2] = in1 ? x[2] * p.scale_log2 : -INFINITY;
+        x[3] = in1 ? x[3] * p.scale_log2 : -INFINITY;
+        float pr[4];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float mx = fmaxf(x[e], x[2 + e]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float mn = fmaxf(m[nt][e], mx);
+          const float mu = (mn == -INFINITY) ? 0.f : mn;
+          const float alpha = fast_exp2(m[nt][e] - mu);
+          m[nt][e] = mn;
+          pr[e] = fast_exp2(x[e] - mu);
+          pr[2 + e] = fast_exp2(x[2 + e] - mu);
+          l[nt][e] = l[nt][e] * alpha + (pr[e] + pr[2 + e]);
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            o[mt][nt][e] *= alpha;
+            o[mt][nt][2 + e] *= alpha;
+          }
+        }
+        uint32_t h0, l0, h1, l1;
+        split_bf16x2(pr[0], pr[1], h0, l0);  // token r     : heads 2c, 2c+1
+        split_bf16x2(pr[2], pr[3], h1, l1);  // token r + 8 : heads 2c, 2c+1
+        pb[nt][0] = movmatrix_trans(h0);
+        pb[nt][1] = movmatrix_trans(h1);
+        pb[nt][2] = movmatrix_trans(l0);
+        pb[nt][3] = movmatrix_trans(l1);
+      }
+
+      // ---- O^T += V^T P^T (hi and lo halves of P)
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_bf16_16816(o[mt][nt], va[mt], pb[nt][0], pb[nt][1]);
+          mma_bf16_16816(o[mt][nt], va[mt], pb[nt][2], pb[nt][3]);
+        }
+      }
+    }
+    stage_base += nst;
+
+    // ---- merge the 8 warps' partial softmax states of this item
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = l[nt][e];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        l[nt][e] = v;
+      }
+    }
+    if (r == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          m_sh[warp * kMaxGroup + nt * 8 + 2 * c + e] = m[nt][e];
+          l_sh[warp * kMaxGroup + nt * 8 + 2 * c + e] = l[nt][e];
+        }
+      }
+    }
+    float* ow = o_sh + (size_t)warp * G * kOStride;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int head = nt * 8 + 2 * c + e;
+        if (head < G) {
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            ow[head * kOStride + mt * 16 + r] = o[mt][nt][e];
+            ow[head * kOStride + mt * 16 + r + 8] = o[mt][nt][2 + e];
+          }
+        }
+      }
+    }
+    named_barrier_sync(1, kMathThreads);
+    {
+      const int bh = item / p.S;
+      const int s = item - bh * p.S;
+      const int b = bh / p.Hkv;
+      const int h = bh - b * p.Hkv;
+      for (int e = threadIdx.x; e < G * kHeadDim; e += kMathThreads) {
+        const int g = e / kHeadDim, d = e - g * kHeadDim;
+        float mt = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kMathWarps; ++w) mt = fmaxf(mt, m_sh[w * kMaxGroup + g]);
+        const int64_t orow = ((int64_t)b * p.Hq + (int64_t)h * G + g) * p.S + s;
+        if (mt == -INFINITY) {
+          p.o_part[orow * kHeadDim + d] = 0.f;
+          if (d == 0) p.lse_part[orow] = -INFINITY;
+          continue;
+        }
+        float lt = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMathWarps; ++w) {
+          const float f = fast_exp2(m_sh[w * kMaxGroup + g] - mt);
+          lt += l_sh[w * kMaxGroup + g] * f;
+          acc += o_sh[((size_t)w * G + g) * kOStride + d] * f;
+        }
+        p.o_part[orow * kHeadDim + d] = acc / lt;
+        if (d == 0) p.lse_part[orow] = (mt + log2f(lt)) * kLn2;
+      }
     }
     named_barrier_sync(1, kMathThreads);
   }
 }
 
 // ------------------------------------------------------------------ launcher
-template <int NGROUPS, int NSTAGES>
+template <int NT, int STAGES>
 static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
                                  const DecodeParams& p, int num_sms, cudaStream_t stream) {
-  using Shape = DecodeShape<NGROUPS, NSTAGES>;
+  using Shape = DecodeShape<NT, STAGES>;
   const size_t smem = Shape::smem_bytes(p.G);
-  auto kern = sparse_decode_kernel<NGROUPS, NSTAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = sparse_decode_kernel<NT, STAGES>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = p.num_items < num_sms ? p.num_items : num_sms;
   kern<<<grid, Shape::kThreads, smem, stream>>>(tk, tv, p);
   return cudaGetLastError();
 }
 
+// The deepest ring whose shared memory fits (the merge area grows with G).
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                               int num_sms, cudaStream_t stream) {
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    optin = 227 * 1024;
+  if (p.G <= 8) {
+    if (DecodeShape<1, 6>::smem_bytes(p.G) <= (size_t)optin)
+      return launch_decode<1, 6>(tk, tv, p, num_sms, stream);
+    return launch_decode<1, 4>(tk, tv, p, num_sms, stream);
+  }
   return launch_decode<2, 4>(tk, tv, p, num_sms, stream);
 }
 

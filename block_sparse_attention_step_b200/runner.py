@@ -26,8 +26,10 @@ class StepBuffers:
         self.device = dev
         B, Hkv, D = w.batch, w.kv_heads, w.head_dim
         self.nb_max = data["nb_max"]
+        from .workloads import pool_strides
+        sp, st, sh = pool_strides(data)
         self.dims = seer.make_dims(B, w.q_heads, Hkv, D, w.block_size, self.nb_max,
-                                   data["num_pages"])
+                                   data["num_pages"], sp, st, sh)
         self.budget = w.budget_tokens if budget_tokens is None else budget_tokens
         self.permille = w.sparsity_permille if sparsity_permille is None else sparsity_permille
         if self.budget is None and self.permille is None:

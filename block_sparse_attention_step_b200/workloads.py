@@ -125,11 +125,15 @@ def _draw_pool(w: Workload, num_pages: int, g, device):
     return pool
 
 
-def generate(w: Workload, seed: int, device="cpu") -> dict:
+def generate(w: Workload, seed: int, device="cpu", layout: str = "nhd") -> dict:
     """Draw one workload.  Returns a dict of tensors on ``device``:
-    q [B][Hq][D] bf16, w_gate [Hkv][D][D] f32, k_pool / v_pool [P][bs][Hkv][D]
-    bf16, page_table [B][NBmax] i32 (-1 past a sequence's last block),
-    seqlens [B] i32, plus ``nb_max`` and ``num_pages`` as ints."""
+    q [B][Hq][D] bf16, w_gate [Hkv][D][D] f32, k_pool / v_pool bf16 pages,
+    page_table [B][NBmax] i32 (-1 past a sequence's last block), seqlens [B]
+    i32, plus ``nb_max``, ``num_pages`` and ``layout`` ("nhd": pages
+    [P][bs][Hkv][D], token-major; "hnd": pages [P][Hkv][bs][D], head-major --
+    the same values, stored permuted)."""
+    if layout not in ("nhd", "hnd"):
+        raise ValueError(f"unknown layout {layout!r}")
     device = torch.device(device)
     g = torch.Generator(device=device)
     g.manual_seed(int(seed))
@@ -159,6 +163,9 @@ def generate(w: Workload, seed: int, device="cpu") -> dict:
     w_gate = torch.randn((w.kv_heads, D, D), generator=g, device=device) * (1.0 / D) ** 0.5
     k_pool = _draw_pool(w, num_pages, g, device)
     v_pool = _draw_pool(w, num_pages, g, device)
+    if layout == "hnd":
+        k_pool = k_pool.permute(0, 2, 1, 3).contiguous()
+        v_pool = v_pool.permute(0, 2, 1, 3).contiguous()
     return {
         "q": q.contiguous(),
         "w_gate": w_gate.float().contiguous(),
@@ -168,14 +175,27 @@ def generate(w: Workload, seed: int, device="cpu") -> dict:
         "seqlens": seqlens.to(torch.int32).contiguous(),
         "nb_max": int(nb_max),
         "num_pages": int(num_pages),
+        "layout": layout,
     }
 
 
+def pool_strides(data: dict):
+    """(stride_page, stride_token, stride_head) in elements of the pools."""
+    k = data["k_pool"]
+    if data.get("layout", "nhd") == "hnd":
+        return k.stride(0), k.stride(2), k.stride(1)
+    return k.stride(0), k.stride(1), k.stride(2)
+
+
 def gather_rows(pool: torch.Tensor, page_table: torch.Tensor, b: int, h: int,
-                seqlen: int, block_size: int) -> torch.Tensor:
+                seqlen: int, block_size: int, layout: str = "nhd") -> torch.Tensor:
     """Token-ordered rows [L][D] of KV head h of sequence b, copied to the
     host in the pool's dtype (a layout walk, no arithmetic)."""
     nb = _ceil_div(int(seqlen), block_size)
     pages = page_table[b, :nb].to(device=pool.device, dtype=torch.int64)
-    rows = pool.index_select(0, pages)[:, :, h, :].reshape(nb * block_size, -1)
-    return rows[:seqlen].cpu()
+    picked = pool.index_select(0, pages)
+    if layout == "nhd":                   # [P][bs][Hkv][D]
+        rows = picked[:, :, h, :]
+    else:                                 # [P][Hkv][bs][D]
+        rows = picked[:, h, :, :]
+    return rows.reshape(nb * block_size, -1)[:seqlen].cpu()

@@ -36,8 +36,8 @@ def row_inputs(w, data, b, h):
     G = w.group
     q = f64(data["q"][b, h * G:(h + 1) * G])
     Wg = f64(data["w_gate"][h])
-    K = f64(W.gather_rows(data["k_pool"], data["page_table"], b, h, L, w.block_size))
-    V = f64(W.gather_rows(data["v_pool"], data["page_table"], b, h, L, w.block_size))
+    K = f64(W.gather_rows(data["k_pool"], data["page_table"], b, h, L, w.block_size, data.get("layout", "nhd")))
+    V = f64(W.gather_rows(data["v_pool"], data["page_table"], b, h, L, w.block_size, data.get("layout", "nhd")))
     return q, Wg, K, V, L
 
 

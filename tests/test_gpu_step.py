@@ -208,3 +208,21 @@ def test_step_full_size_sampled(name, over):
             if run.force_newest:
                 assert row[-1] == nb - 1
     assert np.isfinite(f64(run.out)).all()
+
+
+def test_step_head_major_layout_is_bitwise_identical():
+    """The same drawn values stored head-major ([P][Hkv][bs][D]) give exactly
+    the token-major result: same tiles in shared memory, same sums."""
+    w = W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(batch=3, seqlen_range=(100, 3000))
+    outs = []
+    for layout in ("nhd", "hnd"):
+        data = W.generate(w, 21, DEV, layout=layout)
+        run = StepBuffers(w, data)
+        run.step(update_kbar=2)
+        run.step(update_kbar=1)
+        torch.cuda.synchronize()
+        assert run.status.item() == 0
+        v = run.workspace_views()
+        outs.append((run.out.clone(), run.lse.clone(), run.kbar.clone(), v["idx"].clone()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)

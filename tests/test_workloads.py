@@ -55,3 +55,18 @@ def test_offsets_shift_each_page_by_one_vector():
     t = _small("b16_h40_L32k_bs128_budget4k_newest", batch=1, seqlen=1024)
     d = W.generate(t, 2)
     assert torch.isfinite(d["k_pool"].float()).all()
+
+
+def test_head_major_layout_holds_the_same_values():
+    w = _small("b64_ragged_h64_paged_bs64", batch=3, seqlen_range=(10, 300))
+    a = W.generate(w, 4, layout="nhd")
+    b = W.generate(w, 4, layout="hnd")
+    assert b["k_pool"].shape == (a["num_pages"], 8, 64, 128)
+    assert W.pool_strides(b) == (8 * 64 * 128, 128, 64 * 128)
+    assert W.pool_strides(a) == (64 * 8 * 128, 8 * 128, 128)
+    for bb in range(3):
+        L = int(a["seqlens"][bb])
+        for h in (0, 7):
+            x = W.gather_rows(a["v_pool"], a["page_table"], bb, h, L, 64, "nhd")
+            y = W.gather_rows(b["v_pool"], b["page_table"], bb, h, L, 64, "hnd")
+            assert torch.equal(x, y)
