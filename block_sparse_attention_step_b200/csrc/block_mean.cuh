@@ -15,7 +15,8 @@ constexpr int kPoolWarps = 8;
 __device__ __forceinline__ float4 pool_warp_partial(const uint16_t* base_lane,
                                                     int64_t stride_token, int valid, int warp) {
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
+  // at most bs / 8 = 16 rows per warp: fully unrolled so every load is in flight
+#pragma unroll 16
   for (int t = warp; t < valid; t += kPoolWarps) {
     const uint2 v = __ldg(reinterpret_cast<const uint2*>(base_lane + (int64_t)t * stride_token));
     a0 += __uint_as_float(v.x << 16);

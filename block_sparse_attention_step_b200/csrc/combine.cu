@@ -3,51 +3,38 @@
 // Empty splits carry lse_s = -inf and weigh nothing; if every split is empty
 // the output is 0 and lse is -inf.
 //
-// One CTA of 128 threads (one per dim) per (b, query head).  The S weights are
-// computed once into shared memory; each thread then reads its dim of every
-// partial (coalesced 512-byte rows).
+// One CTA of 128 threads (one per dim) per (b, query head); each thread loads
+// the row's S lse values and its dim of every partial in one batch.  In the
+// whole step it is chained to the decode kernel by programmatic dependent
+// launch and waits for it in griddepcontrol.wait.
+#include "combine_core.cuh"
 #include "seer_kernels.cuh"
 
 namespace seer {
 
 __global__ void __launch_bounds__(kHeadDim) combine_kernel(const CombineParams p) {
-  __shared__ float w[kMaxSplits];
-  __shared__ float inv_total, lse_total;
+  pdl_wait();  // the partials come from the preceding decode grid
   const int64_t row = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;  // b * Hq + qh
-  const float* lse = p.lse_part + row * p.S;
-  if (threadIdx.x < 32) {
-    float m = -INFINITY;
-    for (int s = threadIdx.x; s < p.S; s += 32) m = fmaxf(m, __ldg(lse + s));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float tot = 0.f;
-    for (int s = threadIdx.x; s < p.S; s += 32) {
-      const float e = (m == -INFINITY) ? 0.f : expf(__ldg(lse + s) - m);
-      w[s] = e;
-      tot += e;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    if (threadIdx.x == 0) {
-      inv_total = tot > 0.f ? 1.f / tot : 0.f;
-      lse_total = tot > 0.f ? m + logf(tot) : -INFINITY;
-    }
-  }
-  __syncthreads();
-  const float* o = p.o_part + row * p.S * kHeadDim + threadIdx.x;
-  float acc = 0.f;
-  for (int s = 0; s < p.S; ++s) {
-    const float ws = w[s];
-    if (ws != 0.f) acc += ws * __ldg(o + (int64_t)s * kHeadDim);
-  }
-  const __nv_bfloat16 v = __float2bfloat16_rn(acc * inv_total);
-  p.out[row * kHeadDim + threadIdx.x] = *reinterpret_cast<const uint16_t*>(&v);
-  if (p.lse_out != nullptr && threadIdx.x == 0) p.lse_out[row] = lse_total;
+  const int d = threadIdx.x;
+  float lse;
+  const float v = combine_element(p.lse_part + row * p.S, p.o_part + row * p.S * kHeadDim + d,
+                                  p.S, &lse, LoadReadOnly{});
+  p.out[row * kHeadDim + d] = to_bf16_bits(v);
+  if (p.lse_out != nullptr && d == 0) p.lse_out[row] = lse;
 }
 
-cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream) {
-  dim3 grid(Hq, B);
-  combine_kernel<<<grid, kHeadDim, 0, stream>>>(p);
+cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(Hq, B);
+  cfg.blockDim = dim3(kHeadDim);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

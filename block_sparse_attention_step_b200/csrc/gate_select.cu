@@ -3,13 +3,12 @@
 // the gate-projected query and selects the top-k, without a round trip of
 // the scores through HBM and without two of the step's launches.
 //
-// Each CTA streams its kbar row (NB x 512 bytes) through two 64 KB shared-
+// Each CTA streams its kbar row (NB x 512 bytes) through three 64 KB shared-
 // memory buffers with bulk copies, issued before the gate projection
 // g = W qbar is formed so the projection hides under the first copies; the
 // newest block's mean is recomputed from K with the same summation order as
 // seer_pool_keys and written back; the scores (also written to the caller's
-// scores buffer) stay in shared memory for the exact radix select shared
-// with seer_block_select.  Results are identical to running seer_pool_keys
+// scores buffer) stay in shared memory for the exact one-pass binned top-k.  Results are identical to running seer_pool_keys
 // (incremental), seer_gate_scores and seer_block_select one after another.
 #include "block_mean.cuh"
 #include "seer_kernels.cuh"
@@ -21,15 +20,16 @@ constexpr int kGSThreads = 512;
 constexpr int kGSWarps = kGSThreads / 32;
 constexpr int kGSItems = kMaxBlocks / kGSThreads;  // 8
 constexpr int kGSChunkRows = 128;                  // kbar rows per buffer
+constexpr int kGSBuffers = 3;                      // 64 KB buffers in flight
 
 struct GateSelectSmem {
-  float buf[2][kGSChunkRows * kHeadDim];  // kbar rows in flight
+  float buf[kGSBuffers][kGSChunkRows * kHeadDim];  // kbar rows in flight
   float scores[kMaxBlocks];
   float part[kPoolWarps * kHeadDim];
   float newest[kHeadDim];
   float qbar[kHeadDim];
   float gvec[kHeadDim];
-  uint64_t bar[2];
+  uint64_t bar[kGSBuffers];
   SelectSmem sel;
 };
 
@@ -49,10 +49,17 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
   float* kb_row = p.kbar + bh * p.max_blocks * kHeadDim;
 
   if (tid == 0) {
-    mbar_init(&sm.bar[0], 1);
-    mbar_init(&sm.bar[1], 1);
+    for (int i = 0; i < kGSBuffers; ++i) mbar_init(&sm.bar[i], 1);
     fence_mbar_init();
-    for (int c = 0; c < 2 && c < nchunks; ++c) {
+  }
+  __syncthreads();
+  // Global memory is touched only from here on: wait for the preceding grid
+  // (it may have produced q), then let the decode grid start launching.
+  pdl_wait();
+  pdl_launch_dependents();
+  const int k_row = __ldg(p.k_per_seq + b);  // used at the end; loaded early
+  if (tid == 0) {
+    for (int c = 0; c < kGSBuffers && c < nchunks; ++c) {
       const uint32_t bytes = (uint32_t)min(kGSChunkRows, nb - c * kGSChunkRows) * kHeadDim * 4;
       mbar_arrive_expect_tx(&sm.bar[c], bytes);
       bulk_copy_g2s(sm.buf[c], kb_row + (int64_t)c * kGSChunkRows * kHeadDim, bytes, &sm.bar[c]);
@@ -74,6 +81,14 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
       *reinterpret_cast<float4*>(&sm.part[warp * kHeadDim + 4 * lane]) = a;
     }
   }
+  // this warp's rows of W[h], in flight while the mean query is formed
+  float4 wrow[kHeadDim / kGSWarps];
+  {
+    const float* W = p.w_gate + (int64_t)h * kHeadDim * kHeadDim;
+#pragma unroll
+    for (int r = 0; r < kHeadDim / kGSWarps; ++r)
+      wrow[r] = __ldg(reinterpret_cast<const float4*>(W + (warp + r * kGSWarps) * kHeadDim + 4 * lane));
+  }
   // mean query of the group, warps 8..11
   if (tid >= 256 && tid < 256 + kHeadDim) {
     const int d = tid - 256;
@@ -93,12 +108,10 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
   // g = gate_scale * W[h] qbar
   {
     const float4 qv = *reinterpret_cast<const float4*>(&sm.qbar[4 * lane]);
-    const float* W = p.w_gate + (int64_t)h * kHeadDim * kHeadDim;
 #pragma unroll
-    for (int row = warp; row < kHeadDim; row += kGSWarps) {
-      const float4 w = __ldg(reinterpret_cast<const float4*>(W + row * kHeadDim + 4 * lane));
-      const float v = warp_dot4(w, qv);
-      if (lane == 0) sm.gvec[row] = v * p.gate_scale;
+    for (int r = 0; r < kHeadDim / kGSWarps; ++r) {
+      const float v = warp_dot4(wrow[r], qv);
+      if (lane == 0) sm.gvec[warp + r * kGSWarps] = v * p.gate_scale;
     }
   }
   __syncthreads();
@@ -109,12 +122,13 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
   bool bad = false;
   bool ok = true;
   for (int c = 0; c < nchunks; ++c) {
-    if (ok && !mbar_wait(&sm.bar[c & 1], (c >> 1) & 1)) {
+    const int slot = c % kGSBuffers;
+    if (ok && !mbar_wait(&sm.bar[slot], (c / kGSBuffers) & 1)) {
       flag_status(p.status, SEER_DEV_TIMEOUT);
       ok = false;
     }
     const int rows = min(kGSChunkRows, nb - c * kGSChunkRows);
-    const float* buf = sm.buf[c & 1];
+    const float* buf = sm.buf[slot];
     for (int r = warp; r < rows; r += kGSWarps) {
       const int j = c * kGSChunkRows + r;
       const float4 v = (refresh && j == nb - 1)
@@ -129,30 +143,42 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
     }
     fence_proxy_async_smem();
     __syncthreads();  // every warp is done with this buffer
-    if (tid == 0 && ok && c + 2 < nchunks) {
-      const int cn = c + 2;
+    if (tid == 0 && ok && c + kGSBuffers < nchunks) {
+      const int cn = c + kGSBuffers;
       const uint32_t bytes = (uint32_t)min(kGSChunkRows, nb - cn * kGSChunkRows) * kHeadDim * 4;
-      mbar_arrive_expect_tx(&sm.bar[c & 1], bytes);
-      bulk_copy_g2s(sm.buf[c & 1], kb_row + (int64_t)cn * kGSChunkRows * kHeadDim, bytes,
-                   &sm.bar[c & 1]);
+      mbar_arrive_expect_tx(&sm.bar[slot], bytes);
+      bulk_copy_g2s(sm.buf[slot], kb_row + (int64_t)cn * kGSChunkRows * kHeadDim, bytes,
+                    &sm.bar[slot]);
     }
   }
   if (bad) flag_status(p.status, SEER_DEV_NONFINITE_SCORE);
   for (int j = nb + tid; j < p.max_blocks; j += kGSThreads) scores_out[j] = -INFINITY;
   __syncthreads();
 
-  select_topk<kGSThreads, kGSItems>(sm.scores, nb, __ldg(p.k_per_seq + b), p.force_newest,
-                                    p.k_max, p.idx + bh * p.k_max, p.n_sel + bh, p.status,
-                                    sm.sel);
+  // the kbar buffers are free now: the selection's member list lives there
+  select_topk_binned<kGSThreads, kGSItems>(sm.scores, nb, k_row, p.force_newest, p.k_max,
+                                           p.idx + bh * p.k_max, p.n_sel + bh, p.status, sm.sel,
+                                           reinterpret_cast<uint2*>(sm.buf[0]),
+                                           reinterpret_cast<int*>(sm.buf[1]));
 }
 
-cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream) {
+cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream, bool pdl) {
   const size_t smem = gate_select_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gate_select_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = ensure_smem_limit(gate_select_kernel, smem_set);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.Hkv, B);
-  gate_select_kernel<<<grid, kGSThreads, smem, stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.Hkv, B);
+  cfg.blockDim = dim3(kGSThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gate_select_kernel, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

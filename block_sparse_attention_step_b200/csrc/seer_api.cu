@@ -149,6 +149,54 @@ Workspace carve(const seer_dims* d, int32_t k_max, int32_t S, void* base) {
 
 }  // namespace
 
+struct DecodeLaunch {
+  CUtensorMap tk, tv;
+  DecodeParams p;
+};
+
+// Checks and tensor maps of a decode launch (nothing is enqueued).
+static seer_status decode_prepare(const seer_dims* d, const uint16_t* q, const uint16_t* k_pool,
+                                  const uint16_t* v_pool, const int32_t* page_table,
+                                  const int32_t* seqlens, const int32_t* idx,
+                                  const int32_t* n_sel, int32_t k_max, int32_t num_splits,
+                                  float softmax_scale, float* o_part, float* lse_part,
+                                  int32_t* dev_status, DecodeLaunch* L) {
+  SEER_TRY(check_dims(d));
+  SEER_TRY(check_pool(d, k_pool));
+  SEER_TRY(check_pool(d, v_pool));
+  if (!q || !seqlens || !idx || !n_sel || !o_part || !lse_part) return SEER_ERR_INVALID_ARG;
+  if (k_max < 1 || k_max > d->max_blocks || num_splits < 1 || num_splits > kMaxSplits)
+    return SEER_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(o_part, 8)) return SEER_ERR_UNSUPPORTED;
+  const int64_t items = (int64_t)d->batch * d->num_kv_heads * num_splits;
+  if (items > INT_MAX) return SEER_ERR_UNSUPPORTED;
+  const int token_inner = d->stride_token < d->stride_head ? 1 : 0;
+  SEER_TRY(make_kv_map(k_pool, d, token_inner, &L->tk));
+  SEER_TRY(make_kv_map(v_pool, d, token_inner, &L->tv));
+  DecodeParams& p = L->p;
+  p.q = q;
+  p.page_table = page_table;
+  p.seqlens = seqlens;
+  p.idx = idx;
+  p.n_sel = n_sel;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.status = dev_status;
+  p.B = d->batch;
+  p.Hq = d->num_q_heads;
+  p.Hkv = d->num_kv_heads;
+  p.G = d->num_q_heads / d->num_kv_heads;
+  p.bs = d->block_size;
+  p.max_blocks = d->max_blocks;
+  p.k_max = k_max;
+  p.S = num_splits;
+  p.num_items = (int)items;
+  p.token_inner = token_inner;
+  p.num_pages = d->num_pages;
+  p.scale_log2 = softmax_scale * kLog2e;
+  return SEER_OK;
+}
+
 extern "C" {
 
 int32_t seer_version(void) { return 10000; }
@@ -313,41 +361,10 @@ seer_status seer_sparse_decode(const seer_dims* d, const uint16_t* q, const uint
                                int32_t k_max, int32_t num_splits, float softmax_scale,
                                float* o_part, float* lse_part, int32_t* dev_status,
                                seer_stream stream) {
-  SEER_TRY(check_dims(d));
-  SEER_TRY(check_pool(d, k_pool));
-  SEER_TRY(check_pool(d, v_pool));
-  if (!q || !seqlens || !idx || !n_sel || !o_part || !lse_part) return SEER_ERR_INVALID_ARG;
-  if (k_max < 1 || k_max > d->max_blocks || num_splits < 1 || num_splits > kMaxSplits)
-    return SEER_ERR_INVALID_ARG;
-  if (!aligned(q, 4) || !aligned(o_part, 8)) return SEER_ERR_UNSUPPORTED;
-  const int64_t items = (int64_t)d->batch * d->num_kv_heads * num_splits;
-  if (items > INT_MAX) return SEER_ERR_UNSUPPORTED;
-  const int token_inner = d->stride_token < d->stride_head ? 1 : 0;
-  CUtensorMap tk, tv;
-  SEER_TRY(make_kv_map(k_pool, d, token_inner, &tk));
-  SEER_TRY(make_kv_map(v_pool, d, token_inner, &tv));
-  DecodeParams p;
-  p.q = q;
-  p.page_table = page_table;
-  p.seqlens = seqlens;
-  p.idx = idx;
-  p.n_sel = n_sel;
-  p.o_part = o_part;
-  p.lse_part = lse_part;
-  p.status = dev_status;
-  p.B = d->batch;
-  p.Hq = d->num_q_heads;
-  p.Hkv = d->num_kv_heads;
-  p.G = d->num_q_heads / d->num_kv_heads;
-  p.bs = d->block_size;
-  p.max_blocks = d->max_blocks;
-  p.k_max = k_max;
-  p.S = num_splits;
-  p.num_items = (int)items;
-  p.token_inner = token_inner;
-  p.num_pages = d->num_pages;
-  p.scale_log2 = softmax_scale * kLog2e;
-  SEER_CUDA(run_sparse_decode(tk, tv, p, num_sms_current(), stream));
+  DecodeLaunch L;
+  SEER_TRY(decode_prepare(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_max,
+                          num_splits, softmax_scale, o_part, lse_part, dev_status, &L));
+  SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, false));
   return SEER_OK;
 }
 
@@ -362,7 +379,7 @@ seer_status seer_combine(const seer_dims* d, const float* o_part, const float* l
   p.out = out;
   p.lse_out = lse_out;
   p.S = num_splits;
-  SEER_CUDA(run_combine(p, d->batch, d->num_q_heads, stream));
+  SEER_CUDA(run_combine(p, d->batch, d->num_q_heads, stream, false));
   return SEER_OK;
 }
 
@@ -374,47 +391,53 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   if (a->workspace == nullptr || !aligned(a->workspace, 256)) return SEER_ERR_WORKSPACE;
   const Workspace w = carve(d, a->k_max, a->num_splits, a->workspace);
   if (a->workspace_bytes < w.bytes) return SEER_ERR_WORKSPACE;
+  // every check (and the decode tensor maps) before anything is enqueued
+  if (!a->q || !a->w_gate || !a->seqlens || !a->out) return SEER_ERR_INVALID_ARG;
+  if (!aligned(a->w_gate, 16) || !aligned(a->kbar, 16)) return SEER_ERR_UNSUPPORTED;
+  DecodeLaunch L;
+  SEER_TRY(decode_prepare(d, a->q, a->k_pool, a->v_pool, a->page_table, a->seqlens, w.idx,
+                          w.n_sel, a->k_max, a->num_splits, a->softmax_scale, w.o_part,
+                          w.lse_part, a->dev_status, &L));
+
   if (a->update_kbar == 2)
     SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
                             stream));
   // a0 (incremental) + a1 + a2 in one kernel; same results as the three calls
-  SEER_TRY(check_pool(d, a->k_pool));
-  if (!a->q || !a->w_gate || !a->seqlens) return SEER_ERR_INVALID_ARG;
-  if (a->k_max > d->max_blocks) return SEER_ERR_INVALID_ARG;
-  if (!aligned(a->w_gate, 16) || !aligned(a->kbar, 16) || !aligned(a->q, 4))
-    return SEER_ERR_UNSUPPORTED;
-  {
-    GateSelectParams g;
-    g.q = a->q;
-    g.w_gate = a->w_gate;
-    g.kbar = a->kbar;
-    g.seqlens = a->seqlens;
-    g.k_per_seq = a->k_per_seq;
-    g.scores = w.scores;
-    g.idx = w.idx;
-    g.n_sel = w.n_sel;
-    g.status = a->dev_status;
-    g.k_pool = a->k_pool;
-    g.page_table = a->page_table;
-    g.incremental = a->update_kbar == 1 ? 1 : 0;
-    g.num_pages = d->num_pages;
-    g.stride_page = d->stride_page;
-    g.stride_token = d->stride_token;
-    g.stride_head = d->stride_head;
-    g.Hq = d->num_q_heads;
-    g.Hkv = d->num_kv_heads;
-    g.G = d->num_q_heads / d->num_kv_heads;
-    g.bs = d->block_size;
-    g.max_blocks = d->max_blocks;
-    g.k_max = a->k_max;
-    g.force_newest = a->force_newest ? 1 : 0;
-    g.gate_scale = a->gate_scale;
-    SEER_CUDA(run_gate_select(g, d->batch, stream));
-  }
-  SEER_TRY(seer_sparse_decode(d, a->q, a->k_pool, a->v_pool, a->page_table, a->seqlens, w.idx,
-                              w.n_sel, a->k_max, a->num_splits, a->softmax_scale, w.o_part,
-                              w.lse_part, a->dev_status, stream));
-  SEER_TRY(seer_combine(d, w.o_part, w.lse_part, a->num_splits, a->out, a->lse_out, stream));
+  GateSelectParams g;
+  g.q = a->q;
+  g.w_gate = a->w_gate;
+  g.kbar = a->kbar;
+  g.seqlens = a->seqlens;
+  g.k_per_seq = a->k_per_seq;
+  g.scores = w.scores;
+  g.idx = w.idx;
+  g.n_sel = w.n_sel;
+  g.status = a->dev_status;
+  g.k_pool = a->k_pool;
+  g.page_table = a->page_table;
+  g.incremental = a->update_kbar == 1 ? 1 : 0;
+  g.num_pages = d->num_pages;
+  g.stride_page = d->stride_page;
+  g.stride_token = d->stride_token;
+  g.stride_head = d->stride_head;
+  g.Hq = d->num_q_heads;
+  g.Hkv = d->num_kv_heads;
+  g.G = d->num_q_heads / d->num_kv_heads;
+  g.bs = d->block_size;
+  g.max_blocks = d->max_blocks;
+  g.k_max = a->k_max;
+  g.force_newest = a->force_newest ? 1 : 0;
+  g.gate_scale = a->gate_scale;
+  SEER_CUDA(run_gate_select(g, d->batch, stream, true));
+  // a3, then a4; each grid launches early and waits for its predecessor
+  SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, true));
+  CombineParams c;
+  c.o_part = w.o_part;
+  c.lse_part = w.lse_part;
+  c.out = a->out;
+  c.lse_out = a->lse_out;
+  c.S = a->num_splits;
+  SEER_CUDA(run_combine(c, d->batch, d->num_q_heads, stream, true));
   return SEER_OK;
 }
 

@@ -81,11 +81,11 @@ struct CombineParams {
 cudaError_t run_pool_keys(const PoolParams& p, int B, cudaStream_t stream);
 cudaError_t run_gate_scores(const GateParams& p, int B, cudaStream_t stream);
 cudaError_t run_block_select(const SelectParams& p, int B, cudaStream_t stream);
-cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream);
+cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream, bool pdl);
 cudaError_t run_fill_k(const int32_t* seqlens, int B, int bs, int permille, int budget,
                        int32_t* k_out, cudaStream_t stream);
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
-                              int num_sms, cudaStream_t stream);
-cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream);
+                              int num_sms, cudaStream_t stream, bool pdl);
+cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream, bool pdl);
 
 }  // namespace seer

@@ -16,7 +16,7 @@
 //   * copy thread: pops entries and streams the selected K and V tiles with
 //     4-D TMA loads (64 tokens x 64 dims per box, 128-byte swizzle, L2
 //     evict-first, no multicast) into an NSTAGES-deep ring of 32 KB stages
-//     whose per-stage metadata (valid tokens) rides along;
+//     whose per-stage metadata (valid tokens) rides along (4 stages);
 //   * two groups of four math warps take alternate stages; each warp owns 16
 //     tokens of a stage and never touches global memory in the loop.  The
 //     tensor-core tile is "swap-AB": S^T = K q^T with the 16 tokens as M and
@@ -27,8 +27,10 @@
 //   * online softmax per head column in the exp2 domain; P^T enters the
 //     tensor cores through movmatrix as a bf16 hi + lo pair (weights kept to
 //     ~16 bits); tail tokens past seqlen are masked in registers;
-//   * at the end of an item the 8 warps merge (m, l, O) through shared memory
-//     and write o_part / lse_part.
+//   * at the end of an item each warp drops its (m, l, O) into a shared-memory
+//     slot (mbarrier-counted) and, one item later, merges 1/8 of that item's
+//     outputs into o_part / lse_part: with two slots no warp waits for
+//     another at item boundaries.
 // Every mbarrier wait is bounded (SEER_DEV_TIMEOUT); nothing traps.
 #include "seer_kernels.cuh"
 
@@ -40,7 +42,7 @@ constexpr int kItemSlots = 3;
 constexpr int kOStride = kHeadDim + 4;                 // padded merge row (floats)
 constexpr int kEntries = 256;                          // stage entries in flight (power of 2)
 
-template <int NT, int STAGES>
+template <int NT, int STAGES, int MSLOTS>
 struct DecodeShape {
   static constexpr int kMathWarps = 8;
   static constexpr int kThreads = (kMathWarps + 2) * 32;  // + copy warp + scheduler warp
@@ -60,13 +62,19 @@ struct DecodeShape {
   static constexpr size_t kRec = (kMeta + 4 * kStages + 15) & ~size_t(15);
   static constexpr size_t kEnt = (kRec + 8 * kItemSlots + 15) & ~size_t(15);
   static constexpr size_t kEntCtl = kEnt + 8 * kEntries;  // tail, head
-  static constexpr size_t kML = kEntCtl + 16;
-  static constexpr size_t kO = kML + (size_t)kMathWarps * 2 * kMaxGroup * 4;
-  static size_t smem_bytes(int G) { return 1024 + kO + (size_t)kMathWarps * G * kOStride * 4; }
+  // merge slots: per slot the 8 warps' (m, l) [warps][2][16], the item id and
+  // a full / empty mbarrier pair, then the warps' O [warps][G][kOStride]
+  static constexpr int kMSlots = MSLOTS;
+  static constexpr size_t kMBars = kEntCtl + 16;
+  static constexpr size_t kML = kMBars + 16 * kMSlots + 16;
+  static constexpr size_t kMLBytes = (size_t)kMathWarps * 2 * kMaxGroup * 4;
+  static constexpr size_t kO = kML + kMSlots * kMLBytes;
+  __host__ __device__ static size_t o_slot_floats(int G) { return (size_t)kMathWarps * G * kOStride; }
+  static size_t smem_bytes(int G) { return 1024 + kO + kMSlots * o_slot_floats(G) * 4; }
   static_assert(kRing % 1024 == 0 && kStageBytes % 1024 == 0, "swizzled TMA tiles need 1 KB");
   static_assert(kQBuf % 16 == 0 && kQSlotBytes % 16 == 0, "bulk copy destinations need 16 B");
-  static_assert(kBars % 8 == 0 && kRec % 8 == 0 && kEnt % 16 == 0 && kML % 16 == 0 &&
-                    kO % 16 == 0,
+  static_assert(kBars % 8 == 0 && kRec % 8 == 0 && kEnt % 16 == 0 && kMBars % 8 == 0 &&
+                    kML % 16 == 0 && kO % 16 == 0,
                 "shared-memory carve alignment");
 };
 
@@ -83,10 +91,17 @@ struct ItemCoord {
   int64_t row;  // offset of the (b, h) index row
 };
 
+// Items run split-major (item = s * B * Hkv + bh): under the static
+// round-robin over CTAs each CTA then sees consecutive split indices, whose
+// sizes differ by at most one block, instead of one split index repeated.
+__device__ __forceinline__ int item_bh(const DecodeParams& p, int item) {
+  return item % (p.B * p.Hkv);
+}
+
 __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item, int L, int n) {
   ItemCoord c;
-  const int bh = item / p.S;
-  c.s = item - bh * p.S;
+  const int bh = item_bh(p, item);
+  c.s = item / (p.B * p.Hkv);
   c.b = bh / p.Hkv;
   c.h = bh - c.b * p.Hkv;
   c.L = max(0, min(L, p.max_blocks * p.bs));
@@ -98,11 +113,11 @@ __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item,
   return c;
 }
 
-template <int NT, int STAGES>
-__global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
+template <int NT, int STAGES, int MSLOTS>
+__global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  using Shape = DecodeShape<NT, STAGES>;
+  using Shape = DecodeShape<NT, STAGES, MSLOTS>;
   constexpr int kStages = Shape::kStages;
   constexpr int kQSlotBytes = Shape::kQSlotBytes;
   constexpr int kMathWarps = Shape::kMathWarps;
@@ -122,13 +137,16 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
   int2* ent = reinterpret_cast<int2*>(smem + Shape::kEnt);  // (page, h | sub | valid)
   uint32_t* ent_tail = reinterpret_cast<uint32_t*>(smem + Shape::kEntCtl);
   uint32_t* ent_head = ent_tail + 1;
-  float* m_sh = reinterpret_cast<float*>(smem + Shape::kML);  // [warps][16]
-  float* l_sh = m_sh + kMathWarps * kMaxGroup;                 // [warps][16]
-  float* o_sh = reinterpret_cast<float*>(smem + Shape::kO);    // [warps][G][kOStride]
+  uint64_t* state_full = reinterpret_cast<uint64_t*>(smem + Shape::kMBars);  // [MSLOTS]
+  uint64_t* state_empty = state_full + MSLOTS;                                 // [MSLOTS]
+  int* slot_item = reinterpret_cast<int*>(state_empty + MSLOTS);               // [MSLOTS]
+  float* ml_base = reinterpret_cast<float*>(smem + Shape::kML);  // [slot][warps][m 16 | l 16]
+  float* o_base = reinterpret_cast<float*>(smem + Shape::kO);    // [slot][warps][G][kOStride]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = p.G;
+  const size_t o_slot = Shape::o_slot_floats(G);
 
   if (threadIdx.x == 0) {
     *ent_tail = 0;
@@ -141,9 +159,18 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
       mbar_init(&item_full[i], 1);
       mbar_init(&item_empty[i], kMathWarps);
     }
+    for (int i = 0; i < MSLOTS; ++i) {
+      mbar_init(&state_full[i], kMathWarps);
+      mbar_init(&state_empty[i], kMathWarps);
+    }
     fence_mbar_init();
   }
   __syncthreads();
+  // Everything above touches only shared memory; from here on the kernel reads
+  // what the preceding kernel wrote (the index rows) and writes what it may
+  // still read (the partials), so wait for it, then let the next one launch.
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == kMathWarps + 1) {
     // =============================================================== scheduler
@@ -156,7 +183,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
     int item = blockIdx.x;
     int L_cur = 0, n_cur = 0;
     if (item < p.num_items) {
-      const int bh = item / p.S;
+      const int bh = item_bh(p, item);
       L_cur = __ldg(p.seqlens + bh / p.Hkv);
       n_cur = __ldg(p.n_sel + bh);
     }
@@ -164,7 +191,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
       const int nxt = item + gridDim.x;  // next item's length and count, in flight
       int L_nxt = 0, n_nxt = 0;
       if (nxt < p.num_items) {
-        const int bh = nxt / p.S;
+        const int bh = item_bh(p, nxt);
         L_nxt = __ldg(p.seqlens + bh / p.Hkv);
         n_nxt = __ldg(p.n_sel + bh);
       }
@@ -340,6 +367,49 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
   const int mi = lane >> 3;  // ldmatrix sub-matrix this lane addresses
   uint32_t stage_base = 0;
   bool ok = true;
+  int last_it = -1;
+
+  // This warp's 1/8 of item number u's merge: every warp's (m, l, O) of that
+  // item is in slot u % MSLOTS once state_full completes; thread (warp, lane)
+  // takes outputs e = warp * 32 + lane, + 256, ... of the G x D block.
+  auto merge_share = [&](int u) {
+    const int ms = u % MSLOTS;
+    const uint32_t use = (uint32_t)(u / MSLOTS);
+    if (ok && !mbar_wait(&state_full[ms], use & 1)) {
+      flag_status(p.status, SEER_DEV_TIMEOUT);
+      ok = false;
+    }
+    const int mitem = slot_item[ms];
+    const int bh = item_bh(p, mitem);
+    const int s = mitem / (p.B * p.Hkv);
+    const int b = bh / p.Hkv;
+    const int h = bh - b * p.Hkv;
+    const float* mls = ml_base + (size_t)ms * (Shape::kMLBytes / 4);
+    const float* os = o_base + (size_t)ms * o_slot;
+    for (int e = warp * 32 + lane; e < G * kHeadDim; e += kMathThreads) {
+      const int g = e / kHeadDim, d = e - g * kHeadDim;
+      float mt = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kMathWarps; ++w) mt = fmaxf(mt, mls[w * 2 * kMaxGroup + g]);
+      const int64_t orow = ((int64_t)b * p.Hq + (int64_t)h * G + g) * p.S + s;
+      if (mt == -INFINITY) {
+        p.o_part[orow * kHeadDim + d] = 0.f;
+        if (d == 0) p.lse_part[orow] = -INFINITY;
+        continue;
+      }
+      float lt = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMathWarps; ++w) {
+        const float f = fast_exp2(mls[w * 2 * kMaxGroup + g] - mt);
+        lt += mls[w * 2 * kMaxGroup + kMaxGroup + g] * f;
+        acc += os[((size_t)w * G + g) * kOStride + d] * f;
+      }
+      p.o_part[orow * kHeadDim + d] = acc / lt;
+      if (d == 0) p.lse_part[orow] = (mt + log2f(lt)) * kLn2;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&state_empty[ms]);
+  };
 
   for (int item = blockIdx.x, it_no = 0; item < p.num_items; item += gridDim.x, ++it_no) {
     const int islot = it_no % kItemSlots;
@@ -509,7 +579,10 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
     }
     stage_base += nst;
 
-    // ---- merge the 8 warps' partial softmax states of this item
+    // ---- hand this item's softmax state to the merge: the 8 warps' states
+    // meet in a shared-memory slot; each warp then merges 1/8 of the
+    // previous item, so no warp waits for another at item boundaries (with
+    // two slots; one slot makes it a rendezvous per item)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -521,91 +594,90 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES>::kThreads, 1)
         l[nt][e] = v;
       }
     }
-    if (r == 0) {
+    if (it_no > 0) merge_share(it_no - 1);
+    {
+      const int ms = it_no % MSLOTS;
+      const uint32_t use = (uint32_t)(it_no / MSLOTS);
+      if (ok && !mbar_wait(&state_empty[ms], (use & 1) ^ 1)) {
+        flag_status(p.status, SEER_DEV_TIMEOUT);
+        ok = false;
+      }
+      float* mw = ml_base + (size_t)ms * (Shape::kMLBytes / 4) + warp * 2 * kMaxGroup;
+      if (r == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            mw[nt * 8 + 2 * c + e] = m[nt][e];
+            mw[kMaxGroup + nt * 8 + 2 * c + e] = l[nt][e];
+          }
+        }
+      }
+      float* ow = o_base + (size_t)ms * o_slot + (size_t)warp * G * kOStride;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          m_sh[warp * kMaxGroup + nt * 8 + 2 * c + e] = m[nt][e];
-          l_sh[warp * kMaxGroup + nt * 8 + 2 * c + e] = l[nt][e];
-        }
-      }
-    }
-    float* ow = o_sh + (size_t)warp * G * kOStride;
+          const int head = nt * 8 + 2 * c + e;
+          if (head < G) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int head = nt * 8 + 2 * c + e;
-        if (head < G) {
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            ow[head * kOStride + mt * 16 + r] = o[mt][nt][e];
-            ow[head * kOStride + mt * 16 + r + 8] = o[mt][nt][2 + e];
+            for (int mt = 0; mt < 8; ++mt) {
+              ow[head * kOStride + mt * 16 + r] = o[mt][nt][e];
+              ow[head * kOStride + mt * 16 + r + 8] = o[mt][nt][2 + e];
+            }
           }
         }
       }
+      if (warp == 0 && lane == 0) slot_item[ms] = item;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&state_full[ms]);
     }
-    named_barrier_sync(1, kMathThreads);
-    {
-      const int bh = item / p.S;
-      const int s = item - bh * p.S;
-      const int b = bh / p.Hkv;
-      const int h = bh - b * p.Hkv;
-      for (int e = threadIdx.x; e < G * kHeadDim; e += kMathThreads) {
-        const int g = e / kHeadDim, d = e - g * kHeadDim;
-        float mt = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kMathWarps; ++w) mt = fmaxf(mt, m_sh[w * kMaxGroup + g]);
-        const int64_t orow = ((int64_t)b * p.Hq + (int64_t)h * G + g) * p.S + s;
-        if (mt == -INFINITY) {
-          p.o_part[orow * kHeadDim + d] = 0.f;
-          if (d == 0) p.lse_part[orow] = -INFINITY;
-          continue;
-        }
-        float lt = 0.f, acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kMathWarps; ++w) {
-          const float f = fast_exp2(m_sh[w * kMaxGroup + g] - mt);
-          lt += l_sh[w * kMaxGroup + g] * f;
-          acc += o_sh[((size_t)w * G + g) * kOStride + d] * f;
-        }
-        p.o_part[orow * kHeadDim + d] = acc / lt;
-        if (d == 0) p.lse_part[orow] = (mt + log2f(lt)) * kLn2;
-      }
-    }
-    named_barrier_sync(1, kMathThreads);
+    last_it = it_no;
   }
+  if (last_it >= 0) merge_share(last_it);
 }
 
 // ------------------------------------------------------------------ launcher
-template <int NT, int STAGES>
+template <int NT, int STAGES, int MSLOTS>
 static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
-                                 const DecodeParams& p, int num_sms, cudaStream_t stream) {
-  using Shape = DecodeShape<NT, STAGES>;
+                                 const DecodeParams& p, int num_sms, cudaStream_t stream,
+                                 bool pdl) {
+  using Shape = DecodeShape<NT, STAGES, MSLOTS>;
   const size_t smem = Shape::smem_bytes(p.G);
-  auto kern = sparse_decode_kernel<NT, STAGES>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = sparse_decode_kernel<NT, STAGES, MSLOTS>;
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = ensure_smem_limit(kern, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = p.num_items < num_sms ? p.num_items : num_sms;
-  kern<<<grid, Shape::kThreads, smem, stream>>>(tk, tv, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(Shape::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-// The deepest ring whose shared memory fits (the merge area grows with G).
+// Two merge slots (no per-item rendezvous of the math warps) when shared
+// memory allows, else one.
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
-                              int num_sms, cudaStream_t stream) {
+                              int num_sms, cudaStream_t stream, bool pdl) {
   int dev = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     optin = 227 * 1024;
   if (p.G <= 8) {
-    if (DecodeShape<1, 6>::smem_bytes(p.G) <= (size_t)optin)
-      return launch_decode<1, 6>(tk, tv, p, num_sms, stream);
-    return launch_decode<1, 4>(tk, tv, p, num_sms, stream);
+    if (DecodeShape<1, 4, 2>::smem_bytes(p.G) <= (size_t)optin)
+      return launch_decode<1, 4, 2>(tk, tv, p, num_sms, stream, pdl);
+    return launch_decode<1, 4, 1>(tk, tv, p, num_sms, stream, pdl);
   }
-  return launch_decode<2, 4>(tk, tv, p, num_sms, stream);
+  return launch_decode<2, 4, 1>(tk, tv, p, num_sms, stream, pdl);
 }
 
 }  // namespace seer

@@ -50,6 +50,8 @@ class StepBuffers:
         self.lse = torch.empty((B, w.q_heads), dtype=torch.float32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.scale = 1.0 / math.sqrt(D)
+        # a contiguous cache needs no page table (identity pages)
+        self.page_table = data["page_table"] if w.paged else None
 
     # views into the workspace, in the order the library carves it
     def workspace_views(self):
@@ -76,12 +78,12 @@ class StepBuffers:
 
     def pool_full(self, stream=None):
         d = self.data
-        seer.seer_pool_keys(self.dims, d["k_pool"], d["page_table"], d["seqlens"], 0, self.kbar,
+        seer.seer_pool_keys(self.dims, d["k_pool"], self.page_table, d["seqlens"], 0, self.kbar,
                             self.status, stream)
 
     def args(self, update_kbar: int = 0, q=None) -> "seer.seer_step_args":
         d = self.data
-        return seer.step_args(d["q"] if q is None else q, d["k_pool"], d["v_pool"], d["page_table"],
+        return seer.step_args(d["q"] if q is None else q, d["k_pool"], d["v_pool"], self.page_table,
                               d["seqlens"], d["w_gate"], self.kbar, self.k_per_seq,
                               update_kbar=update_kbar, force_newest=self.force_newest,
                               k_max=self.k_max, num_splits=self.num_splits, gate_scale=self.scale,

@@ -171,6 +171,9 @@ FULL = [
     ("b16_h40_L32k_bs128_budget4k_newest", {}),
     ("b64_ragged_h64_paged_bs64", {"sparsity_permille": 900}),
     ("b64_ragged_h64_paged_bs64", {"sparsity_permille": 0}),
+    ("b64_ragged_h64_paged_bs64", {"sparsity_permille": 500}),
+    ("b64_ragged_h64_paged_bs64", {"sparsity_permille": 800}),
+    ("b64_ragged_h64_paged_bs64", {"sparsity_permille": 950}),
 ]
 
 
@@ -226,3 +229,25 @@ def test_step_head_major_layout_is_bitwise_identical():
         outs.append((run.out.clone(), run.lse.clone(), run.kbar.clone(), v["idx"].clone()))
     for a, b in zip(*outs):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", ["b16_h40_L32k_bs64_s90", "b64_ragged_h64_paged_bs64"])
+def test_step_fused_combine_equals_standalone_combine(name):
+    """The step merges the split partials inside the decode kernel; running the
+    standalone combine on the same partials gives the same bits."""
+    w = W.WORKLOADS[name].replace(batch=3)
+    if w.seqlen is not None:
+        w = w.replace(seqlen=4000)
+    else:
+        w = w.replace(seqlen_range=(64, 4000))
+    data = W.generate(w, 31, DEV)
+    run = StepBuffers(w, data, num_splits=5)
+    run.step(update_kbar=2)
+    v = run.workspace_views()
+    out2 = torch.empty_like(run.out)
+    lse2 = torch.empty_like(run.lse)
+    seer.seer_combine(run.dims, v["o_part"], v["lse_part"], run.num_splits, out2, lse2)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    assert torch.equal(out2, run.out)
+    assert torch.equal(lse2, run.lse)
