@@ -250,159 +250,4 @@ __device__ void select_topk_sorted(const float* row, int nb, int k, int force_ne
   if (tid == 0) *n_out = total;
 }
 
-// The same selection in one histogram pass: the candidates' keys are binned
-// by (key - min) * 256 / (max - min + 1) -- monotone in the key, spread
-// over the scores' actual range rather than fixed bit fields -- one warp finds
-// the bin holding the k'-th largest key, and only that bin's members (a
-// handful for real scores) are ranked exactly by (key, index).  A bin with
-// more than kMaxMembers keys (massive ties) falls back to select_topk.
-// members: kMaxMembers uint2 of shared memory.
-constexpr int kMaxMembers = 1024;
-
-template <int THREADS, int ITEMS>
-__device__ void select_topk_binned(const float* row, int nb, int k, int force_newest, int k_max,
-                                   int32_t* out, int32_t* n_out, int32_t* status, SelectSmem& sm,
-                                   uint2* members, int* scratch /* 4 ints */) {
-  static_assert(THREADS * ITEMS >= kMaxBlocks, "one item per block");
-  constexpr int kWarps = THREADS / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int kk = k < 1 ? 1 : k;
-  if (kk > k_max) kk = k_max;
-  const int n = min(kk, nb);
-  const int forced = (force_newest && n > 0) ? 1 : 0;
-  const int cand = nb - forced;
-  const int want = n - forced;
-  if (want > 0 && want < cand) {
-    // -- key range of the candidates
-    uint32_t key[ITEMS];
-    uint32_t lo = 0xffffffffu, hi = 0u;
-    bool nan_seen = false;
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      const int j = tid * ITEMS + i;
-      key[i] = (j < cand) ? order_key(row[j], nan_seen) : 0u;
-      if (j < cand) {
-        lo = min(lo, key[i]);
-        hi = max(hi, key[i]);
-      }
-    }
-    lo = __reduce_min_sync(0xffffffffu, lo);
-    hi = __reduce_max_sync(0xffffffffu, hi);
-    if (lane == 0) {
-      sm.warp_sums[warp] = (int)lo;
-      members[warp] = make_uint2(lo, hi);  // members doubles as the reduction buffer
-    }
-    for (int e = tid; e < 256; e += THREADS) sm.hist[e] = 0;
-    if (tid == 0) scratch[2] = 0;  // member count
-    __syncthreads();
-    if (warp == 0) {
-      uint32_t l2 = lane < kWarps ? members[lane].x : 0xffffffffu;
-      uint32_t h2 = lane < kWarps ? members[lane].y : 0u;
-      l2 = __reduce_min_sync(0xffffffffu, l2);
-      h2 = __reduce_max_sync(0xffffffffu, h2);
-      if (lane == 0) {
-        scratch[0] = (int)l2;
-        scratch[1] = (int)h2;
-      }
-    }
-    __syncthreads();
-    const uint32_t kmin = (uint32_t)scratch[0];
-    const uint64_t span = (uint64_t)((uint32_t)scratch[1] - kmin) + 1u;
-    // -- histogram of the scaled keys (warp-aggregated atomics)
-    int bin[ITEMS];
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      const int j = tid * ITEMS + i;
-      bin[i] = (j < cand) ? (int)(((uint64_t)(key[i] - kmin) * 256u) / span) : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, bin[i]);
-      if (bin[i] >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin[i]], __popc(peers));
-    }
-    __syncthreads();
-    // -- the bin holding the want-th largest key
-    if (warp == 0) {
-      int cnt[8], tot = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        cnt[e] = sm.hist[255 - 8 * lane - e];
-        tot += cnt[e];
-      }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const int excl = incl - tot;
-      if (excl < want && want <= incl) {
-        int acc = excl;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (acc + cnt[e] >= want) {
-            sm.pick_digit = 255 - 8 * lane - e;
-            sm.pick_above = acc;
-            break;
-          }
-          acc += cnt[e];
-        }
-      }
-    }
-    __syncthreads();
-    const int tbin = sm.pick_digit;
-    const int rem = want - sm.pick_above;  // members of tbin still to take
-    if (sm.hist[tbin] > kMaxMembers) {
-      select_topk<THREADS, ITEMS>(row, nb, k, force_newest, k_max, out, n_out, status, sm);
-      return;
-    }
-    // -- exact ranks inside the threshold bin
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      if (bin[i] == tbin) {
-        const int slot = atomicAdd(&scratch[2], 1);
-        members[slot] = make_uint2(key[i], (uint32_t)(tid * ITEMS + i));
-      }
-    }
-    __syncthreads();
-    const int m = scratch[2];
-    bool sel[ITEMS];
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      if (bin[i] == tbin) {
-        const uint32_t j = (uint32_t)(tid * ITEMS + i);
-        int beaten = 0;
-        for (int q = 0; q < m; ++q) {
-          const uint2 o = members[q];
-          beaten += (o.x > key[i]) || (o.x == key[i] && o.y < j);
-        }
-        sel[i] = beaten < rem;
-      } else {
-        sel[i] = bin[i] > tbin;
-      }
-    }
-    if (nan_seen) flag_status(status, SEER_DEV_NONFINITE_SCORE);
-    if (k > k_max && tid == 0) flag_status(status, SEER_DEV_K_CLAMPED);
-    if (forced) {
-#pragma unroll
-      for (int i = 0; i < ITEMS; ++i)
-        if (tid * ITEMS + i == nb - 1) sel[i] = true;
-    }
-    int local = 0;
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) local += sel[i];
-    int total;
-    int pos = block_exclusive_scan<THREADS>(local, total, sm.warp_sums);
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      if (sel[i]) {
-        if (pos < k_max) out[pos] = tid * ITEMS + i;
-        ++pos;
-      }
-    }
-    for (int q = total + tid; q < k_max; q += THREADS) out[q] = -1;
-    if (tid == 0) *n_out = total;
-    return;
-  }
-  // nothing to choose between (all or none on merit): the radix path is trivial
-  select_topk<THREADS, ITEMS>(row, nb, k, force_newest, k_max, out, n_out, status, sm);
-}
-
 }  // namespace seer

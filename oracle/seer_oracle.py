@@ -60,6 +60,7 @@ __all__ = [
     "split_partials",
     "combine",
     "decode_row",
+    "block_mass",
 ]
 
 
@@ -297,3 +298,29 @@ def decode_row(q_group, W, K, V, seqlen, block_size, k, force_newest,
                                 softmax_scale)
     return {"kbar": kbar, "scores": scores, "indices": idx, "out": out,
             "lse": lse}
+
+
+def block_mass(q_group, K, seqlen, blocks, block_size, scale):
+    """Attention mass of every block: mass[g][j] = sum of query head g's
+    softmax weights (the Agent Skill page's Step 4 definition, over the
+    selected blocks) on the tokens t < L of block j; 0 for blocks that were
+    not selected.  With every block selected this is the dense model's
+    block-level attention distribution, the target the self-distilled gate
+    is trained toward (paper summary page, Abstract: "self-distilled gating").
+    Returns [G][NB]."""
+    L = int(seqlen)
+    G = q_group.shape[0]
+    nb = num_blocks(L, block_size)
+    mass = np.zeros((G, nb), dtype=np.float64)
+    blocks = sorted(int(j) for j in blocks)
+    if not blocks:
+        return mass
+    rows = np.concatenate([np.arange(j * block_size, min((j + 1) * block_size, L)) for j in blocks])
+    x = (q_group @ K[rows].T) * float(scale)
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    p = e / e.sum(axis=1, keepdims=True)
+    owner = rows // block_size
+    for j in blocks:
+        mass[:, j] = p[:, owner == j].sum(axis=1)
+    return mass

@@ -288,3 +288,44 @@ def test_bf16_conversion_is_exact():
     x = torch.randn(1000).to(torch.bfloat16)
     bits = x.view(torch.int16).numpy().view(np.uint16)
     np.testing.assert_array_equal(O.bf16_bits_to_f64(bits), x.double().numpy())
+
+
+
+# ---------------------------------------------------------------- block mass
+
+def test_block_mass_hand_cases():
+    for case in _load("attention_hand.json")["cases"]:
+        if "block_mass" not in case:
+            continue
+        got = O.block_mass(np.array(case["q"], float), np.array(case["K"], float), case["seqlen"],
+                           case["blocks"], case["block_size"], case["scale"])
+        np.testing.assert_allclose(got, np.array(case["block_mass"], float), atol=1e-14,
+                                   err_msg=case["name"])
+
+
+def test_block_mass_dense_equals_library_softmax_block_sums():
+    from scipy.special import softmax
+    rng = np.random.default_rng(12)
+    G, D, L, bs = 3, 16, 300, 64
+    q, K = rng.standard_normal((G, D)), rng.standard_normal((L, D))
+    nb = O.num_blocks(L, bs)
+    got = O.block_mass(q, K, L, range(nb), bs, 0.25)
+    p = softmax(q @ K.T * 0.25, axis=1)
+    want = np.stack([p[:, j * bs:min((j + 1) * bs, L)].sum(axis=1) for j in range(nb)], axis=1)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(got.sum(axis=1), 1.0, rtol=1e-13)
+
+
+def test_block_mass_sparse_properties():
+    rng = np.random.default_rng(13)
+    G, D, L, bs = 4, 16, 500, 64
+    q, K = rng.standard_normal((G, D)), rng.standard_normal((L, D))
+    sel = [0, 3, 7]
+    got = O.block_mass(q, K, L, sel, bs, 0.3)
+    assert got.shape == (G, 8)
+    np.testing.assert_allclose(got.sum(axis=1), 1.0, rtol=1e-13)
+    assert (got[:, [1, 2, 4, 5, 6]] == 0).all()
+    # masses weight the selected blocks' values: out = sum_j mass_j * (p-weighted block mean)
+    V = np.ones((L, D))
+    out, _ = O.masked_attention(q, K, V, L, sel, bs, 0.3)
+    np.testing.assert_allclose(out[:, 0], got.sum(axis=1), rtol=1e-13)
