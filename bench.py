@@ -260,7 +260,7 @@ def run_ours(args):
     # replicas: enough that one rotation reads > 4x L2
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
     probe = W.generate(w, args.seed + 1000 * rank, dev, layout=args.layout)
-    run0 = StepBuffers(w, probe, num_splits=args.splits)
+    run0 = StepBuffers(w, probe, num_splits=args.splits, mass=args.mass)
     run0.pool_full()
     torch.cuda.synchronize()
     sel_bytes, sel_tokens = selected_bytes(run0, probe, w)
@@ -271,7 +271,7 @@ def run_ours(args):
     runs = [run0]
     for r in range(1, replicas):
         d = W.generate(w, args.seed + 1000 * rank + r, dev, layout=args.layout)
-        rr = StepBuffers(w, d, num_splits=run0.num_splits, k_max=run0.k_max)
+        rr = StepBuffers(w, d, num_splits=run0.num_splits, k_max=run0.k_max, mass=args.mass)
         rr.pool_full()
         runs.append(rr)
     step_args = [r.args(update_kbar=1) for r in runs]
@@ -359,7 +359,8 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; random-init gate projection)",
-        "config": workload_config(w, run0, replicas, touched, args.layout),
+        "config": dict(workload_config(w, run0, replicas, touched, args.layout),
+                       block_mass=bool(args.mass)),
         "selected_kv_bytes_per_step": sel_bytes,
         "selected_tokens_per_step": sel_tokens,
         "step_hbm_gbs": (touched / (ms_step * 1e-3)) / 1e9,
@@ -371,7 +372,7 @@ def run_ours(args):
                      "traffic": recorded_traffic(w.name), "kernel": "sparse_decode_kernel",
                      "bytes_per_launch": dec_bytes, "peak_source": f"{peak_kind} hbm_gbs"},
         "e2e": e2e,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + int(args.mass)) * args.steps,
         "clocks": clock_info,
         "device_status": status,
     }
@@ -435,9 +436,15 @@ def decode_alone(runs, steps, stream, replicas):
     def launch(i):
         r, v = runs[i % replicas], views[i % replicas]
         d = r.data
-        seer.seer_sparse_decode(r.dims, d["q"], d["k_pool"], d["v_pool"], r.page_table,
-                                d["seqlens"], v["idx"], v["n_sel"], r.k_max, r.num_splits,
-                                r.scale, v["o_part"], v["lse_part"], r.status, stream)
+        if r.block_lse is not None:
+            seer.seer_sparse_decode_mass(r.dims, d["q"], d["k_pool"], d["v_pool"], r.page_table,
+                                         d["seqlens"], v["idx"], v["n_sel"], r.k_max,
+                                         r.num_splits, r.scale, v["o_part"], v["lse_part"],
+                                         r.block_lse, r.status, stream)
+        else:
+            seer.seer_sparse_decode(r.dims, d["q"], d["k_pool"], d["v_pool"], r.page_table,
+                                    d["seqlens"], v["idx"], v["n_sel"], r.k_max, r.num_splits,
+                                    r.scale, v["o_part"], v["lse_part"], r.status, stream)
     for i in range(3):
         launch(i)
     torch.cuda.synchronize()
@@ -509,6 +516,8 @@ def main(argv=None):
     p.add_argument("--ref-rows", type=int, default=4, help="oracle rows per reference step")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", action="store_true", help="launch each step directly, no CUDA graph")
+    p.add_argument("--mass", action="store_true",
+                   help="also emit every block's attention mass (dense-mode gate target)")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")

@@ -194,6 +194,7 @@ static seer_status decode_prepare(const seer_dims* d, const uint16_t* q, const u
   p.token_inner = token_inner;
   p.num_pages = d->num_pages;
   p.scale_log2 = softmax_scale * kLog2e;
+  p.block_lse = nullptr;
   return SEER_OK;
 }
 
@@ -368,6 +369,49 @@ seer_status seer_sparse_decode(const seer_dims* d, const uint16_t* q, const uint
   return SEER_OK;
 }
 
+size_t seer_block_lse_elems(const seer_dims* d) {
+  if (check_dims(d) != SEER_OK) return 0;
+  return (size_t)d->batch * d->num_q_heads * d->max_blocks * (d->block_size / kTileTokens) * 4;
+}
+
+seer_status seer_sparse_decode_mass(const seer_dims* d, const uint16_t* q, const uint16_t* k_pool,
+                                    const uint16_t* v_pool, const int32_t* page_table,
+                                    const int32_t* seqlens, const int32_t* idx,
+                                    const int32_t* n_sel, int32_t k_max, int32_t num_splits,
+                                    float softmax_scale, float* o_part, float* lse_part,
+                                    float* block_lse, int32_t* dev_status, seer_stream stream) {
+  if (block_lse == nullptr) return SEER_ERR_INVALID_ARG;
+  DecodeLaunch L;
+  SEER_TRY(decode_prepare(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_max,
+                          num_splits, softmax_scale, o_part, lse_part, dev_status, &L));
+  L.p.block_lse = block_lse;
+  SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, false));
+  return SEER_OK;
+}
+
+seer_status seer_block_mass(const seer_dims* d, const int32_t* idx, const int32_t* n_sel,
+                            int32_t k_max, const int32_t* seqlens, const float* block_lse,
+                            const float* lse, float* mass, seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (!idx || !n_sel || !seqlens || !block_lse || !lse || !mass) return SEER_ERR_INVALID_ARG;
+  if (k_max < 1 || k_max > d->max_blocks) return SEER_ERR_INVALID_ARG;
+  MassParams p;
+  p.idx = idx;
+  p.n_sel = n_sel;
+  p.seqlens = seqlens;
+  p.block_lse = block_lse;
+  p.lse = lse;
+  p.mass = mass;
+  p.Hq = d->num_q_heads;
+  p.Hkv = d->num_kv_heads;
+  p.G = d->num_q_heads / d->num_kv_heads;
+  p.bs = d->block_size;
+  p.max_blocks = d->max_blocks;
+  p.k_max = k_max;
+  SEER_CUDA(run_block_mass(p, d->batch, stream));
+  return SEER_OK;
+}
+
 seer_status seer_combine(const seer_dims* d, const float* o_part, const float* lse_part,
                          int32_t num_splits, uint16_t* out, float* lse_out, seer_stream stream) {
   SEER_TRY(check_dims(d));
@@ -398,6 +442,9 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   SEER_TRY(decode_prepare(d, a->q, a->k_pool, a->v_pool, a->page_table, a->seqlens, w.idx,
                           w.n_sel, a->k_max, a->num_splits, a->softmax_scale, w.o_part,
                           w.lse_part, a->dev_status, &L));
+  const bool mass = a->block_mass != nullptr || a->block_lse != nullptr;
+  if (mass && (!a->block_mass || !a->block_lse || !a->lse_out)) return SEER_ERR_INVALID_ARG;
+  L.p.block_lse = mass ? a->block_lse : nullptr;
 
   if (a->update_kbar == 2)
     SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
@@ -438,6 +485,22 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   c.lse_out = a->lse_out;
   c.S = a->num_splits;
   SEER_CUDA(run_combine(c, d->batch, d->num_q_heads, stream, true));
+  if (mass) {
+    MassParams m;
+    m.idx = w.idx;
+    m.n_sel = w.n_sel;
+    m.seqlens = a->seqlens;
+    m.block_lse = a->block_lse;
+    m.lse = a->lse_out;
+    m.mass = a->block_mass;
+    m.Hq = d->num_q_heads;
+    m.Hkv = d->num_kv_heads;
+    m.G = d->num_q_heads / d->num_kv_heads;
+    m.bs = d->block_size;
+    m.max_blocks = d->max_blocks;
+    m.k_max = a->k_max;
+    SEER_CUDA(run_block_mass(m, d->batch, stream));
+  }
   return SEER_OK;
 }
 

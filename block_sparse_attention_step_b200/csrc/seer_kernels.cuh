@@ -68,6 +68,19 @@ struct DecodeParams {
   int token_inner;  // tensor map dims are (D, token, head, page), not (D, head, token, page)
   int64_t num_pages;
   float scale_log2;  // softmax_scale * log2(e)
+  // optional: per (b, query head, block, piece) ln sum_t e^{x_t}, piece =
+  // sub-tile * 4 + warp (16 tokens each); nullptr: not written
+  float* block_lse;
+};
+
+struct MassParams {
+  const int32_t* idx;
+  const int32_t* n_sel;
+  const int32_t* seqlens;
+  const float* block_lse;
+  const float* lse;
+  float* mass;
+  int Hq, Hkv, G, bs, max_blocks, k_max;
 };
 
 struct CombineParams {
@@ -87,5 +100,6 @@ cudaError_t run_fill_k(const int32_t* seqlens, int B, int bs, int permille, int 
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                               int num_sms, cudaStream_t stream, bool pdl);
 cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream, bool pdl);
+cudaError_t run_block_mass(const MassParams& p, int B, cudaStream_t stream);
 
 }  // namespace seer

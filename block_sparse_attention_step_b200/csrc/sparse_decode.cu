@@ -59,9 +59,9 @@ struct DecodeShape {
   static constexpr size_t kQBuf = kRing + (size_t)kStages * kStageBytes;
   static constexpr size_t kBars = kQBuf + (size_t)kItemSlots * kQSlotBytes;
   static constexpr size_t kMeta = kBars + 8 * (2 * kStages + 2 * kItemSlots);
-  static constexpr size_t kRec = (kMeta + 4 * kStages + 15) & ~size_t(15);
+  static constexpr size_t kRec = (kMeta + 8 * kStages + 15) & ~size_t(15);
   static constexpr size_t kEnt = (kRec + 8 * kItemSlots + 15) & ~size_t(15);
-  static constexpr size_t kEntCtl = kEnt + 8 * kEntries;  // tail, head
+  static constexpr size_t kEntCtl = kEnt + 16 * kEntries;  // tail, head
   // merge slots: per slot the 8 warps' (m, l) [warps][2][16], the item id and
   // a full / empty mbarrier pair, then the warps' O [warps][G][kOStride]
   static constexpr int kMSlots = MSLOTS;
@@ -113,7 +113,7 @@ __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item,
   return c;
 }
 
-template <int NT, int STAGES, int MSLOTS>
+template <int NT, int STAGES, int MSLOTS, bool MASS>
 __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
@@ -132,9 +132,9 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
   uint64_t* empty_bar = full_bar + kStages;
   uint64_t* item_full = empty_bar + kStages;
   uint64_t* item_empty = item_full + kItemSlots;
-  int* stage_valid = reinterpret_cast<int*>(smem + Shape::kMeta);
+  int2* stage_meta = reinterpret_cast<int2*>(smem + Shape::kMeta);  // (valid, block * 2 + sub)
   int2* item_rec = reinterpret_cast<int2*>(smem + Shape::kRec);  // (item, stages)
-  int2* ent = reinterpret_cast<int2*>(smem + Shape::kEnt);  // (page, h | sub | valid)
+  int4* ent = reinterpret_cast<int4*>(smem + Shape::kEnt);  // (page, h | sub | valid, block, -)
   uint32_t* ent_tail = reinterpret_cast<uint32_t*>(smem + Shape::kEntCtl);
   uint32_t* ent_head = ent_tail + 1;
   uint64_t* state_full = reinterpret_cast<uint64_t*>(smem + Shape::kMBars);  // [MSLOTS]
@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
           const int t = e * kTileTokens;
           const int valid = min(kTileTokens, ic.L - (j * p.bs + t));
           ent[(tail + incl - ne + e) & (kEntries - 1)] =
-              make_int2(pg, (ic.h << 16) | (e << 8) | valid);
+              make_int4(pg, (ic.h << 16) | (e << 8) | valid, j, 0);
         }
         tail += (uint32_t)total;
         __syncwarp();
@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         }
       }
       if (room) {
-        ent[tail & (kEntries - 1)] = make_int2(-1, 0);
+        ent[tail & (kEntries - 1)] = make_int4(-1, 0, 0, 0);
         __threadfence_block();
         st_volatile(ent_tail, tail + 1u);
       }
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         }
       }
       __threadfence_block();
-      const int2 e = ent[head & (kEntries - 1)];
+      const int4 e = ent[head & (kEntries - 1)];
       __threadfence_block();
       st_volatile(ent_head, ++head);
       if (e.x < 0) break;
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       }
       const int h = (int)((uint32_t)e.y >> 16);
       const int t = ((e.y >> 8) & 0xff) * kTileTokens;
-      stage_valid[slot] = e.y & 0xff;
+      stage_meta[slot] = make_int2(e.y & 0xff, (e.z << 1) | ((e.y >> 8) & 1));
       uint8_t* st = ring + slot * kStageBytes;
       mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
       const int c1 = p.token_inner ? t : h;
@@ -419,6 +419,9 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       ok = false;
     }
     const int nst = ok ? item_rec[islot].y : 0;
+    const int ibh = item_bh(p, item);
+    const int64_t mass_row0 = ((int64_t)(ibh / p.Hkv) * p.Hq + (int64_t)(ibh % p.Hkv) * G) *
+                              p.max_blocks;  // first query head's block-mass row
 
     // q^T fragments (B operand of S^T = K q^T): n = head, k = dim.
     uint32_t qb[NT][8][2];
@@ -469,7 +472,8 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         if (lane == 0) mbar_arrive(&empty_bar[slot]);
         continue;
       }
-      const int valid = stage_valid[slot];
+      const int2 smeta = stage_meta[slot];
+      const int valid = smeta.x;
       const uint32_t k_base = smem_u32(ring + slot * kStageBytes);
       const uint32_t v_base = k_base + 2 * kHalfTileBytes;
 
@@ -529,6 +533,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
 
       // ---- online softmax per head column, P^T fragments via movmatrix
       uint32_t pb[NT][4];  // hi b0, hi b1, lo b0, lo b1
+      float mass_sum[NT][2], mass_mu[NT][2];  // per head column: this lane's e^(x - mu) sum, mu
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         float x[4];
@@ -552,6 +557,10 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
           pr[e] = fast_exp2(x[e] - mu);
           pr[2 + e] = fast_exp2(x[2 + e] - mu);
           l[nt][e] = l[nt][e] * alpha + (pr[e] + pr[2 + e]);
+          if constexpr (MASS) {
+            mass_sum[nt][e] = pr[e] + pr[2 + e];
+            mass_mu[nt][e] = mu;
+          }
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
             o[mt][nt][e] *= alpha;
@@ -574,6 +583,29 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         for (int nt = 0; nt < NT; ++nt) {
           mma_bf16_16816(o[mt][nt], va[mt], pb[nt][0], pb[nt][1]);
           mma_bf16_16816(o[mt][nt], va[mt], pb[nt][2], pb[nt][3]);
+        }
+      }
+      if constexpr (MASS) {
+        // This warp's 16 tokens of the block: ln sum_t e^{x_t} (natural log of
+        // the scaled scores), one piece of the block's attention mass.  Done
+        // after the P.V issue so it overlaps the tensor pipe; one butterfly
+        // reduces both head columns of a lane: after the first exchange
+        // even-r lanes carry column 2c, odd-r lanes column 2c + 1.
+        const int pieces = (p.bs / kTileTokens) * 4;
+        const int64_t col = (int64_t)(smeta.y >> 1) * pieces + (smeta.y & 1) * 4 + wq;
+        const bool odd = (r & 1) != 0;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float keep = odd ? mass_sum[nt][1] : mass_sum[nt][0];
+          keep += __shfl_xor_sync(0xffffffffu, odd ? mass_sum[nt][0] : mass_sum[nt][1], 4);
+          keep += __shfl_xor_sync(0xffffffffu, keep, 8);
+          keep += __shfl_xor_sync(0xffffffffu, keep, 16);
+          const int head = nt * 8 + 2 * c + (odd ? 1 : 0);
+          if (r < 2 && head < G) {
+            const float mu = odd ? mass_mu[nt][1] : mass_mu[nt][0];
+            p.block_lse[(mass_row0 + (int64_t)head * p.max_blocks) * pieces + col] =
+                keep > 0.f ? (mu + __log2f(keep)) * kLn2 : -INFINITY;
+          }
         }
       }
     }
@@ -638,13 +670,13 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
 }
 
 // ------------------------------------------------------------------ launcher
-template <int NT, int STAGES, int MSLOTS>
+template <int NT, int STAGES, int MSLOTS, bool MASS>
 static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
                                  const DecodeParams& p, int num_sms, cudaStream_t stream,
                                  bool pdl) {
   using Shape = DecodeShape<NT, STAGES, MSLOTS>;
   const size_t smem = Shape::smem_bytes(p.G);
-  auto kern = sparse_decode_kernel<NT, STAGES, MSLOTS>;
+  auto kern = sparse_decode_kernel<NT, STAGES, MSLOTS, MASS>;
   static std::atomic<uint64_t> smem_set{0};
   cudaError_t e = ensure_smem_limit(kern, smem_set);
   if (e != cudaSuccess) return e;
@@ -672,12 +704,16 @@ cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, cons
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     optin = 227 * 1024;
+  const bool mass = p.block_lse != nullptr;
   if (p.G <= 8) {
     if (DecodeShape<1, 4, 2>::smem_bytes(p.G) <= (size_t)optin)
-      return launch_decode<1, 4, 2>(tk, tv, p, num_sms, stream, pdl);
-    return launch_decode<1, 4, 1>(tk, tv, p, num_sms, stream, pdl);
+      return mass ? launch_decode<1, 4, 2, true>(tk, tv, p, num_sms, stream, pdl)
+                  : launch_decode<1, 4, 2, false>(tk, tv, p, num_sms, stream, pdl);
+    return mass ? launch_decode<1, 4, 1, true>(tk, tv, p, num_sms, stream, pdl)
+                : launch_decode<1, 4, 1, false>(tk, tv, p, num_sms, stream, pdl);
   }
-  return launch_decode<2, 4, 1>(tk, tv, p, num_sms, stream, pdl);
+  return mass ? launch_decode<2, 4, 1, true>(tk, tv, p, num_sms, stream, pdl)
+              : launch_decode<2, 4, 1, false>(tk, tv, p, num_sms, stream, pdl);
 }
 
 }  // namespace seer

@@ -19,7 +19,7 @@ class StepBuffers:
     def __init__(self, w, data: dict, num_splits: Optional[int] = None,
                  sparsity_permille: Optional[int] = None, budget_tokens: Optional[int] = None,
                  force_newest: Optional[bool] = None, k_max: Optional[int] = None,
-                 device: Optional[torch.device] = None):
+                 device: Optional[torch.device] = None, mass: bool = False):
         self.w = w
         self.data = data
         dev = device or data["q"].device
@@ -52,6 +52,13 @@ class StepBuffers:
         self.scale = 1.0 / math.sqrt(D)
         # a contiguous cache needs no page table (identity pages)
         self.page_table = data["page_table"] if w.paged else None
+        # optional per-block attention mass of every step
+        self.block_lse = self.block_mass = None
+        if mass:
+            self.block_lse = torch.empty(seer.seer_block_lse_elems(self.dims), dtype=torch.float32,
+                                         device=dev)
+            self.block_mass = torch.empty((B, w.q_heads, self.nb_max), dtype=torch.float32,
+                                          device=dev)
 
     # views into the workspace, in the order the library carves it
     def workspace_views(self):
@@ -88,7 +95,8 @@ class StepBuffers:
                               update_kbar=update_kbar, force_newest=self.force_newest,
                               k_max=self.k_max, num_splits=self.num_splits, gate_scale=self.scale,
                               softmax_scale=self.scale, workspace=self.workspace, out=self.out,
-                              lse_out=self.lse, dev_status=self.status)
+                              lse_out=self.lse, dev_status=self.status,
+                              block_lse=self.block_lse, block_mass=self.block_mass)
 
     def step(self, update_kbar: int = 0, stream=None, args=None):
         seer.seer_decode_step(self.dims, args if args is not None else self.args(update_kbar), stream)

@@ -32,6 +32,7 @@ EXPORTS = (
     "seer_k_from_budget", "seer_fill_k", "seer_default_splits", "seer_step_workspace_bytes",
     "seer_pool_keys", "seer_gate_scores", "seer_block_select", "seer_sparse_decode",
     "seer_combine", "seer_decode_step", "seer_decode_step_host", "seer_decode_step_noalloc",
+    "seer_block_lse_elems", "seer_sparse_decode_mass", "seer_block_mass",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -60,7 +61,8 @@ class seer_step_args(ctypes.Structure):
                 ("num_splits", ctypes.c_int32), ("gate_scale", ctypes.c_float),
                 ("softmax_scale", ctypes.c_float), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t), ("out", ctypes.c_void_p),
-                ("lse_out", ctypes.c_void_p), ("dev_status", ctypes.c_void_p)]
+                ("lse_out", ctypes.c_void_p), ("dev_status", ctypes.c_void_p),
+                ("block_lse", ctypes.c_void_p), ("block_mass", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -84,6 +86,10 @@ _SIGS = {
     "seer_decode_step": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_decode_step_host": (_I, [_D, ctypes.POINTER(seer_step_args), _P, _P, _P, _P]),
     "seer_decode_step_noalloc": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
+    "seer_block_lse_elems": (ctypes.c_size_t, [_D]),
+    "seer_sparse_decode_mass": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P,
+                                     _P, _P, _P]),
+    "seer_block_mass": (_I, [_D, _P, _P, _I, _P, _P, _P, _P, _P]),
 }
 
 _lib_handle = None
@@ -223,7 +229,7 @@ def seer_combine(d, o_part, lse_part, num_splits, out, lse_out=None, stream=None
 
 def step_args(q, k_pool, v_pool, page_table, seqlens, w_gate, kbar, k_per_seq, *, update_kbar,
               force_newest, k_max, num_splits, gate_scale, softmax_scale, workspace, out,
-              lse_out=None, dev_status=None) -> seer_step_args:
+              lse_out=None, dev_status=None, block_lse=None, block_mass=None) -> seer_step_args:
     a = seer_step_args()
     a.q = _ptr(q, torch.bfloat16, "q", allow_none=True)
     a.k_pool = _ptr(k_pool, torch.bfloat16, "k_pool")
@@ -244,6 +250,8 @@ def step_args(q, k_pool, v_pool, page_table, seqlens, w_gate, kbar, k_per_seq, *
     a.out = _ptr(out, torch.bfloat16, "out")
     a.lse_out = _ptr(lse_out, torch.float32, "lse_out", allow_none=True)
     a.dev_status = _ptr(dev_status, torch.int32, "dev_status", allow_none=True)
+    a.block_lse = _ptr(block_lse, torch.float32, "block_lse", allow_none=True)
+    a.block_mass = _ptr(block_mass, torch.float32, "block_mass", allow_none=True)
     return a
 
 
@@ -264,3 +272,29 @@ def seer_decode_step_noalloc(d, args: seer_step_args, stream=None):
     ``args.workspace`` (for callers that cannot allocate device memory)."""
     _check("seer_decode_step_noalloc", _lib().seer_decode_step_noalloc(
         ctypes.byref(d), ctypes.byref(args), _stream(stream)))
+
+
+def seer_block_lse_elems(d) -> int:
+    return _lib().seer_block_lse_elems(ctypes.byref(d))
+
+
+def seer_sparse_decode_mass(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_max,
+                            num_splits, softmax_scale, o_part, lse_part, block_lse,
+                            dev_status=None, stream=None):
+    _check("seer_sparse_decode_mass", _lib().seer_sparse_decode_mass(
+        ctypes.byref(d), _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
+        _ptr(v_pool, torch.bfloat16, "v_pool"),
+        _ptr(page_table, torch.int32, "page_table", allow_none=True),
+        _ptr(seqlens, torch.int32, "seqlens"), _ptr(idx, torch.int32, "idx"),
+        _ptr(n_sel, torch.int32, "n_sel"), int(k_max), int(num_splits), float(softmax_scale),
+        _ptr(o_part, torch.float32, "o_part"), _ptr(lse_part, torch.float32, "lse_part"),
+        _ptr(block_lse, torch.float32, "block_lse"),
+        _ptr(dev_status, torch.int32, "dev_status", allow_none=True), _stream(stream)))
+
+
+def seer_block_mass(d, idx, n_sel, k_max, seqlens, block_lse, lse, mass, stream=None):
+    _check("seer_block_mass", _lib().seer_block_mass(
+        ctypes.byref(d), _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
+        int(k_max), _ptr(seqlens, torch.int32, "seqlens"),
+        _ptr(block_lse, torch.float32, "block_lse"), _ptr(lse, torch.float32, "lse"),
+        _ptr(mass, torch.float32, "mass"), _stream(stream)))

@@ -225,8 +225,13 @@ typedef struct seer_step_args {
   void *workspace;           /* seer_step_workspace_bytes() bytes, 256-aligned */
   size_t workspace_bytes;
   uint16_t *out;
-  float *lse_out;            /* may be NULL */
+  float *lse_out;            /* may be NULL, unless block_mass is set */
   int32_t *dev_status;       /* may be NULL */
+  /* Optional per-block attention mass of this step (see seer_block_mass):
+   * both NULL, or block_lse (seer_block_lse_elems() floats) and block_mass
+   * ([B][Hq][max_blocks] fp32) together with lse_out. */
+  float *block_lse;
+  float *block_mass;
 } seer_step_args;
 
 SEER_API seer_status seer_decode_step(const seer_dims *d, const seer_step_args *a,
@@ -240,6 +245,39 @@ SEER_API seer_status seer_decode_step(const seer_dims *d, const seer_step_args *
 SEER_API seer_status seer_decode_step_host(const seer_dims *d, const seer_step_args *a,
                                   const uint16_t *q_host, uint16_t *q_dev,
                                   uint16_t *out_host, seer_stream stream);
+
+/* ------------------------------------------------- per-block attention mass
+ * The dense model's block-level attention distribution is what the
+ * self-distilled gate is trained toward (SeerAttention-R, Abstract:
+ * "learning attention sparsity through a self-distilled gating mechanism";
+ * Agent Skill page, Step 2: the full model is the teacher).  With every block
+ * selected (k = NB, e.g. sparsity 0) these calls give that target for one
+ * decode step; with a sparse selection they give the mass of each selected
+ * block.  mass[b,qh,j] = sum over the tokens t < seqlen of block j of query
+ * head qh's softmax weight; the mass of a KV head's group is the mean over
+ * its G query heads.
+ *
+ * seer_sparse_decode_mass is seer_sparse_decode (same arguments, same
+ * outputs, bit for bit) that also writes block_lse [B][Hq][max_blocks][P],
+ * P = 4 * block_size / 64: per 16-token piece of each processed block, the
+ * natural log of sum_t e^{scaled score}.  Only the selected blocks' pieces
+ * are written.  seer_block_mass turns them into mass [B][Hq][max_blocks] fp32
+ * with the merged lse of each row (seer_combine's lse_out): selected blocks
+ * e^{piece - lse} summed, every other block 0. */
+SEER_API size_t seer_block_lse_elems(const seer_dims *d);
+
+SEER_API seer_status seer_sparse_decode_mass(
+    const seer_dims *d, const uint16_t *q, const uint16_t *k_pool,
+    const uint16_t *v_pool, const int32_t *page_table, const int32_t *seqlens,
+    const int32_t *idx, const int32_t *n_sel, int32_t k_max,
+    int32_t num_splits, float softmax_scale, float *o_part, float *lse_part,
+    float *block_lse, int32_t *dev_status, seer_stream stream);
+
+SEER_API seer_status seer_block_mass(const seer_dims *d, const int32_t *idx,
+                                     const int32_t *n_sel, int32_t k_max,
+                                     const int32_t *seqlens,
+                                     const float *block_lse, const float *lse,
+                                     float *mass, seer_stream stream);
 
 /* ------------------------------------------------------ no-allocation step
  * No counterpart in the paper: this entry point exists for callers that

@@ -1,0 +1,93 @@
+"""Per-block attention mass (the dense-mode target of the self-distilled gate)
+against the fp64 oracle: dense mode (every block selected) and sparse
+selections, both block sizes, paged and contiguous caches, G up to 16; the
+decode partials of the mass variant equal the plain decode's bit for bit."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_step_b200 import seer
+from block_sparse_attention_step_b200 import workloads as W
+from block_sparse_attention_step_b200.runner import StepBuffers
+from oracle import seer_oracle as O
+
+from gpu_util import f64, require_gpu, row_inputs, scale_of
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+MASS_ATOL = 2e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _check_mass(w, data, run, rows):
+    v = run.workspace_views()
+    idx = v["idx"].cpu().numpy()
+    n_sel = v["n_sel"].cpu().numpy()
+    mass = f64(run.block_mass)
+    G = w.group
+    for (b, h) in rows:
+        q, _, K, _, L = row_inputs(w, data, b, h)
+        sel = idx[b, h, :n_sel[b, h]]
+        ref = O.block_mass(q, K, L, sel, w.block_size, scale_of(w))
+        nb = ref.shape[1]
+        got = mass[b, h * G:(h + 1) * G]
+        np.testing.assert_allclose(got[:, :nb], ref, atol=MASS_ATOL, err_msg=str((b, h)))
+        assert (got[:, nb:] == 0).all()
+        if len(sel):
+            np.testing.assert_allclose(got.sum(axis=1), 1.0, atol=1e-4)
+
+
+CASES = {
+    "dense_paged_bs64_g8": (W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(
+        batch=3, seqlen_range=(1, 2000), sparsity_permille=0), None),
+    "sparse_paged_bs64_g8": (W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(
+        batch=3, seqlen_range=(64, 3000), sparsity_permille=900), None),
+    "dense_contig_bs128_g5": (W.WORKLOADS["b16_h40_L32k_bs128_budget4k_newest"].replace(
+        batch=2, seqlen=1500, budget_tokens=None, sparsity_permille=0, force_newest=False), None),
+    "sparse_contig_bs128_g16": (W.WORKLOADS["b16_h40_L32k_bs128_budget4k_newest"].replace(
+        batch=2, q_heads=32, kv_heads=2, seqlen=3000, budget_tokens=1024), 3),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_step_block_mass_matches_oracle(name):
+    w, splits = CASES[name]
+    data = W.generate(w, 41, DEV)
+    run = StepBuffers(w, data, num_splits=splits, mass=True)
+    run.step(update_kbar=2)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    _check_mass(w, data, run, [(b, h) for b in range(w.batch) for h in range(w.kv_heads)])
+
+
+def test_mass_decode_partials_equal_plain_decode():
+    w = W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(batch=3, seqlen_range=(64, 3000))
+    data = W.generate(w, 43, DEV)
+    run = StepBuffers(w, data, mass=True)
+    run.step(update_kbar=2)
+    v = run.workspace_views()
+    d = data
+    o1, l1 = v["o_part"].clone(), v["lse_part"].clone()
+    o2, l2 = torch.empty_like(o1), torch.empty_like(l1)
+    seer.seer_sparse_decode(run.dims, d["q"], d["k_pool"], d["v_pool"], run.page_table,
+                            d["seqlens"], v["idx"], v["n_sel"], run.k_max, run.num_splits,
+                            run.scale, o2, l2)
+    bl = torch.full_like(run.block_lse, float("nan"))
+    o3, l3 = torch.empty_like(o1), torch.empty_like(l1)
+    seer.seer_sparse_decode_mass(run.dims, d["q"], d["k_pool"], d["v_pool"], run.page_table,
+                                 d["seqlens"], v["idx"], v["n_sel"], run.k_max, run.num_splits,
+                                 run.scale, o3, l3, bl)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(o1, o3) and torch.equal(l1, l3)
+    mass2 = torch.empty_like(run.block_mass)
+    seer.seer_block_mass(run.dims, v["idx"], v["n_sel"], run.k_max, d["seqlens"], bl, run.lse,
+                         mass2)
+    torch.cuda.synchronize()
+    assert torch.equal(mass2, run.block_mass)

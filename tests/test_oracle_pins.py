@@ -329,3 +329,8 @@ def test_block_mass_sparse_properties():
     V = np.ones((L, D))
     out, _ = O.masked_attention(q, K, V, L, sel, bs, 0.3)
     np.testing.assert_allclose(out[:, 0], got.sum(axis=1), rtol=1e-13)
+    # a V whose column j is the indicator of block j turns the attention output into the masses
+    Vb = np.zeros((L, D))
+    Vb[np.arange(L), np.arange(L) // bs] = 1.0
+    outb, _ = O.masked_attention(q, K, Vb, L, sel, bs, 0.3)
+    np.testing.assert_allclose(outb[:, :8], got, rtol=1e-12, atol=1e-15)
