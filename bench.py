@@ -432,6 +432,8 @@ def decode_alone(runs, steps, stream, replicas):
     import torch
     from block_sparse_attention_step_b200 import seer
     views = [r.workspace_views() for r in runs]
+    # the item counter the step uses too (zeroed once; each launch leaves it zero)
+    counter = torch.zeros(2, dtype=torch.int32, device=runs[0].out.device)
 
     def launch(i):
         r, v = runs[i % replicas], views[i % replicas]
@@ -440,11 +442,12 @@ def decode_alone(runs, steps, stream, replicas):
             seer.seer_sparse_decode_mass(r.dims, d["q"], d["k_pool"], d["v_pool"], r.page_table,
                                          d["seqlens"], v["idx"], v["n_sel"], r.k_max,
                                          r.num_splits, r.scale, v["o_part"], v["lse_part"],
-                                         r.block_lse, r.status, stream)
+                                         r.block_lse, r.status, stream, work_counter=counter)
         else:
             seer.seer_sparse_decode(r.dims, d["q"], d["k_pool"], d["v_pool"], r.page_table,
                                     d["seqlens"], v["idx"], v["n_sel"], r.k_max, r.num_splits,
-                                    r.scale, v["o_part"], v["lse_part"], r.status, stream)
+                                    r.scale, v["o_part"], v["lse_part"], r.status, stream,
+                                    work_counter=counter)
     for i in range(3):
         launch(i)
     torch.cuda.synchronize()

@@ -5,13 +5,12 @@
 // ranks below -inf.  The newest block NB-1, when forced, is taken first and
 // counts toward k.  Output: the chosen indices ascending, -1 padded.
 //
-// One CTA of 1024 threads per (b, h); thread t owns blocks 4t .. 4t+3 so a
-// block-wide scan visits blocks in index order.  Scores become order-
-// preserving 32-bit keys; a 4-pass MSB radix select (8-bit digits, shared-
-// memory histograms, one warp picking the digit) finds the k'-th largest key
-// T and how many keys equal to T are still needed; a scan over "key == T"
-// ranks the ties by index, and a second scan compacts the chosen blocks in
-// ascending order.  No sort, no data-dependent loop bounds beyond NB.
+// One CTA of 1024 threads per (b, h); thread t owns one block (rows of at
+// most 1024 blocks) or blocks 4t .. 4t+3, so a block-wide scan visits blocks
+// in index order.  The value-binned select (one histogram pass over equal-
+// width score bins, the threshold bin's few blocks ranked pairwise by order
+// key and index) picks the blocks; rows whose threshold bin is crowded fall
+// back to the 4-pass radix select.  No sort.
 #include "seer_kernels.cuh"
 #include "select_core.cuh"
 
@@ -27,9 +26,14 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(const SelectP
   int L = __ldg(p.seqlens + b);
   L = max(0, min(L, p.max_blocks * p.bs));
   const int nb = ceil_div_i(L, p.bs);
-  select_topk<kSelThreads, kSelItems>(p.scores + bh * p.max_blocks, nb, __ldg(p.k_per_seq + b),
-                                      p.force_newest, p.k_max, p.idx + bh * p.k_max,
-                                      p.n_sel + bh, p.status, sm);
+  const float* row = p.scores + bh * p.max_blocks;
+  const int k = __ldg(p.k_per_seq + b);
+  if (nb <= kSelThreads)
+    select_topk_binned<kSelThreads, 1>(row, nb, k, p.force_newest, p.k_max, p.idx + bh * p.k_max,
+                                       p.n_sel + bh, p.status, sm);
+  else
+    select_topk_binned<kSelThreads, kSelItems>(row, nb, k, p.force_newest, p.k_max,
+                                               p.idx + bh * p.k_max, p.n_sel + bh, p.status, sm);
 }
 
 cudaError_t run_block_select(const SelectParams& p, int B, cudaStream_t stream) {

@@ -8,9 +8,9 @@
 // g = W qbar is formed so the projection hides under the first copies; the
 // newest block's mean is recomputed from K with the same summation order as
 // seer_pool_keys and written back; the scores (also written to the caller's
-// scores buffer) stay in shared memory for the exact top-k (a register
-// bitonic sort for rows of at most 512 blocks, the radix select otherwise).  Results are identical to running seer_pool_keys
-// (incremental), seer_gate_scores and seer_block_select one after another.
+// scores buffer) stay in shared memory for the exact value-binned top-k.
+// Results are identical to running seer_pool_keys (incremental),
+// seer_gate_scores and seer_block_select one after another.
 #include "block_mean.cuh"
 #include "seer_kernels.cuh"
 #include "select_core.cuh"
@@ -58,6 +58,7 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
   // (it may have produced q), then let the decode grid start launching.
   pdl_wait();
   pdl_launch_dependents();
+  if (p.work_counter != nullptr && b == 0 && h == 0 && tid < 2) p.work_counter[tid] = 0u;
   const int k_row = __ldg(p.k_per_seq + b);  // used at the end; loaded early
   if (tid == 0) {
     for (int c = 0; c < kGSBuffers && c < nchunks; ++c) {
@@ -156,15 +157,13 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
   for (int j = nb + tid; j < p.max_blocks; j += kGSThreads) scores_out[j] = -INFINITY;
   __syncthreads();
 
-  // the kbar buffers are free now: exchange keys and block flags live there
   if (nb <= kGSThreads)
-    select_topk_sorted<kGSThreads>(sm.scores, nb, k_row, p.force_newest, p.k_max,
-                                   p.idx + bh * p.k_max, p.n_sel + bh, p.status,
-                                   reinterpret_cast<uint64_t*>(sm.buf[0]),
-                                   reinterpret_cast<int*>(sm.buf[1]), sm.sel.warp_sums);
-  else
-    select_topk<kGSThreads, kGSItems>(sm.scores, nb, k_row, p.force_newest, p.k_max,
+    select_topk_binned<kGSThreads, 1>(sm.scores, nb, k_row, p.force_newest, p.k_max,
                                       p.idx + bh * p.k_max, p.n_sel + bh, p.status, sm.sel);
+  else
+    select_topk_binned<kGSThreads, kGSItems>(sm.scores, nb, k_row, p.force_newest, p.k_max,
+                                             p.idx + bh * p.k_max, p.n_sel + bh, p.status,
+                                             sm.sel);
 }
 
 cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream, bool pdl) {

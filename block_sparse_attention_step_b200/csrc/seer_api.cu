@@ -125,6 +125,7 @@ struct Workspace {
   int32_t* n_sel;
   float* o_part;
   float* lse_part;
+  uint32_t* work_counter;  // the decode grid's item counter (2 words)
   size_t bytes;
 };
 
@@ -143,6 +144,7 @@ Workspace carve(const seer_dims* d, int32_t k_max, int32_t S, void* base) {
   w.n_sel = reinterpret_cast<int32_t*>(take(bh * sizeof(int32_t)));
   w.o_part = reinterpret_cast<float*>(take(bq * S * kHeadDim * sizeof(float)));
   w.lse_part = reinterpret_cast<float*>(take(bq * S * sizeof(float)));
+  w.work_counter = reinterpret_cast<uint32_t*>(take(2 * sizeof(uint32_t)));
   w.bytes = off;
   return w;
 }
@@ -160,16 +162,17 @@ static seer_status decode_prepare(const seer_dims* d, const uint16_t* q, const u
                                   const int32_t* seqlens, const int32_t* idx,
                                   const int32_t* n_sel, int32_t k_max, int32_t num_splits,
                                   float softmax_scale, float* o_part, float* lse_part,
-                                  int32_t* dev_status, DecodeLaunch* L) {
+                                  uint32_t* work_counter, int32_t* dev_status, DecodeLaunch* L) {
   SEER_TRY(check_dims(d));
   SEER_TRY(check_pool(d, k_pool));
   SEER_TRY(check_pool(d, v_pool));
   if (!q || !seqlens || !idx || !n_sel || !o_part || !lse_part) return SEER_ERR_INVALID_ARG;
   if (k_max < 1 || k_max > d->max_blocks || num_splits < 1 || num_splits > kMaxSplits)
     return SEER_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(o_part, 8)) return SEER_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(o_part, 8) || !aligned(work_counter, 8))
+    return SEER_ERR_UNSUPPORTED;
   const int64_t items = (int64_t)d->batch * d->num_kv_heads * num_splits;
-  if (items > INT_MAX) return SEER_ERR_UNSUPPORTED;
+  if (items > INT_MAX / 2) return SEER_ERR_UNSUPPORTED;  // item ids carry a flag bit
   const int token_inner = d->stride_token < d->stride_head ? 1 : 0;
   SEER_TRY(make_kv_map(k_pool, d, token_inner, &L->tk));
   SEER_TRY(make_kv_map(v_pool, d, token_inner, &L->tv));
@@ -195,6 +198,7 @@ static seer_status decode_prepare(const seer_dims* d, const uint16_t* q, const u
   p.num_pages = d->num_pages;
   p.scale_log2 = softmax_scale * kLog2e;
   p.block_lse = nullptr;
+  p.work_counter = work_counter;
   return SEER_OK;
 }
 
@@ -360,11 +364,12 @@ seer_status seer_sparse_decode(const seer_dims* d, const uint16_t* q, const uint
                                const uint16_t* v_pool, const int32_t* page_table,
                                const int32_t* seqlens, const int32_t* idx, const int32_t* n_sel,
                                int32_t k_max, int32_t num_splits, float softmax_scale,
-                               float* o_part, float* lse_part, int32_t* dev_status,
-                               seer_stream stream) {
+                               float* o_part, float* lse_part, uint32_t* work_counter,
+                               int32_t* dev_status, seer_stream stream) {
   DecodeLaunch L;
   SEER_TRY(decode_prepare(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_max,
-                          num_splits, softmax_scale, o_part, lse_part, dev_status, &L));
+                          num_splits, softmax_scale, o_part, lse_part, work_counter, dev_status,
+                          &L));
   SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, false));
   return SEER_OK;
 }
@@ -379,11 +384,13 @@ seer_status seer_sparse_decode_mass(const seer_dims* d, const uint16_t* q, const
                                     const int32_t* seqlens, const int32_t* idx,
                                     const int32_t* n_sel, int32_t k_max, int32_t num_splits,
                                     float softmax_scale, float* o_part, float* lse_part,
-                                    float* block_lse, int32_t* dev_status, seer_stream stream) {
+                                    float* block_lse, uint32_t* work_counter, int32_t* dev_status,
+                                    seer_stream stream) {
   if (block_lse == nullptr) return SEER_ERR_INVALID_ARG;
   DecodeLaunch L;
   SEER_TRY(decode_prepare(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_max,
-                          num_splits, softmax_scale, o_part, lse_part, dev_status, &L));
+                          num_splits, softmax_scale, o_part, lse_part, work_counter, dev_status,
+                          &L));
   L.p.block_lse = block_lse;
   SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, false));
   return SEER_OK;
@@ -441,7 +448,7 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   DecodeLaunch L;
   SEER_TRY(decode_prepare(d, a->q, a->k_pool, a->v_pool, a->page_table, a->seqlens, w.idx,
                           w.n_sel, a->k_max, a->num_splits, a->softmax_scale, w.o_part,
-                          w.lse_part, a->dev_status, &L));
+                          w.lse_part, w.work_counter, a->dev_status, &L));
   const bool mass = a->block_mass != nullptr || a->block_lse != nullptr;
   if (mass && (!a->block_mass || !a->block_lse || !a->lse_out)) return SEER_ERR_INVALID_ARG;
   L.p.block_lse = mass ? a->block_lse : nullptr;
@@ -475,6 +482,7 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   g.k_max = a->k_max;
   g.force_newest = a->force_newest ? 1 : 0;
   g.gate_scale = a->gate_scale;
+  g.work_counter = w.work_counter;  // zeroed by the gate grid for the decode grid
   SEER_CUDA(run_gate_select(g, d->batch, stream, true));
   // a3, then a4; each grid launches early and waits for its predecessor
   SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, true));

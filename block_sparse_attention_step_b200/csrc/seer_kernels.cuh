@@ -52,6 +52,7 @@ struct GateSelectParams {
   int64_t num_pages, stride_page, stride_token, stride_head;
   int Hq, Hkv, G, bs, max_blocks, k_max, force_newest;
   float gate_scale;
+  uint32_t* work_counter;  // optional: zeroed for the decode grid that follows
 };
 
 struct DecodeParams {
@@ -71,6 +72,9 @@ struct DecodeParams {
   // optional: per (b, query head, block, piece) ln sum_t e^{x_t}, piece =
   // sub-tile * 4 + warp (16 tokens each); nullptr: not written
   float* block_lse;
+  // optional: 2 words (next item, CTAs done); items are then handed out by
+  // atomicAdd and the last CTA zeroes both; nullptr = round-robin items
+  uint32_t* work_counter;
 };
 
 struct MassParams {

@@ -6,8 +6,10 @@
 // blocks idx[b,h, floor(s*n/S) .. floor((s+1)*n/S)); the result is one
 // normalised partial output and its log-sum-exp per query head.
 //
-// How it runs on sm_100a (one persistent CTA per SM, static item list):
-//   * scheduler warp: for each (b, h, s) item it reads the item's index slice
+// How it runs on sm_100a (one persistent CTA per SM; the (b, h, s) items are
+// handed out through a global counter when the caller gives one, so CTAs that
+// stream faster take more items, else round-robin):
+//   * scheduler warp: for each item it reads the item's index slice
 //     and page numbers lane-parallel (the dependent global loads stay off the
 //     copy path), publishes an item record (the G query rows, copied into
 //     shared memory by a bulk copy, and the number of 64-token stages) in a
@@ -118,6 +120,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   using Shape = DecodeShape<NT, STAGES, MSLOTS>;
+  static_assert(Shape::kMathWarps == 8 && Shape::kGroups == 2, "merge order assumes 2 x 4 warps");
   constexpr int kStages = Shape::kStages;
   constexpr int kQSlotBytes = Shape::kQSlotBytes;
   constexpr int kMathWarps = Shape::kMathWarps;
@@ -180,17 +183,26 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     // to the entry ring read by the copy thread.
     int ok = 1;
     uint32_t tail = 0;
-    int item = blockIdx.x;
+    // CTA c starts on item c.  Round-robin (no counter): the next item's
+    // length and count are fetched one item ahead.  Shared counter: the next
+    // item is claimed only once the copy thread is down to kClaimAhead queued
+    // stages (plus the ring in flight, several microseconds of streaming that
+    // hide the claim's round trips), so a CTA never sits on claimed items
+    // while another runs dry and the CTAs finish together.
+    const bool dyn = p.work_counter != nullptr;
+    constexpr uint32_t kClaimAhead = 4;
+    int item = (int)blockIdx.x;
     int L_cur = 0, n_cur = 0;
     if (item < p.num_items) {
       const int bh = item_bh(p, item);
       L_cur = __ldg(p.seqlens + bh / p.Hkv);
       n_cur = __ldg(p.n_sel + bh);
     }
-    for (int it_no = 0; item < p.num_items && ok; item += gridDim.x, ++it_no) {
-      const int nxt = item + gridDim.x;  // next item's length and count, in flight
-      int L_nxt = 0, n_nxt = 0;
-      if (nxt < p.num_items) {
+    int it_no = 0;
+    for (; item < p.num_items && ok; ++it_no) {
+      int nxt = p.num_items, L_nxt = 0, n_nxt = 0;
+      if (!dyn && item + (int)gridDim.x < p.num_items) {
+        nxt = item + (int)gridDim.x;
         const int bh = item_bh(p, nxt);
         L_nxt = __ldg(p.seqlens + bh / p.Hkv);
         n_nxt = __ldg(p.n_sel + bh);
@@ -281,8 +293,50 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         }
         __syncwarp();
       }
+      if (dyn && ok) {
+        if (lane == 0) {  // wait until the copy thread is nearly through the queue
+          const long long t0 = clock64();
+          while (tail - ld_volatile(ent_head) > kClaimAhead) {
+            if (clock64() - t0 > (1ll << 31)) {
+              flag_status(p.status, SEER_DEV_TIMEOUT);
+              ok = 0;
+              break;
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        unsigned v = 0u;
+        if (lane == 0) v = atomicAdd(p.work_counter, 1u) + gridDim.x;
+        v = __shfl_sync(0xffffffffu, v, 0);
+        if (v < (unsigned)p.num_items) {
+          nxt = (int)v;
+          const int bh = item_bh(p, nxt);
+          L_nxt = __ldg(p.seqlens + bh / p.Hkv);
+          n_nxt = __ldg(p.n_sel + bh);
+        }
+      }
+      item = nxt;
       L_cur = L_nxt;
       n_cur = n_nxt;
+    }
+    // end-of-items record for the math warps
+    if (lane == 0) {
+      const int islot = it_no % kItemSlots;
+      if (mbar_wait(&item_empty[islot], ((it_no / kItemSlots) & 1) ^ 1)) {
+        item_rec[islot] = make_int2(-1, 0);
+        mbar_arrive(&item_full[islot]);
+      } else {
+        flag_status(p.status, SEER_DEV_TIMEOUT);
+      }
+    }
+    // the last CTA to stop fetching puts the counter back to zero for the
+    // next launch that shares it
+    if (p.work_counter != nullptr && lane == 0) {
+      __threadfence();
+      if (atomicAdd(p.work_counter + 1, 1u) == gridDim.x - 1) {
+        atomicExch(p.work_counter, 0u);
+        atomicExch(p.work_counter + 1, 0u);
+      }
     }
     // terminator (the copy thread stops on a negative page)
     if (lane == 0) {
@@ -379,7 +433,12 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       flag_status(p.status, SEER_DEV_TIMEOUT);
       ok = false;
     }
-    const int mitem = slot_item[ms];
+    // Group (item's first stage's parity) first, then the other group: the
+    // sum then runs in the same order whichever group took the item's first
+    // stage, so an item's partials do not depend on which CTA ran it or what
+    // that CTA ran before.
+    const int mitem = slot_item[ms] >> 1;
+    const int first = slot_item[ms] & 1;
     const int bh = item_bh(p, mitem);
     const int s = mitem / (p.B * p.Hkv);
     const int b = bh / p.Hkv;
@@ -399,7 +458,8 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       }
       float lt = 0.f, acc = 0.f;
 #pragma unroll
-      for (int w = 0; w < kMathWarps; ++w) {
+      for (int wr = 0; wr < kMathWarps; ++wr) {
+        const int w = wr ^ (first << 2);  // kMathWarps == 8, groups of 4
         const float f = fast_exp2(mls[w * 2 * kMaxGroup + g] - mt);
         lt += mls[w * 2 * kMaxGroup + kMaxGroup + g] * f;
         acc += os[((size_t)w * G + g) * kOStride + d] * f;
@@ -411,14 +471,19 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     if (lane == 0) mbar_arrive(&state_empty[ms]);
   };
 
-  for (int item = blockIdx.x, it_no = 0; item < p.num_items; item += gridDim.x, ++it_no) {
+  for (int it_no = 0; ok; ++it_no) {
     const int islot = it_no % kItemSlots;
     const uint32_t iphase = (it_no / kItemSlots) & 1;
-    if (ok && !mbar_wait(&item_full[islot], iphase)) {
+    if (!mbar_wait(&item_full[islot], iphase)) {
       flag_status(p.status, SEER_DEV_TIMEOUT);
       ok = false;
+      break;
     }
-    const int nst = ok ? item_rec[islot].y : 0;
+    const int2 rec = item_rec[islot];
+    if (rec.x < 0) break;  // end of items
+    const int item = rec.x;
+    const int nst = ok ? rec.y : 0;
+    const int first_group = (int)(stage_base % Shape::kGroups);  // takes the item's stage 0
     const int ibh = item_bh(p, item);
     const int64_t mass_row0 = ((int64_t)(ibh / p.Hkv) * p.Hq + (int64_t)(ibh % p.Hkv) * G) *
                               p.max_blocks;  // first query head's block-mass row
@@ -660,7 +725,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
           }
         }
       }
-      if (warp == 0 && lane == 0) slot_item[ms] = item;
+      if (warp == 0 && lane == 0) slot_item[ms] = (item << 1) | first_group;
       __syncwarp();
       if (lane == 0) mbar_arrive(&state_full[ms]);
     }

@@ -81,14 +81,14 @@ _SIGS = {
     "seer_gate_scores": (_I, [_D, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P]),
     "seer_block_select": (_I, [_D, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
     "seer_sparse_decode": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P,
-                                _P, _P]),
+                                _P, _P, _P]),
     "seer_combine": (_I, [_D, _P, _P, _I, _P, _P, _P]),
     "seer_decode_step": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_decode_step_host": (_I, [_D, ctypes.POINTER(seer_step_args), _P, _P, _P, _P]),
     "seer_decode_step_noalloc": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_block_lse_elems": (ctypes.c_size_t, [_D]),
     "seer_sparse_decode_mass": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P,
-                                     _P, _P, _P]),
+                                     _P, _P, _P, _P]),
     "seer_block_mass": (_I, [_D, _P, _P, _I, _P, _P, _P, _P, _P]),
 }
 
@@ -208,7 +208,9 @@ def seer_block_select(d, scores, seqlens, k_per_seq, force_newest, k_max, idx, n
 
 
 def seer_sparse_decode(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_max, num_splits,
-                       softmax_scale, o_part, lse_part, dev_status=None, stream=None):
+                       softmax_scale, o_part, lse_part, dev_status=None, stream=None, *,
+                       work_counter=None):
+    """work_counter: None (round-robin items) or 2 zeroed int32 words on the device."""
     _check("seer_sparse_decode", _lib().seer_sparse_decode(
         ctypes.byref(d), _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
         _ptr(v_pool, torch.bfloat16, "v_pool"),
@@ -216,6 +218,7 @@ def seer_sparse_decode(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_
         _ptr(seqlens, torch.int32, "seqlens"), _ptr(idx, torch.int32, "idx"),
         _ptr(n_sel, torch.int32, "n_sel"), int(k_max), int(num_splits), float(softmax_scale),
         _ptr(o_part, torch.float32, "o_part"), _ptr(lse_part, torch.float32, "lse_part"),
+        _ptr(work_counter, torch.int32, "work_counter", allow_none=True),
         _ptr(dev_status, torch.int32, "dev_status", allow_none=True), _stream(stream)))
 
 
@@ -280,7 +283,7 @@ def seer_block_lse_elems(d) -> int:
 
 def seer_sparse_decode_mass(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_max,
                             num_splits, softmax_scale, o_part, lse_part, block_lse,
-                            dev_status=None, stream=None):
+                            dev_status=None, stream=None, *, work_counter=None):
     _check("seer_sparse_decode_mass", _lib().seer_sparse_decode_mass(
         ctypes.byref(d), _ptr(q, torch.bfloat16, "q"), _ptr(k_pool, torch.bfloat16, "k_pool"),
         _ptr(v_pool, torch.bfloat16, "v_pool"),
@@ -289,6 +292,7 @@ def seer_sparse_decode_mass(d, q, k_pool, v_pool, page_table, seqlens, idx, n_se
         _ptr(n_sel, torch.int32, "n_sel"), int(k_max), int(num_splits), float(softmax_scale),
         _ptr(o_part, torch.float32, "o_part"), _ptr(lse_part, torch.float32, "lse_part"),
         _ptr(block_lse, torch.float32, "block_lse"),
+        _ptr(work_counter, torch.int32, "work_counter", allow_none=True),
         _ptr(dev_status, torch.int32, "dev_status", allow_none=True), _stream(stream)))
 
 

@@ -144,7 +144,8 @@ SEER_API int32_t seer_default_splits(const seer_dims *d, int32_t k_max,
                             int32_t num_sms);
 
 /* Bytes of caller workspace seer_decode_step needs (scores, idx, n_sel,
- * o_part and lse_part, each 256-byte aligned). */
+ * o_part, lse_part and the decode grid's 2-word item counter, each 256-byte
+ * aligned).  The step initialises all of it; its contents need not be zero. */
 SEER_API size_t seer_step_workspace_bytes(const seer_dims *d, int32_t k_max,
                                  int32_t num_splits);
 
@@ -189,7 +190,16 @@ SEER_API seer_status seer_block_select(const seer_dims *d, const float *scores,
  * online softmax, so each K/V byte is read from HBM once.  Tokens t >=
  * seqlen_b never enter the math; unselected blocks are never read.  Writes
  * o_part (normalised per split) and lse_part (natural log); an empty split
- * writes o = 0, lse = -inf.  1 <= num_splits <= 64. */
+ * writes o = 0, lse = -inf.  1 <= num_splits <= 64.
+ *
+ * work_counter (optional, may be NULL): two uint32 words of device memory,
+ * 8-byte aligned, zero before the first launch that uses them.  The
+ * persistent grid then hands out its (b, h, split) items through them, so
+ * CTAs that stream faster take more items and the grid finishes together;
+ * the last CTA puts both words back to zero, so a launch that completes
+ * without SEER_DEV_TIMEOUT leaves them ready for the next one.  Launches that
+ * share the words must not overlap.  NULL: items round-robin over the CTAs.
+ * The results do not depend on the choice. */
 SEER_API seer_status seer_sparse_decode(const seer_dims *d, const uint16_t *q,
                                const uint16_t *k_pool, const uint16_t *v_pool,
                                const int32_t *page_table,
@@ -197,6 +207,7 @@ SEER_API seer_status seer_sparse_decode(const seer_dims *d, const uint16_t *q,
                                const int32_t *n_sel, int32_t k_max,
                                int32_t num_splits, float softmax_scale,
                                float *o_part, float *lse_part,
+                               uint32_t *work_counter,
                                int32_t *dev_status, seer_stream stream);
 
 /* a4. Log-sum-exp combine of the split partials: lse = log sum_s e^{lse_s},
@@ -271,7 +282,8 @@ SEER_API seer_status seer_sparse_decode_mass(
     const uint16_t *v_pool, const int32_t *page_table, const int32_t *seqlens,
     const int32_t *idx, const int32_t *n_sel, int32_t k_max,
     int32_t num_splits, float softmax_scale, float *o_part, float *lse_part,
-    float *block_lse, int32_t *dev_status, seer_stream stream);
+    float *block_lse, uint32_t *work_counter, int32_t *dev_status,
+    seer_stream stream);
 
 SEER_API seer_status seer_block_mass(const seer_dims *d, const int32_t *idx,
                                      const int32_t *n_sel, int32_t k_max,

@@ -193,6 +193,46 @@ def test_block_select_bit_exact(nbm, bs, force):
     assert status.item() == 0
 
 
+def _extreme_rows(rng, nbm):
+    """Rows that crowd one score bin or break a naive value range: all equal,
+    one huge outlier, denormal spread, ±3e38 with +inf, half-integer ties."""
+    rows = [np.zeros(nbm, np.float32),
+            rng.standard_normal(nbm).astype(np.float32),
+            (rng.standard_normal(nbm) * 1e-40).astype(np.float32),
+            rng.standard_normal(nbm).astype(np.float32),
+            (np.round(rng.standard_normal(nbm) * 2) / 2).astype(np.float32),
+            np.full(nbm, -np.inf, np.float32)]
+    rows[1][nbm // 3] = 1e30
+    rows[3][:3] = [-3e38, 3e38, np.inf]
+    rows[5][::7] = 1.0
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("nbm", [300, 512, 1024, 3000])
+def test_block_select_crowded_and_extreme_rows(nbm):
+    rng = np.random.default_rng(nbm)
+    s = _extreme_rows(rng, nbm)[:, None, :]          # [B=6][H=1][nbm]
+    B = s.shape[0]
+    bs = 64
+    for force in (False, True):
+        for k in (1, 13, nbm // 10, nbm - 1):
+            d = seer.make_dims(B, 1, 1, 128, bs, nbm, B * nbm)
+            idx = torch.full((B, 1, nbm), 77, dtype=torch.int32, device=DEV)
+            n_sel = torch.full((B, 1), 77, dtype=torch.int32, device=DEV)
+            status = torch.zeros(1, dtype=torch.int32, device=DEV)
+            seqlens = torch.full((B,), nbm * bs, dtype=torch.int32, device=DEV)
+            ks = torch.full((B,), k, dtype=torch.int32, device=DEV)
+            seer.seer_block_select(d, torch.from_numpy(s).to(DEV), seqlens, ks, force, nbm, idx,
+                                   n_sel, status)
+            idx_h, n_h = idx.cpu().numpy(), n_sel.cpu().numpy()
+            for b in range(B):
+                ref = O.select_blocks(s[b, 0].astype(np.float64), k, force)
+                assert n_h[b, 0] == len(ref), (nbm, force, k, b)
+                assert idx_h[b, 0, :len(ref)].tolist() == ref.tolist(), (nbm, force, k, b)
+                assert (idx_h[b, 0, len(ref):] == -1).all()
+            assert status.item() == 0
+
+
 def test_block_select_nan_flags_status():
     d = seer.make_dims(1, 1, 1, 128, 64, 6, 6)
     s = torch.tensor([[[1.0, float("nan"), 3.0, float("-inf"), float("nan"), 2.0]]], device=DEV)

@@ -91,3 +91,27 @@ def test_mass_decode_partials_equal_plain_decode():
                          mass2)
     torch.cuda.synchronize()
     assert torch.equal(mass2, run.block_mass)
+
+
+def test_decode_item_counter_gives_the_same_bits_and_resets():
+    """Items handed out through the shared counter (as in the step) or round-
+    robin give bit-identical partials; the counter is zero after every launch."""
+    w = W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(batch=5, seqlen_range=(64, 5000))
+    data = W.generate(w, 47, DEV)
+    run = StepBuffers(w, data, num_splits=5)
+    run.step(update_kbar=2)
+    v = run.workspace_views()
+    d = data
+    ctr = torch.zeros(2, dtype=torch.int32, device=DEV)
+    outs = []
+    for counter in (None, ctr, ctr):
+        o, l = torch.empty_like(v["o_part"]), torch.empty_like(v["lse_part"])
+        seer.seer_sparse_decode(run.dims, d["q"], d["k_pool"], d["v_pool"], run.page_table,
+                                d["seqlens"], v["idx"], v["n_sel"], run.k_max, run.num_splits,
+                                run.scale, o, l, run.status, work_counter=counter)
+        torch.cuda.synchronize()
+        assert ctr.tolist() == [0, 0]
+        outs.append((o, l))
+    assert run.status.item() == 0
+    for o, l in outs:
+        assert torch.equal(o, v["o_part"]) and torch.equal(l, v["lse_part"])

@@ -123,6 +123,31 @@ def test_step_edge_cases_empty_and_single_token():
     check_rows(w, data, run, [(b, h) for b in (1, 2, 3) for h in range(2)], report)
 
 
+@pytest.mark.parametrize("seqlen,force", [(2000, True), (40000, False)])
+def test_step_zero_query_ties_every_score(seqlen, force):
+    """q = 0 makes every gate score exactly 0: the selection must be the lowest
+    block indices (plus the forced newest block), on rows of at most 512
+    blocks and on longer ones; the output is the mean of the chosen V rows."""
+    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=2, q_heads=8, kv_heads=2,
+                                                           seqlen=seqlen, force_newest=force)
+    data = W.generate(w, 9, DEV)
+    data["q"].zero_()
+    run = StepBuffers(w, data)
+    run.step(update_kbar=2)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    views = run.workspace_views()
+    assert (views["scores"].cpu().numpy()[:, :, :-(-seqlen // 64)] == 0).all()
+    idx, n_sel = views["idx"].cpu().numpy(), views["n_sel"].cpu().numpy()
+    k = int(run.k_per_seq[0])
+    ref = O.select_blocks(np.zeros(-(-seqlen // 64)), k, force)
+    for b in range(2):
+        for h in range(2):
+            assert idx[b, h, :n_sel[b, h]].tolist() == ref.tolist(), (b, h)
+    report = {"exact": 0, "near_tie": 0}
+    check_rows(w, data, run, [(b, h) for b in range(2) for h in range(2)], report)
+
+
 def test_step_incremental_kbar_matches_full_rebuild():
     """Run at L - 1 with a full rebuild, append the token at L - 1 (its K/V
     rows are already in the pool) with the incremental update, and compare

@@ -84,7 +84,10 @@ def test_invalid_arguments_fail_before_any_launch(lib):
     # misaligned pool pointer -> SEER_ERR_UNSUPPORTED
     odd = ctypes.c_void_p(4096 + 2)
     assert lib.seer_sparse_decode(ctypes.byref(d), fake, odd, fake, null, fake, fake, fake, 4, 1,
-                                  0.1, fake, fake, null, null) == 2
+                                  0.1, fake, fake, null, null, null) == 2
+    # misaligned item counter
+    assert lib.seer_sparse_decode(ctypes.byref(d), fake, fake, fake, null, fake, fake, fake, 4, 1,
+                                  0.1, fake, fake, ctypes.c_void_p(4096 + 4), null, null) == 2
     # unaligned strides
     d2 = seer.make_dims(2, 8, 2, 128, 64, 4, 8)
     d2.stride_token = 130
@@ -103,7 +106,7 @@ def test_workspace_and_default_splits(lib):
     ws = seer.seer_step_workspace_bytes(d, 52, 8)
     r = lambda x: (x + 255) // 256 * 256
     expect = (r(16 * 8 * 512 * 4) + r(16 * 8 * 52 * 4) + r(16 * 8 * 4) +
-              r(16 * 40 * 8 * 128 * 4) + r(16 * 40 * 8 * 4))
+              r(16 * 40 * 8 * 128 * 4) + r(16 * 40 * 8 * 4) + r(2 * 4))
     assert ws == expect
     assert seer.seer_step_workspace_bytes(d, 0, 8) == 0
     s = seer.seer_default_splits(d, 52, 148)
