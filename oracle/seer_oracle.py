@@ -61,6 +61,9 @@ __all__ = [
     "combine",
     "decode_row",
     "block_mass",
+    "unified_scores",
+    "unified_scores_f32",
+    "select_blocks_unified",
 ]
 
 
@@ -324,3 +327,37 @@ def block_mass(q_group, K, seqlen, blocks, block_size, scale):
     for j in blocks:
         mass[:, j] = p[:, owner == j].sum(axis=1)
     return mass
+
+
+def unified_scores(per_head_scores) -> np.ndarray:
+    """Cross-head block ranking of one sequence: one block set shared by every
+    KV head, as in the unified cross-head selection of the LessIsMore
+    abstract on the author page (aggregate the heads' evidence, then rank
+    once).  Reading taken: each block's aggregate is the sum over KV heads of
+    its gate score (ranking by the sum is ranking by the mean).  fp64; NaN or
+    +inf with -inf in a column give NaN, -inf alone gives -inf.
+    per_head_scores: [Hkv][NB].  Returns [NB]."""
+    s = np.asarray(per_head_scores, dtype=np.float64)
+    out = np.zeros(s.shape[1], dtype=np.float64)
+    for h in range(s.shape[0]):
+        out = out + s[h]
+    return out
+
+
+def unified_scores_f32(per_head_scores_f32) -> np.ndarray:
+    """The same aggregate in fp32, heads added in order h = 0, 1, ...: the
+    values the GPU's unified select ranks when it is given fp32 scores, so
+    that a test on given scores can demand identical indices (the integer
+    decision is taken in the kernel's precision on both sides)."""
+    s = np.asarray(per_head_scores_f32, dtype=np.float32)
+    out = np.zeros(s.shape[1], dtype=np.float32)
+    for h in range(s.shape[0]):
+        out = (out + s[h]).astype(np.float32)
+    return out
+
+
+def select_blocks_unified(per_head_scores, k: int, force_newest: bool) -> np.ndarray:
+    """Top-k of the cross-head aggregate (``unified_scores``) under the same
+    order, forced block and ascending output as ``select_blocks``; every KV
+    head of the sequence then attends these blocks."""
+    return select_blocks(unified_scores(per_head_scores), k, force_newest)

@@ -334,3 +334,51 @@ def test_block_mass_sparse_properties():
     Vb[np.arange(L), np.arange(L) // bs] = 1.0
     outb, _ = O.masked_attention(q, K, Vb, L, sel, bs, 0.3)
     np.testing.assert_allclose(outb[:, :8], got, rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------- unified cross-head selection
+
+def test_unified_select_hand_cases():
+    for c in _load("select_unified_hand.json")["cases"]:
+        ph = np.array([[_f(v) for v in row] for row in c["per_head"]])
+        agg = O.unified_scores(ph)
+        want = np.array([_f(v) for v in c["aggregate"]])
+        assert np.array_equal(agg, want, equal_nan=True), c
+        assert O.select_blocks_unified(ph, c["k"], c["force_newest"]).tolist() == c["indices"], c
+        per_head = [O.select_blocks(r, c["k"], c["force_newest"]).tolist() for r in ph]
+        assert per_head == c["per_head_indices"], c
+
+
+def test_unified_select_brute_force_and_reductions():
+    rng = np.random.default_rng(17)
+    for trial in range(300):
+        H = int(rng.integers(1, 4))
+        nb = int(rng.integers(1, 8))
+        ph = rng.integers(-2, 3, (H, nb)).astype(float)
+        k = int(rng.integers(1, nb + 2))
+        force = bool(rng.integers(0, 2))
+        # aggregate written out column by column, then the exhaustive search
+        col = [sum(float(ph[h, j]) for h in range(H)) for j in range(nb)]
+        got = O.select_blocks_unified(ph, k, force).tolist()
+        assert got == _brute_select(col, k, force), (ph, k, force)
+        # head order does not matter; one head is the per-head selection;
+        # identical heads select what each head alone selects
+        assert O.select_blocks_unified(ph[::-1], k, force).tolist() == got
+        assert O.select_blocks_unified(ph[:1], k, force).tolist() == \
+            O.select_blocks(ph[0], k, force).tolist()
+        same = np.repeat(ph[:1], 3, axis=0)
+        assert O.select_blocks_unified(same, k, force).tolist() == \
+            O.select_blocks(ph[0], k, force).tolist()
+
+
+def test_unified_f32_aggregate_is_the_in_order_fp32_sum():
+    rng = np.random.default_rng(19)
+    ph = rng.standard_normal((5, 300)).astype(np.float32)
+    got = O.unified_scores_f32(ph)
+    want = ph[0].copy()
+    for h in range(1, 5):
+        want = np.float32(want + ph[h])
+    assert got.dtype == np.float32 and np.array_equal(got, want)
+    # within fp32 rounding of the fp64 sum
+    np.testing.assert_allclose(got, O.unified_scores(ph), rtol=0, atol=4e-6)
+
