@@ -34,6 +34,7 @@ if ROOT not in sys.path:
 METRIC = "sparse-decode tokens/s and µs/step at 32K ctx, 90% sparsity; HBM GB/s vs roofline"
 UNIT = "tokens/s"
 KERNELS_PER_STEP = 3   # gate+select (with the incremental pooled-key update), decode, combine
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal, for the second roofline denominator
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -260,7 +261,7 @@ def run_ours(args):
     # replicas: enough that one rotation reads > 4x L2
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
     probe = W.generate(w, args.seed + 1000 * rank, dev, layout=args.layout)
-    run0 = StepBuffers(w, probe, num_splits=args.splits, mass=args.mass)
+    run0 = StepBuffers(w, probe, num_splits=args.splits, mass=args.mass, unified=args.unified)
     run0.pool_full()
     torch.cuda.synchronize()
     sel_bytes, sel_tokens = selected_bytes(run0, probe, w)
@@ -271,7 +272,8 @@ def run_ours(args):
     runs = [run0]
     for r in range(1, replicas):
         d = W.generate(w, args.seed + 1000 * rank + r, dev, layout=args.layout)
-        rr = StepBuffers(w, d, num_splits=run0.num_splits, k_max=run0.k_max, mass=args.mass)
+        rr = StepBuffers(w, d, num_splits=run0.num_splits, k_max=run0.k_max, mass=args.mass,
+                         unified=args.unified)
         rr.pool_full()
         runs.append(rr)
     step_args = [r.args(update_kbar=1) for r in runs]
@@ -326,8 +328,14 @@ def run_ours(args):
     ms_max = max_over_ranks(ms_total, dev) if world > 1 else ms_total
     ms_step = ms_max / args.steps
 
+    # ---- per-step spread (outside the timed region): an event pair per step
+    pct = step_percentiles(one_step, min(args.steps, 400), stream)
+
     # ---- the dominant kernel alone (roofline), K more launches
     dec_us = decode_alone(runs, args.steps, stream, replicas)
+
+    # ---- every stage through its standalone entry point (separate launches)
+    stages = standalone_stages(runs, min(args.steps, 400), stream, replicas)
 
     # ---- end to end through the host entry point: q from pinned host memory
     # in, out to pinned host memory back, every step
@@ -360,19 +368,24 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded; random-init gate projection)",
         "config": dict(workload_config(w, run0, replicas, touched, args.layout),
-                       block_mass=bool(args.mass)),
+                       block_mass=bool(args.mass),
+                       selection_scope="one block set per sequence (all KV heads)"
+                       if args.unified else "per KV head"),
         "selected_kv_bytes_per_step": sel_bytes,
         "selected_tokens_per_step": sel_tokens,
         "step_hbm_gbs": (touched / (ms_step * 1e-3)) / 1e9,
         "selected_kv_gbs": (sel_bytes / (ms_step * 1e-3)) / 1e9,
         "stage_us": {"step": ms_step * 1e3, "sparse_decode_alone": dec_us,
-                     "rest_of_step": ms_step * 1e3 - dec_us},
+                     "rest_of_step": ms_step * 1e3 - dec_us, "standalone": stages},
+        "step_us_percentiles": pct,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": recorded_traffic(w.name), "kernel": "sparse_decode_kernel",
-                     "bytes_per_launch": dec_bytes, "peak_source": f"{peak_kind} hbm_gbs"},
+                     "bytes_per_launch": dec_bytes, "peak_source": f"{peak_kind} hbm_gbs",
+                     "peak_nominal": NOMINAL_HBM_GBS,
+                     "frac_nominal": achieved / NOMINAL_HBM_GBS},
         "e2e": e2e,
-        "gpu_launches": (KERNELS_PER_STEP + int(args.mass)) * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + int(args.mass) + int(args.unified)) * args.steps,
         "clocks": clock_info,
         "device_status": status,
     }
@@ -423,6 +436,66 @@ def decode_bytes(run, sel_bytes, w):
     rows, and the split partials written."""
     B, Hq, Hkv, S, D = w.batch, w.q_heads, w.kv_heads, run.num_splits, w.head_dim
     return (sel_bytes + B * Hq * D * 2 + B * Hkv * (run.k_max + 1) * 4 + B * Hq * S * (D + 1) * 4)
+
+
+def step_percentiles(one_step, n, stream):
+    """p10 / p50 / p90 of single-step device times, each step between its own
+    pair of CUDA events (taken after the timed region; the pairs add a little
+    per-step overhead, so p50 sits slightly above the timed mean)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        one_step(i)
+        b.record(stream)
+    torch.cuda.synchronize()
+    t = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
+    pick = lambda f: t[min(len(t) - 1, int(f * len(t)))]
+    return {"p10": pick(0.10), "p50": pick(0.50), "p90": pick(0.90), "n": n}
+
+
+def standalone_stages(runs, n, stream, replicas):
+    """Mean device time of each stage through its own C-ABI entry point
+    (incremental pooling, gate scores, block select, combine), n launches each
+    over the rotating replicas.  The step fuses pooling, gate and select into
+    one kernel and chains the rest, so these do not add up to the step."""
+    import torch
+    from block_sparse_attention_step_b200 import seer
+    views = [r.workspace_views() for r in runs]
+
+    def timed(launch):
+        for i in range(3):
+            launch(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n):
+            launch(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n * 1e3
+
+    def pool(i):
+        r = runs[i % replicas]
+        seer.seer_pool_keys(r.dims, r.data["k_pool"], r.page_table, r.data["seqlens"], 1, r.kbar,
+                            r.status, stream)
+
+    def gate(i):
+        r, v = runs[i % replicas], views[i % replicas]
+        seer.seer_gate_scores(r.dims, r.data["q"], r.data["w_gate"], r.kbar, r.data["seqlens"],
+                              r.scale, v["scores"], r.status, stream)
+
+    def select(i):
+        r, v = runs[i % replicas], views[i % replicas]
+        seer.seer_block_select(r.dims, v["scores"], r.data["seqlens"], r.k_per_seq,
+                               r.force_newest, r.k_max, v["idx"], v["n_sel"], r.status, stream)
+
+    def combine(i):
+        r, v = runs[i % replicas], views[i % replicas]
+        seer.seer_combine(r.dims, v["o_part"], v["lse_part"], r.num_splits, r.out, r.lse, stream)
+
+    return {"pool_keys_incremental": timed(pool), "gate_scores": timed(gate),
+            "block_select": timed(select), "combine": timed(combine)}
 
 
 def decode_alone(runs, steps, stream, replicas):
@@ -495,10 +568,20 @@ def cpu_baseline(w, run, args):
     k = run.k_per_seq.cpu().tolist()
     sec_row, n, threads = oracle_rows_timed(w, run.data, rows, args.cpu_budget, k, run.force_newest)
     step_s = sec_row * len(rows)
-    return {"value": w.batch / step_s, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n} of {len(rows)} (b, kv-head) rows of this workload, fp64 numpy oracle "
-                      f"(pool, gate, select, masked attention), {sec_row * 1e3:.1f} ms/row, scaled "
-                      f"to the whole batch"}
+    out = {"value": w.batch / step_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+           "sample": f"{n} of {len(rows)} (b, kv-head) rows of this workload, fp64 numpy oracle "
+                     f"(pool, gate, select, masked attention), {sec_row * 1e3:.1f} ms/row, scaled "
+                     f"to the whole batch"}
+    try:  # the same oracle held to one BLAS thread, on a shorter sample
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            sec1, n1, _ = oracle_rows_timed(w, run.data, rows, args.cpu_budget / 3, k,
+                                            run.force_newest)
+        out["value_1core"] = w.batch / (sec1 * len(rows))
+        out["sample_1core"] = f"{n1} rows, one BLAS thread, {sec1 * 1e3:.1f} ms/row"
+    except ImportError:
+        pass
+    return out
 
 
 def main(argv=None):
@@ -521,6 +604,8 @@ def main(argv=None):
     p.add_argument("--no-graph", action="store_true", help="launch each step directly, no CUDA graph")
     p.add_argument("--mass", action="store_true",
                    help="also emit every block's attention mass (dense-mode gate target)")
+    p.add_argument("--unified", action="store_true",
+                   help="one block set per sequence shared by all KV heads (cross-head ranking)")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")

@@ -42,6 +42,62 @@ cudaError_t run_block_select(const SelectParams& p, int B, cudaStream_t stream) 
   return cudaGetLastError();
 }
 
+// Unified cross-head selection (the LessIsMore abstract on the author page:
+// one block ranking shared by every KV head instead of per-head subsets).
+// One CTA per sequence adds the KV heads' score rows block by block, in head
+// order, in fp32 (the aggregate; ranking by the sum is ranking by the mean),
+// runs the same exact value-binned top-k on it, and writes the one index row
+// to every head, so the decode kernel is unchanged.  Waits for the preceding
+// grid (the gate scores) when chained by programmatic dependent launch.
+__global__ void __launch_bounds__(kSelThreads) unified_select_kernel(const SelectParams p) {
+  __shared__ SelectSmem sm;
+  __shared__ float agg[kMaxBlocks];
+  __shared__ int32_t chosen[kMaxBlocks];
+  __shared__ int32_t n_chosen;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
+  int L = __ldg(p.seqlens + b);
+  L = max(0, min(L, p.max_blocks * p.bs));
+  const int nb = ceil_div_i(L, p.bs);
+  const float* rows = p.scores + (int64_t)b * p.Hkv * p.max_blocks;
+  for (int j = tid; j < nb; j += kSelThreads) {
+    float a = 0.f;
+    for (int h = 0; h < p.Hkv; ++h) a += rows[(int64_t)h * p.max_blocks + j];
+    agg[j] = a;
+  }
+  __syncthreads();
+  const int k = __ldg(p.k_per_seq + b);
+  if (nb <= kSelThreads)
+    select_topk_binned<kSelThreads, 1>(agg, nb, k, p.force_newest, p.k_max, chosen, &n_chosen,
+                                       p.status, sm);
+  else
+    select_topk_binned<kSelThreads, kSelItems>(agg, nb, k, p.force_newest, p.k_max, chosen,
+                                               &n_chosen, p.status, sm);
+  __syncthreads();
+  for (int h = 0; h < p.Hkv; ++h) {
+    const int64_t bh = (int64_t)b * p.Hkv + h;
+    for (int q = tid; q < p.k_max; q += kSelThreads) p.idx[bh * p.k_max + q] = chosen[q];
+    if (tid == 0) p.n_sel[bh] = n_chosen;
+  }
+}
+
+cudaError_t run_unified_select(const SelectParams& p, int B, cudaStream_t stream, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, unified_select_kernel, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 // k per sequence from seqlens (budget mode when budget > 0).
 __global__ void fill_k_kernel(const int32_t* seqlens, int B, int bs, int permille, int budget,
                               int32_t* k_out) {

@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(256) gate_scores_kernel(const GateParams p) {
     for (int row = warp; row < kHeadDim; row += 8) {
       const float4 w = __ldg(reinterpret_cast<const float4*>(W + row * kHeadDim + 4 * lane));
       const float v = warp_dot4(w, qv);
-      if (lane == 0) gvec[row] = v * p.gate_scale;
+      if (lane == 0) gvec[row] = __fmul_rn(v, p.gate_scale);
     }
   }
   __syncthreads();

@@ -360,6 +360,29 @@ seer_status seer_block_select(const seer_dims* d, const float* scores, const int
   return SEER_OK;
 }
 
+seer_status seer_block_select_unified(const seer_dims* d, const float* scores, const int32_t* seqlens,
+                                      const int32_t* k_per_seq, int32_t force_newest, int32_t k_max,
+                                      int32_t* idx, int32_t* n_sel, int32_t* dev_status,
+                                      seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (!scores || !seqlens || !k_per_seq || !idx || !n_sel) return SEER_ERR_INVALID_ARG;
+  if (k_max < 1 || k_max > d->max_blocks) return SEER_ERR_INVALID_ARG;
+  SelectParams p;
+  p.scores = scores;
+  p.seqlens = seqlens;
+  p.k_per_seq = k_per_seq;
+  p.idx = idx;
+  p.n_sel = n_sel;
+  p.status = dev_status;
+  p.Hkv = d->num_kv_heads;
+  p.bs = d->block_size;
+  p.max_blocks = d->max_blocks;
+  p.k_max = k_max;
+  p.force_newest = force_newest ? 1 : 0;
+  SEER_CUDA(run_unified_select(p, d->batch, stream, false));
+  return SEER_OK;
+}
+
 seer_status seer_sparse_decode(const seer_dims* d, const uint16_t* q, const uint16_t* k_pool,
                                const uint16_t* v_pool, const int32_t* page_table,
                                const int32_t* seqlens, const int32_t* idx, const int32_t* n_sel,
@@ -438,6 +461,7 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   SEER_TRY(check_dims(d));
   if (a == nullptr || a->k_per_seq == nullptr || a->kbar == nullptr) return SEER_ERR_INVALID_ARG;
   if (a->update_kbar < 0 || a->update_kbar > 2) return SEER_ERR_INVALID_ARG;
+  if (a->unified_heads != 0 && a->unified_heads != 1) return SEER_ERR_INVALID_ARG;
   if (a->k_max < 1 || a->num_splits < 1) return SEER_ERR_INVALID_ARG;
   if (a->workspace == nullptr || !aligned(a->workspace, 256)) return SEER_ERR_WORKSPACE;
   const Workspace w = carve(d, a->k_max, a->num_splits, a->workspace);
@@ -483,7 +507,23 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   g.force_newest = a->force_newest ? 1 : 0;
   g.gate_scale = a->gate_scale;
   g.work_counter = w.work_counter;  // zeroed by the gate grid for the decode grid
+  g.scores_only = a->unified_heads ? 1 : 0;
   SEER_CUDA(run_gate_select(g, d->batch, stream, true));
+  if (a->unified_heads) {  // one block set per sequence, shared by its KV heads
+    SelectParams u;
+    u.scores = w.scores;
+    u.seqlens = a->seqlens;
+    u.k_per_seq = a->k_per_seq;
+    u.idx = w.idx;
+    u.n_sel = w.n_sel;
+    u.status = a->dev_status;
+    u.Hkv = d->num_kv_heads;
+    u.bs = d->block_size;
+    u.max_blocks = d->max_blocks;
+    u.k_max = a->k_max;
+    u.force_newest = a->force_newest ? 1 : 0;
+    SEER_CUDA(run_unified_select(u, d->batch, stream, true));
+  }
   // a3, then a4; each grid launches early and waits for its predecessor
   SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, true));
   CombineParams c;

@@ -52,6 +52,7 @@ struct GateSelectParams {
   int64_t num_pages, stride_page, stride_token, stride_head;
   int Hq, Hkv, G, bs, max_blocks, k_max, force_newest;
   float gate_scale;
+  int scores_only;          // 1: stop after the scores (the unified select follows)
   uint32_t* work_counter;  // optional: zeroed for the decode grid that follows
 };
 
@@ -99,6 +100,7 @@ cudaError_t run_pool_keys(const PoolParams& p, int B, cudaStream_t stream);
 cudaError_t run_gate_scores(const GateParams& p, int B, cudaStream_t stream);
 cudaError_t run_block_select(const SelectParams& p, int B, cudaStream_t stream);
 cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream, bool pdl);
+cudaError_t run_unified_select(const SelectParams& p, int B, cudaStream_t stream, bool pdl);
 cudaError_t run_fill_k(const int32_t* seqlens, int B, int bs, int permille, int budget,
                        int32_t* k_out, cudaStream_t stream);
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,

@@ -19,7 +19,8 @@ class StepBuffers:
     def __init__(self, w, data: dict, num_splits: Optional[int] = None,
                  sparsity_permille: Optional[int] = None, budget_tokens: Optional[int] = None,
                  force_newest: Optional[bool] = None, k_max: Optional[int] = None,
-                 device: Optional[torch.device] = None, mass: bool = False):
+                 device: Optional[torch.device] = None, mass: bool = False,
+                 unified: bool = False):
         self.w = w
         self.data = data
         dev = device or data["q"].device
@@ -35,6 +36,7 @@ class StepBuffers:
         if self.budget is None and self.permille is None:
             raise ValueError("workload has neither a budget nor a sparsity")
         self.force_newest = w.force_newest if force_newest is None else force_newest
+        self.unified = bool(unified)   # one block set per sequence for all KV heads
         self.k_per_seq = torch.empty(B, dtype=torch.int32, device=dev)
         seer.seer_fill_k(self.dims, data["seqlens"], self.permille or 0, self.budget or 0,
                          self.k_per_seq)
@@ -96,7 +98,8 @@ class StepBuffers:
                               k_max=self.k_max, num_splits=self.num_splits, gate_scale=self.scale,
                               softmax_scale=self.scale, workspace=self.workspace, out=self.out,
                               lse_out=self.lse, dev_status=self.status,
-                              block_lse=self.block_lse, block_mass=self.block_mass)
+                              block_lse=self.block_lse, block_mass=self.block_mass,
+                              unified_heads=self.unified)
 
     def step(self, update_kbar: int = 0, stream=None, args=None):
         seer.seer_decode_step(self.dims, args if args is not None else self.args(update_kbar), stream)

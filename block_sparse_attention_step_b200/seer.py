@@ -30,7 +30,8 @@ DEV_TIMEOUT = 16
 EXPORTS = (
     "seer_version", "seer_status_string", "seer_dims_default", "seer_k_from_sparsity",
     "seer_k_from_budget", "seer_fill_k", "seer_default_splits", "seer_step_workspace_bytes",
-    "seer_pool_keys", "seer_gate_scores", "seer_block_select", "seer_sparse_decode",
+    "seer_pool_keys", "seer_gate_scores", "seer_block_select", "seer_block_select_unified",
+    "seer_sparse_decode",
     "seer_combine", "seer_decode_step", "seer_decode_step_host", "seer_decode_step_noalloc",
     "seer_block_lse_elems", "seer_sparse_decode_mass", "seer_block_mass",
 )
@@ -62,7 +63,8 @@ class seer_step_args(ctypes.Structure):
                 ("softmax_scale", ctypes.c_float), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t), ("out", ctypes.c_void_p),
                 ("lse_out", ctypes.c_void_p), ("dev_status", ctypes.c_void_p),
-                ("block_lse", ctypes.c_void_p), ("block_mass", ctypes.c_void_p)]
+                ("block_lse", ctypes.c_void_p), ("block_mass", ctypes.c_void_p),
+                ("unified_heads", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -80,6 +82,7 @@ _SIGS = {
     "seer_pool_keys": (_I, [_D, _P, _P, _P, _I, _P, _P, _P]),
     "seer_gate_scores": (_I, [_D, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P]),
     "seer_block_select": (_I, [_D, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
+    "seer_block_select_unified": (_I, [_D, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
     "seer_sparse_decode": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P,
                                 _P, _P, _P]),
     "seer_combine": (_I, [_D, _P, _P, _I, _P, _P, _P]),
@@ -207,6 +210,15 @@ def seer_block_select(d, scores, seqlens, k_per_seq, force_newest, k_max, idx, n
         _ptr(dev_status, torch.int32, "dev_status", allow_none=True), _stream(stream)))
 
 
+def seer_block_select_unified(d, scores, seqlens, k_per_seq, force_newest, k_max, idx, n_sel,
+                      dev_status=None, stream=None):
+    _check("seer_block_select_unified", _lib().seer_block_select_unified(
+        ctypes.byref(d), _ptr(scores, torch.float32, "scores"), _ptr(seqlens, torch.int32, "seqlens"),
+        _ptr(k_per_seq, torch.int32, "k_per_seq"), int(bool(force_newest)), int(k_max),
+        _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
+        _ptr(dev_status, torch.int32, "dev_status", allow_none=True), _stream(stream)))
+
+
 def seer_sparse_decode(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, k_max, num_splits,
                        softmax_scale, o_part, lse_part, dev_status=None, stream=None, *,
                        work_counter=None):
@@ -232,7 +244,8 @@ def seer_combine(d, o_part, lse_part, num_splits, out, lse_out=None, stream=None
 
 def step_args(q, k_pool, v_pool, page_table, seqlens, w_gate, kbar, k_per_seq, *, update_kbar,
               force_newest, k_max, num_splits, gate_scale, softmax_scale, workspace, out,
-              lse_out=None, dev_status=None, block_lse=None, block_mass=None) -> seer_step_args:
+              lse_out=None, dev_status=None, block_lse=None, block_mass=None,
+              unified_heads=False) -> seer_step_args:
     a = seer_step_args()
     a.q = _ptr(q, torch.bfloat16, "q", allow_none=True)
     a.k_pool = _ptr(k_pool, torch.bfloat16, "k_pool")
@@ -255,6 +268,7 @@ def step_args(q, k_pool, v_pool, page_table, seqlens, w_gate, kbar, k_per_seq, *
     a.dev_status = _ptr(dev_status, torch.int32, "dev_status", allow_none=True)
     a.block_lse = _ptr(block_lse, torch.float32, "block_lse", allow_none=True)
     a.block_mass = _ptr(block_mass, torch.float32, "block_mass", allow_none=True)
+    a.unified_heads = int(bool(unified_heads))
     return a
 
 

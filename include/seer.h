@@ -183,6 +183,20 @@ SEER_API seer_status seer_block_select(const seer_dims *d, const float *scores,
                               int32_t k_max, int32_t *idx, int32_t *n_sel,
                               int32_t *dev_status, seer_stream stream);
 
+/* a2, unified variant (next to the per-head selection): one block set per
+ * sequence shared by every KV head, after the unified cross-head ranking of
+ * the LessIsMore abstract on the author page.  A block's aggregate is the sum
+ * of its scores over the KV heads, added in head order in fp32; the top-k of
+ * the aggregate follows the same order, k, forced block, padding and flag
+ * rules as seer_block_select, and the one index row (and n_sel) is written to
+ * every head's row, so seer_sparse_decode needs no change.  Arguments as for
+ * seer_block_select; scores of all KV heads must be present. */
+SEER_API seer_status seer_block_select_unified(const seer_dims *d, const float *scores,
+                              const int32_t *seqlens,
+                              const int32_t *k_per_seq, int32_t force_newest,
+                              int32_t k_max, int32_t *idx, int32_t *n_sel,
+                              int32_t *dev_status, seer_stream stream);
+
 /* a3. Split-KV sparse flash-decoding (Agent Skill page, Step 4: masked
  * softmax attention, scale softmax_scale).  For each (b, h, split s) the
  * selected blocks idx[b,h, floor(s*n/S) .. floor((s+1)*n/S)) are staged by
@@ -243,6 +257,9 @@ typedef struct seer_step_args {
    * ([B][Hq][max_blocks] fp32) together with lse_out. */
   float *block_lse;
   float *block_mass;
+  /* 0: each KV head selects its own blocks (seer_block_select); 1: one block
+   * set per sequence shared by all its KV heads (seer_block_select_unified). */
+  int32_t unified_heads;
 } seer_step_args;
 
 SEER_API seer_status seer_decode_step(const seer_dims *d, const seer_step_args *a,

@@ -148,6 +148,38 @@ def test_step_zero_query_ties_every_score(seqlen, force):
     check_rows(w, data, run, [(b, h) for b in range(2) for h in range(2)], report)
 
 
+@pytest.mark.parametrize("update_kbar", [1, 2])
+def test_step_many_rows_matches_standalone_stages(update_kbar):
+    """More (b, h) rows than SMs (the fused gate kernel runs in several waves):
+    its scores and indices equal the standalone gate + select kernels bit for
+    bit, on rows of at most 512 blocks and longer ones, and the outputs match
+    the oracle on sampled rows."""
+    w = W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(
+        batch=80, q_heads=8, kv_heads=2, seqlen_range=(1, 45000), sparsity_permille=800)
+    data = W.generate(w, 23, DEV)
+    run = StepBuffers(w, data)
+    run.pool_full()
+    run.step(update_kbar=update_kbar)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    v = run.workspace_views()
+    scores = torch.empty_like(v["scores"])
+    idx = torch.full_like(v["idx"], 77)
+    n_sel = torch.full_like(v["n_sel"], 77)
+    seer.seer_gate_scores(run.dims, data["q"], data["w_gate"], run.kbar, data["seqlens"],
+                          run.scale, scores, run.status)
+    seer.seer_block_select(run.dims, scores, data["seqlens"], run.k_per_seq, run.force_newest,
+                           run.k_max, idx, n_sel, run.status)
+    torch.cuda.synchronize()
+    assert torch.equal(scores, v["scores"])
+    assert torch.equal(idx, v["idx"]) and torch.equal(n_sel, v["n_sel"])
+    nb = -(-data["seqlens"].cpu() // 64)
+    assert (nb > 512).any() and (nb <= 512).any()
+    report = {"exact": 0, "near_tie": 0}
+    rows = [(b, h) for b in range(0, 80, 7) for h in range(2)]
+    check_rows(w, data, run, rows, report)
+
+
 def test_step_incremental_kbar_matches_full_rebuild():
     """Run at L - 1 with a full rebuild, append the token at L - 1 (its K/V
     rows are already in the pool) with the incremental update, and compare
