@@ -277,6 +277,8 @@ def run_ours(args):
         rr.pool_full()
         runs.append(rr)
     step_args = [r.args(update_kbar=1) for r in runs]
+    # the per-stage step (3 kernels chained by PDL) or the single-launch step
+    step_call = seer.seer_decode_step_fused if args.fused else seer.seer_decode_step
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize()
 
@@ -293,13 +295,13 @@ def run_ours(args):
         side.wait_stream(stream)
         with torch.cuda.stream(side):
             for i in range(replicas):
-                seer.seer_decode_step(runs[i].dims, step_args[i], side)
+                step_call(runs[i].dims, step_args[i], side)
         stream.wait_stream(side)
         torch.cuda.synchronize()
         for i in range(replicas):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                seer.seer_decode_step(runs[i].dims, step_args[i], torch.cuda.current_stream())
+                step_call(runs[i].dims, step_args[i], torch.cuda.current_stream())
             graphs.append(g)
         torch.cuda.synchronize()
 
@@ -307,7 +309,7 @@ def run_ours(args):
         if graphs:
             graphs[i % replicas].replay()
         else:
-            seer.seer_decode_step(runs[i % replicas].dims, step_args[i % replicas], stream)
+            step_call(runs[i % replicas].dims, step_args[i % replicas], stream)
 
     clocks = ClockSampler(local) if rank == 0 else None
     for i in range(args.warmup):
@@ -370,7 +372,9 @@ def run_ours(args):
         "config": dict(workload_config(w, run0, replicas, touched, args.layout),
                        block_mass=bool(args.mass),
                        selection_scope="one block set per sequence (all KV heads)"
-                       if args.unified else "per KV head"),
+                       if args.unified else "per KV head",
+                       step_launch="single cooperative launch" if args.fused
+                       else "per stage, PDL-chained"),
         "selected_kv_bytes_per_step": sel_bytes,
         "selected_tokens_per_step": sel_tokens,
         "step_hbm_gbs": (touched / (ms_step * 1e-3)) / 1e9,
@@ -385,7 +389,8 @@ def run_ours(args):
                      "peak_nominal": NOMINAL_HBM_GBS,
                      "frac_nominal": achieved / NOMINAL_HBM_GBS},
         "e2e": e2e,
-        "gpu_launches": (KERNELS_PER_STEP + int(args.mass) + int(args.unified)) * args.steps,
+        "gpu_launches": (1 if args.fused else
+                         KERNELS_PER_STEP + int(args.mass) + int(args.unified)) * args.steps,
         "clocks": clock_info,
         "device_status": status,
     }
@@ -606,6 +611,8 @@ def main(argv=None):
                    help="also emit every block's attention mass (dense-mode gate target)")
     p.add_argument("--unified", action="store_true",
                    help="one block set per sequence shared by all KV heads (cross-head ranking)")
+    p.add_argument("--fused", action="store_true",
+                   help="the whole step as one cooperative launch (seer_decode_step_fused)")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")

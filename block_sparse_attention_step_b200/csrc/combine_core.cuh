@@ -52,14 +52,56 @@ __device__ __forceinline__ float combine_element(const float* lse_row, const flo
       for (int i = 0; i < kChunk; ++i) {
         if (s0 + i < S) {
           const float w = expf(l[i] - m);
-          tot += w;
-          if (w != 0.f) acc += w * x[i];
+          tot = __fadd_rn(tot, w);
+          if (w != 0.f) acc = __fmaf_rn(w, x[i], acc);
         }
       }
     }
   }
   *lse_merged = tot > 0.f ? m + logf(tot) : -INFINITY;
-  return tot > 0.f ? acc * (1.f / tot) : 0.f;
+  return tot > 0.f ? __fmul_rn(acc, 1.f / tot) : 0.f;
 }
+
+// The same merge for one whole (b, query head) row by one warp: lane l takes
+// dims 4l .. 4l+3 and every split's 4 values in one 16-byte load; the split
+// weights come from the lse values through shuffles.  Same arithmetic in the
+// same order as combine_element, so the same bits.  S <= 64.
+template <typename LOAD4>
+__device__ __forceinline__ void combine_row_warp(const float* lse_row, const float* o_row, int S,
+                                                 uint16_t* out_row, float* lse_out, LOAD4 load4) {
+  const int lane = threadIdx.x & 31;
+  const float la = lane < S ? __ldcg(lse_row + lane) : -INFINITY;
+  const float lb = lane + 32 < S ? __ldcg(lse_row + lane + 32) : -INFINITY;
+  float m = fmaxf(la, lb);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float tot = 0.f, acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  if (m != -INFINITY) {
+    for (int s = 0; s < S; ++s) {
+      const float l = __shfl_sync(0xffffffffu, s < 32 ? la : lb, s & 31);
+      const float4 x = load4(o_row + (int64_t)s * kHeadDim + 4 * lane);
+      const float w = expf(l - m);
+      tot = __fadd_rn(tot, w);
+      if (w != 0.f) {
+        acc0 = __fmaf_rn(w, x.x, acc0);
+        acc1 = __fmaf_rn(w, x.y, acc1);
+        acc2 = __fmaf_rn(w, x.z, acc2);
+        acc3 = __fmaf_rn(w, x.w, acc3);
+      }
+    }
+  }
+  const float r = tot > 0.f ? 1.f / tot : 0.f;
+  out_row[4 * lane + 0] = to_bf16_bits(tot > 0.f ? __fmul_rn(acc0, r) : 0.f);
+  out_row[4 * lane + 1] = to_bf16_bits(tot > 0.f ? __fmul_rn(acc1, r) : 0.f);
+  out_row[4 * lane + 2] = to_bf16_bits(tot > 0.f ? __fmul_rn(acc2, r) : 0.f);
+  out_row[4 * lane + 3] = to_bf16_bits(tot > 0.f ? __fmul_rn(acc3, r) : 0.f);
+  if (lse_out != nullptr && lane == 0) *lse_out = tot > 0.f ? m + logf(tot) : -INFINITY;
+}
+
+struct Load4L2 {  // 16-byte loads of data written by other CTAs of this kernel
+  __device__ __forceinline__ float4 operator()(const float* p) const {
+    return __ldcg(reinterpret_cast<const float4*>(p));
+  }
+};
 
 }  // namespace seer

@@ -1,0 +1,244 @@
+// One gate row -- a0 (incremental) + a1 + a2 for one (sequence b, KV head h) --
+// as a device function that a whole CTA runs, shared by the gate + select
+// kernel of the step (one row per CTA, 512 threads) and the single-launch
+// fused step (rows of a persistent CTA, 320 threads):
+//   * optionally append the new token's K and V rows at position L - 1 of the
+//     paged cache (the step's KV append);
+//   * refresh the newest block's pooled key from K (the summation order of
+//     seer_pool_keys) and write it back to kbar;
+//   * g = gate_scale * W[h] qbar, qbar the mean of the group's queries;
+//   * stream the kbar row through a ring of NBUF chunk buffers (bulk copies
+//     on mbarriers) and score every block, 8 rows per worker warp per chunk
+//     in one reduction that gives the same bits as warp_dot4 row by row;
+//   * select the top-k with the exact value-binned select (or stop after the
+//     scores when the unified cross-head select follows).
+// Results are identical to seer_pool_keys (incremental), seer_gate_scores and
+// seer_block_select run one after another.
+#pragma once
+
+#include "block_mean.cuh"
+#include "seer_kernels.cuh"
+#include "select_core.cuh"
+
+namespace seer {
+
+// Shared-memory scratch of a gate row besides the chunk buffers.  part,
+// newest, qbar and gvec are read and written as float4: the struct and those
+// members sit on 16-byte boundaries.  The pooling partials are consumed
+// before the first score is written, so they share the scores' space.
+struct alignas(16) GateRowScratch {
+  union {
+    float scores[kMaxBlocks];
+    float part[kPoolWarps * kHeadDim];
+  };
+  float newest[kHeadDim];
+  float qbar[kHeadDim];
+  float gvec[kHeadDim];
+  SelectSmem sel;
+};
+static_assert(offsetof(GateRowScratch, part) % 16 == 0 &&
+                  offsetof(GateRowScratch, newest) % 16 == 0 &&
+                  offsetof(GateRowScratch, qbar) % 16 == 0 &&
+                  offsetof(GateRowScratch, gvec) % 16 == 0 &&
+                  offsetof(GateRowScratch, sel) % 8 == 0,
+              "float4 members of the gate scratch on 16-byte boundaries");
+
+// Same rows and summation order as pool_warp_partial, through L2 (the row
+// appended by this CTA a moment ago must not come from a stale read-only
+// cache line).
+__device__ __forceinline__ float4 pool_warp_partial_l2(const uint16_t* base_lane,
+                                                       int64_t stride_token, int valid,
+                                                       int warp) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 16
+  for (int t = warp; t < valid; t += kPoolWarps) {
+    const uint2 v = __ldcg(reinterpret_cast<const uint2*>(base_lane + (int64_t)t * stride_token));
+    a0 += __uint_as_float(v.x << 16);
+    a1 += __uint_as_float(v.x & 0xffff0000u);
+    a2 += __uint_as_float(v.y << 16);
+    a3 += __uint_as_float(v.y & 0xffff0000u);
+  }
+  return make_float4(a0, a1, a2, a3);
+}
+
+// The kbar chunk buffers of a gate row: NBUF slots of CHUNK_ROWS rows each,
+// anywhere in shared memory (16-byte aligned).
+template <int NBUF>
+struct ChunkRing {
+  float* slot[NBUF];
+};
+
+// THREADS: the CTA (every thread calls this; it synchronises the CTA).
+// WORKERS: warps 0 .. WORKERS-1 form g and the scores (8 W rows and 8 kbar
+// rows per warp at a time).  CHUNK_ROWS = 8 * WORKERS kbar rows per buffer.
+// Threads QFIRST .. QFIRST + QTHREADS - 1 form the mean query.  Thread 0
+// issues the copies.  `seq` counts the chunks this CTA consumed before (slot
+// and parity of the ring), so a persistent CTA's rows share one ring.
+// Returns false when a wait ran out (SEER_DEV_TIMEOUT is flagged).
+template <int THREADS, int WORKERS, int NBUF, int QFIRST, int QTHREADS>
+__device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRing<NBUF>& ring,
+                         uint64_t* bars, uint32_t& seq, GateRowScratch& gs) {
+  constexpr int CHUNK_ROWS = 8 * WORKERS;
+  constexpr int kWRows = kHeadDim / WORKERS;  // W rows per worker warp
+  static_assert(THREADS % 32 == 0 && THREADS / 32 >= kPoolWarps, "pooling uses 8 warps");
+  static_assert(WORKERS * 32 <= THREADS && kWRows % 8 == 0, "8 W rows per reduction");
+  static_assert(kHeadDim % QTHREADS == 0 && QFIRST + QTHREADS <= THREADS, "mean query threads");
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t bh = (int64_t)b * p.Hkv + h;
+  int L = __ldg(p.seqlens + b);
+  L = max(0, min(L, p.max_blocks * p.bs));
+  const int nb = ceil_div_i(L, p.bs);
+  const int nchunks = ceil_div_i(nb, CHUNK_ROWS);
+  float* kb_row = p.kbar + bh * p.max_blocks * kHeadDim;
+  const int k_row = __ldg(p.k_per_seq + b);
+  bool ok = true;
+
+  // the first chunks of the row go out before anything else
+  if (tid == 0) {
+    for (int c = 0; c < NBUF && c < nchunks; ++c) {
+      const uint32_t slot = (seq + c) % NBUF;
+      const uint32_t bytes = (uint32_t)min(CHUNK_ROWS, nb - c * CHUNK_ROWS) * kHeadDim * 4;
+      mbar_arrive_expect_tx(&bars[slot], bytes);
+      bulk_copy_g2s(ring.slot[slot], kb_row + (int64_t)c * CHUNK_ROWS * kHeadDim, bytes,
+                    &bars[slot]);
+    }
+  }
+
+  // KV append: the new token's K and V rows of head h at position L - 1
+  const bool append = p.k_new != nullptr && L > 0;
+  bool bad_page = false;
+  if (append) {
+    const int64_t page = page_of(p.page_table, b, (L - 1) / p.bs, p.max_blocks);
+    bad_page = page < 0 || page >= p.num_pages;
+    if (warp == 0 && !bad_page) {
+      const int64_t off = page * p.stride_page + (int64_t)((L - 1) % p.bs) * p.stride_token +
+                          (int64_t)h * p.stride_head + 4 * lane;
+      const int64_t src = ((int64_t)b * p.Hkv + h) * kHeadDim + 4 * lane;
+      *reinterpret_cast<uint2*>(p.k_pool_w + off) = __ldg(reinterpret_cast<const uint2*>(p.k_new + src));
+      *reinterpret_cast<uint2*>(p.v_pool_w + off) = __ldg(reinterpret_cast<const uint2*>(p.v_new + src));
+    }
+    __syncthreads();  // the pooled-key refresh below reads the appended row
+  }
+
+  // newest block's pooled key (incremental update), warps 0..7
+  const bool refresh = p.incremental && nb > 0;
+  int valid_new = 0;
+  if (refresh) {
+    valid_new = L - (nb - 1) * p.bs;
+    const int64_t page = page_of(p.page_table, b, nb - 1, p.max_blocks);
+    const bool bad = page < 0 || page >= p.num_pages;
+    bad_page |= bad;
+    if (warp < kPoolWarps && !bad) {
+      const uint16_t* base =
+          p.k_pool + page * p.stride_page + (int64_t)h * p.stride_head + 4 * lane;
+      const float4 a = append ? pool_warp_partial_l2(base, p.stride_token, valid_new, warp)
+                              : pool_warp_partial(base, p.stride_token, valid_new, warp);
+      *reinterpret_cast<float4*>(&gs.part[warp * kHeadDim + 4 * lane]) = a;
+    }
+  }
+  // this warp's rows of W[h] (rows warp + WORKERS * i), in flight meanwhile
+  float4 wrow[kWRows];
+  if (warp < WORKERS) {
+    const float* W = p.w_gate + (int64_t)h * kHeadDim * kHeadDim;
+#pragma unroll
+    for (int r = 0; r < kWRows; ++r)
+      wrow[r] = __ldg(reinterpret_cast<const float4*>(W + (warp + r * WORKERS) * kHeadDim +
+                                                      4 * lane));
+  }
+  // mean query of the group
+  if (tid >= QFIRST && tid < QFIRST + QTHREADS) {
+#pragma unroll
+    for (int m = 0; m < kHeadDim / QTHREADS; ++m) {
+      const int d = tid - QFIRST + m * QTHREADS;
+      const uint16_t* qg = p.q + ((int64_t)b * p.Hq + (int64_t)h * p.G) * kHeadDim + d;
+      float s = 0.f;
+      for (int g = 0; g < p.G; ++g) s += __uint_as_float((uint32_t)__ldg(qg + g * kHeadDim) << 16);
+      gs.qbar[d] = s / (float)p.G;
+    }
+  }
+  __syncthreads();
+  if (refresh && tid < kHeadDim) {
+    float v = 0.f;
+    if (!bad_page) v = pool_finish(gs.part, tid, valid_new);
+    gs.newest[tid] = v;
+    kb_row[(int64_t)(nb - 1) * kHeadDim + tid] = v;
+  }
+  if (bad_page && tid == 0) flag_status(p.status, SEER_DEV_BAD_PAGE);
+  // g = gate_scale * W[h] qbar, 8 rows per reduction
+  if (warp < WORKERS) {
+    const float4 qv = *reinterpret_cast<const float4*>(&gs.qbar[4 * lane]);
+#pragma unroll
+    for (int g8 = 0; g8 < kWRows / 8; ++g8) {
+      float4 w8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w8[i] = wrow[g8 * 8 + i];
+      const float v = warp_dot4_x8(w8, qv);
+      if ((lane & 3) == 0)
+        gs.gvec[warp + (g8 * 8 + ((lane >> 2) & 7)) * WORKERS] = __fmul_rn(v, p.gate_scale);
+    }
+  }
+  __syncthreads();
+
+  // scores, chunk by chunk; thread 0 refills each buffer once it is read
+  const float4 gv = *reinterpret_cast<const float4*>(&gs.gvec[4 * lane]);
+  float* scores_out = p.scores + bh * p.max_blocks;
+  bool bad = false;
+  for (int c = 0; c < nchunks; ++c) {
+    const uint32_t slot = (seq + c) % NBUF;
+    if (ok && !mbar_wait(&bars[slot], ((seq + c) / NBUF) & 1)) {
+      flag_status(p.status, SEER_DEV_TIMEOUT);
+      ok = false;
+    }
+    const int rows = min(CHUNK_ROWS, nb - c * CHUNK_ROWS);
+    const float* buf = ring.slot[slot];
+    if (warp < WORKERS) {  // this warp's 8 rows warp + WORKERS * i, one reduction
+      float4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = warp + i * WORKERS;
+        const int j = c * CHUNK_ROWS + r;
+        v[i] = (r >= rows) ? make_float4(0.f, 0.f, 0.f, 0.f)
+               : (refresh && j == nb - 1)
+                   ? *reinterpret_cast<const float4*>(&gs.newest[4 * lane])
+                   : *reinterpret_cast<const float4*>(&buf[r * kHeadDim + 4 * lane]);
+      }
+      const float sc = warp_dot4_x8(v, gv);
+      const int r = warp + ((lane >> 2) & 7) * WORKERS;
+      if ((lane & 3) == 0 && r < rows) {
+        const int j = c * CHUNK_ROWS + r;
+        gs.scores[j] = sc;
+        scores_out[j] = sc;
+        bad |= !isfinite(sc);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();  // every warp is done with this buffer
+    if (tid == 0 && ok && c + NBUF < nchunks) {
+      const int cn = c + NBUF;
+      const uint32_t bytes = (uint32_t)min(CHUNK_ROWS, nb - cn * CHUNK_ROWS) * kHeadDim * 4;
+      mbar_arrive_expect_tx(&bars[slot], bytes);
+      bulk_copy_g2s(ring.slot[slot], kb_row + (int64_t)cn * CHUNK_ROWS * kHeadDim, bytes,
+                    &bars[slot]);
+    }
+  }
+  seq += (uint32_t)nchunks;
+  if (bad) flag_status(p.status, SEER_DEV_NONFINITE_SCORE);
+  for (int j = nb + tid; j < p.max_blocks; j += THREADS) scores_out[j] = -INFINITY;
+  if (p.scores_only) return ok;  // uniform: the cross-head select runs next
+  __syncthreads();
+
+  constexpr int kLongItems = (kMaxBlocks + THREADS - 1) / THREADS;
+  int32_t* idx_row = p.idx + bh * p.k_max;
+  if (nb <= THREADS)
+    select_topk_binned<THREADS, 1>(gs.scores, nb, k_row, p.force_newest, p.k_max, idx_row,
+                                   p.n_sel + bh, p.status, gs.sel);
+  else if (nb <= 2 * THREADS)
+    select_topk_binned<THREADS, 2>(gs.scores, nb, k_row, p.force_newest, p.k_max, idx_row,
+                                   p.n_sel + bh, p.status, gs.sel);
+  else
+    select_topk_binned<THREADS, kLongItems>(gs.scores, nb, k_row, p.force_newest, p.k_max,
+                                            idx_row, p.n_sel + bh, p.status, gs.sel);
+  return ok;
+}
+
+}  // namespace seer

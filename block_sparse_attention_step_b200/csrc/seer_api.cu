@@ -114,9 +114,16 @@ seer_status check_pool(const seer_dims* d, const uint16_t* pool) {
     if (st_ != SEER_OK) return st_;        \
   } while (0)
 
-#define SEER_CUDA(expr)                               \
-  do {                                                \
-    if ((expr) != cudaSuccess) return SEER_ERR_CUDA;  \
+// the CUDA error behind this host thread's last SEER_ERR_CUDA
+static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+#define SEER_CUDA(expr)                   \
+  do {                                    \
+    const cudaError_t seer_e_ = (expr);   \
+    if (seer_e_ != cudaSuccess) {         \
+      g_last_cuda_error = seer_e_;        \
+      return SEER_ERR_CUDA;               \
+    }                                     \
   } while (0)
 
 struct Workspace {
@@ -125,7 +132,9 @@ struct Workspace {
   int32_t* n_sel;
   float* o_part;
   float* lse_part;
-  uint32_t* work_counter;  // the decode grid's item counter (2 words)
+  uint32_t* work_counter;  // control words: decode item counter (2), epoch, phase counters
+  uint32_t* row_flag;      // [B][Hkv] single-launch step: row selection published
+  size_t ctl_bytes;        // from work_counter to the end of row_flag
   size_t bytes;
 };
 
@@ -144,7 +153,9 @@ Workspace carve(const seer_dims* d, int32_t k_max, int32_t S, void* base) {
   w.n_sel = reinterpret_cast<int32_t*>(take(bh * sizeof(int32_t)));
   w.o_part = reinterpret_cast<float*>(take(bq * S * kHeadDim * sizeof(float)));
   w.lse_part = reinterpret_cast<float*>(take(bq * S * sizeof(float)));
-  w.work_counter = reinterpret_cast<uint32_t*>(take(2 * sizeof(uint32_t)));
+  w.work_counter = reinterpret_cast<uint32_t*>(take(8 * sizeof(uint32_t)));
+  w.row_flag = reinterpret_cast<uint32_t*>(take(bh * sizeof(uint32_t)));
+  w.ctl_bytes = round256(8 * sizeof(uint32_t)) + round256(bh * sizeof(uint32_t));
   w.bytes = off;
   return w;
 }
@@ -205,6 +216,10 @@ static seer_status decode_prepare(const seer_dims* d, const uint16_t* q, const u
 extern "C" {
 
 int32_t seer_version(void) { return 10000; }
+
+const char* seer_last_cuda_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 const char* seer_status_string(seer_status s) {
   switch (s) {
@@ -462,6 +477,8 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   if (a == nullptr || a->k_per_seq == nullptr || a->kbar == nullptr) return SEER_ERR_INVALID_ARG;
   if (a->update_kbar < 0 || a->update_kbar > 2) return SEER_ERR_INVALID_ARG;
   if (a->unified_heads != 0 && a->unified_heads != 1) return SEER_ERR_INVALID_ARG;
+  if ((a->k_new == nullptr) != (a->v_new == nullptr)) return SEER_ERR_INVALID_ARG;
+  if (a->k_new && (!aligned(a->k_new, 8) || !aligned(a->v_new, 8))) return SEER_ERR_UNSUPPORTED;
   if (a->k_max < 1 || a->num_splits < 1) return SEER_ERR_INVALID_ARG;
   if (a->workspace == nullptr || !aligned(a->workspace, 256)) return SEER_ERR_WORKSPACE;
   const Workspace w = carve(d, a->k_max, a->num_splits, a->workspace);
@@ -481,7 +498,7 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
     SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
                             stream));
   // a0 (incremental) + a1 + a2 in one kernel; same results as the three calls
-  GateSelectParams g;
+  GateSelectParams g = {};
   g.q = a->q;
   g.w_gate = a->w_gate;
   g.kbar = a->kbar;
@@ -492,6 +509,12 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   g.n_sel = w.n_sel;
   g.status = a->dev_status;
   g.k_pool = a->k_pool;
+  // the KV append writes the caller's pools (their own buffers, given as const
+  // because nothing else in the step writes them)
+  g.k_pool_w = const_cast<uint16_t*>(a->k_pool);
+  g.v_pool_w = const_cast<uint16_t*>(a->v_pool);
+  g.k_new = a->k_new;
+  g.v_new = a->v_new;
   g.page_table = a->page_table;
   g.incremental = a->update_kbar == 1 ? 1 : 0;
   g.num_pages = d->num_pages;
@@ -549,6 +572,78 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
     m.k_max = a->k_max;
     SEER_CUDA(run_block_mass(m, d->batch, stream));
   }
+  return SEER_OK;
+}
+
+seer_status seer_step_workspace_init(const seer_dims* d, int32_t k_max, int32_t num_splits,
+                                     void* workspace, size_t workspace_bytes,
+                                     seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (k_max < 1 || num_splits < 1) return SEER_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned(workspace, 256)) return SEER_ERR_WORKSPACE;
+  const Workspace w = carve(d, k_max, num_splits, workspace);
+  if (workspace_bytes < w.bytes) return SEER_ERR_WORKSPACE;
+  SEER_CUDA(cudaMemsetAsync(w.work_counter, 0, w.ctl_bytes, stream));
+  return SEER_OK;
+}
+
+seer_status seer_decode_step_fused(const seer_dims* d, const seer_step_args* a,
+                                   seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (a == nullptr || a->k_per_seq == nullptr || a->kbar == nullptr) return SEER_ERR_INVALID_ARG;
+  if (a->update_kbar < 0 || a->update_kbar > 2) return SEER_ERR_INVALID_ARG;
+  if (a->k_max < 1 || a->num_splits < 1) return SEER_ERR_INVALID_ARG;
+  if ((a->k_new == nullptr) != (a->v_new == nullptr)) return SEER_ERR_INVALID_ARG;
+  if (a->unified_heads != 0 || a->block_lse != nullptr || a->block_mass != nullptr)
+    return SEER_ERR_UNSUPPORTED;  // those run through seer_decode_step
+  if (a->workspace == nullptr || !aligned(a->workspace, 256)) return SEER_ERR_WORKSPACE;
+  const Workspace w = carve(d, a->k_max, a->num_splits, a->workspace);
+  if (a->workspace_bytes < w.bytes) return SEER_ERR_WORKSPACE;
+  if (!a->q || !a->w_gate || !a->seqlens || !a->out) return SEER_ERR_INVALID_ARG;
+  if (!aligned(a->w_gate, 16) || !aligned(a->kbar, 16)) return SEER_ERR_UNSUPPORTED;
+  if (a->k_new && (!aligned(a->k_new, 8) || !aligned(a->v_new, 8))) return SEER_ERR_UNSUPPORTED;
+  DecodeLaunch L;
+  SEER_TRY(decode_prepare(d, a->q, a->k_pool, a->v_pool, a->page_table, a->seqlens, w.idx,
+                          w.n_sel, a->k_max, a->num_splits, a->softmax_scale, w.o_part,
+                          w.lse_part, w.work_counter, a->dev_status, &L));
+  if (a->update_kbar == 2)  // a full rebuild is its own pass over K (prefill time)
+    SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
+                            stream));
+  FusedParams f = {};
+  GateSelectParams& g = f.gate;
+  g.q = a->q;
+  g.w_gate = a->w_gate;
+  g.kbar = a->kbar;
+  g.seqlens = a->seqlens;
+  g.k_per_seq = a->k_per_seq;
+  g.scores = w.scores;
+  g.idx = w.idx;
+  g.n_sel = w.n_sel;
+  g.status = a->dev_status;
+  g.k_pool = a->k_pool;
+  g.k_pool_w = const_cast<uint16_t*>(a->k_pool);
+  g.v_pool_w = const_cast<uint16_t*>(a->v_pool);
+  g.k_new = a->k_new;
+  g.v_new = a->v_new;
+  g.page_table = a->page_table;
+  g.incremental = a->update_kbar == 1 ? 1 : 0;
+  g.num_pages = d->num_pages;
+  g.stride_page = d->stride_page;
+  g.stride_token = d->stride_token;
+  g.stride_head = d->stride_head;
+  g.Hq = d->num_q_heads;
+  g.Hkv = d->num_kv_heads;
+  g.G = d->num_q_heads / d->num_kv_heads;
+  g.bs = d->block_size;
+  g.max_blocks = d->max_blocks;
+  g.k_max = a->k_max;
+  g.force_newest = a->force_newest ? 1 : 0;
+  g.gate_scale = a->gate_scale;
+  f.ctl = w.work_counter;
+  f.row_flag = w.row_flag;
+  f.out = a->out;
+  f.lse_out = a->lse_out;
+  SEER_CUDA(run_fused_step(L.tk, L.tv, L.p, f, num_sms_current(), stream));
   return SEER_OK;
 }
 

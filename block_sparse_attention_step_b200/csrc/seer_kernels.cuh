@@ -47,6 +47,10 @@ struct GateSelectParams {
   int32_t* n_sel;
   int32_t* status;
   const uint16_t* k_pool;     // for the incremental pooled-key refresh
+  uint16_t* k_pool_w;         // the same pools, written by the KV append
+  uint16_t* v_pool_w;
+  const uint16_t* k_new;      // optional [B][Hkv][D]: the token appended at L - 1
+  const uint16_t* v_new;
   const int32_t* page_table;
   int incremental;
   int64_t num_pages, stride_page, stride_token, stride_head;
@@ -78,6 +82,20 @@ struct DecodeParams {
   uint32_t* work_counter;
 };
 
+// The single-launch step: the decode kernel with the gate rows before it and
+// the combine after it, in one cooperative grid.  Control words (zero before
+// the first launch; every completed launch leaves them ready for the next):
+//   ctl[0] next item, ctl[1] schedulers done (the decode's item counter),
+//   ctl[2] launch epoch, ctl[3] CTAs done decoding, ctl[4] CTAs done
+//   combining; row_flag[bh] = epoch + 1 once row bh's selection is out.
+struct FusedParams {
+  GateSelectParams gate;
+  uint32_t* ctl;
+  uint32_t* row_flag;
+  uint16_t* out;
+  float* lse_out;
+};
+
 struct MassParams {
   const int32_t* idx;
   const int32_t* n_sel;
@@ -103,6 +121,8 @@ cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t strea
 cudaError_t run_unified_select(const SelectParams& p, int B, cudaStream_t stream, bool pdl);
 cudaError_t run_fill_k(const int32_t* seqlens, int B, int bs, int permille, int budget,
                        int32_t* k_out, cudaStream_t stream);
+cudaError_t run_fused_step(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                           const FusedParams& f, int num_sms, cudaStream_t stream);
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                               int num_sms, cudaStream_t stream, bool pdl);
 cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream, bool pdl);

@@ -34,7 +34,8 @@
 //     outputs into o_part / lse_part: with two slots no warp waits for
 //     another at item boundaries.
 // Every mbarrier wait is bounded (SEER_DEV_TIMEOUT); nothing traps.
-#include "seer_kernels.cuh"
+#include "gate_row.cuh"
+#include "combine_core.cuh"
 
 namespace seer {
 
@@ -73,6 +74,18 @@ struct DecodeShape {
   static constexpr size_t kO = kML + kMSlots * kMLBytes;
   __host__ __device__ static size_t o_slot_floats(int G) { return (size_t)kMathWarps * G * kOStride; }
   static size_t smem_bytes(int G) { return 1024 + kO + kMSlots * o_slot_floats(G) * 4; }
+  // The single-launch step's gate rows stream kbar through the stage ring
+  // plus one or two more 32 KB slots (192 KB in flight when they fit), and
+  // keep their scratch and chunk mbarriers in the merge area -- all idle
+  // until the decode starts.
+  static constexpr size_t kGateBars = (kML + sizeof(GateRowScratch) + 7) & ~size_t(7);
+  static constexpr size_t kGateExtra = (kGateBars + 8 * (kStages + 2) + 127) & ~size_t(127);
+  static constexpr int kGateSlots =
+      (1024 + kGateExtra + 2 * kStageBytes + 512 <= 227 * 1024) ? kStages + 2 : kStages + 1;
+  static size_t smem_bytes_fused(int G) {
+    const size_t gate = 1024 + kGateExtra + (size_t)(kGateSlots - kStages) * kStageBytes;
+    return smem_bytes(G) > gate ? smem_bytes(G) : gate;
+  }
   static_assert(kRing % 1024 == 0 && kStageBytes % 1024 == 0, "swizzled TMA tiles need 1 KB");
   static_assert(kQBuf % 16 == 0 && kQSlotBytes % 16 == 0, "bulk copy destinations need 16 B");
   static_assert(kBars % 8 == 0 && kRec % 8 == 0 && kEnt % 16 == 0 && kMBars % 8 == 0 &&
@@ -115,10 +128,18 @@ __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item,
   return c;
 }
 
-template <int NT, int STAGES, int MSLOTS, bool MASS>
+template <bool FUSED>
+__device__ __forceinline__ int ld_row_data(const int32_t* ptr) {
+  // rows written by other CTAs of the same grid must come through L2
+  if constexpr (FUSED) return __ldcg(ptr);
+  else return __ldg(ptr);
+}
+
+template <int NT, int STAGES, int MSLOTS, bool MASS, bool FUSED>
 __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p,
+                         const FusedParams f) {
   using Shape = DecodeShape<NT, STAGES, MSLOTS>;
   static_assert(Shape::kMathWarps == 8 && Shape::kGroups == 2, "merge order assumes 2 x 4 warps");
   constexpr int kStages = Shape::kStages;
@@ -175,6 +196,41 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
 
+  // ---- single-launch step, phase A: the gate rows of this CTA (all threads)
+  __shared__ uint32_t epoch_next;  // this launch's row-flag value
+  if constexpr (FUSED) {
+    constexpr int kSlots = Shape::kGateSlots;
+    static_assert(kStageBytes == 8 * kMathWarps * kHeadDim * 4, "a stage holds one kbar chunk");
+    GateRowScratch& gs = *reinterpret_cast<GateRowScratch*>(smem + Shape::kML);
+    uint64_t* gbar = reinterpret_cast<uint64_t*>(smem + Shape::kGateBars);
+    ChunkRing<kSlots> gring;
+#pragma unroll
+    for (int i = 0; i < kStages; ++i) gring.slot[i] = reinterpret_cast<float*>(ring + i * kStageBytes);
+#pragma unroll
+    for (int i = kStages; i < kSlots; ++i)
+      gring.slot[i] = reinterpret_cast<float*>(smem + Shape::kGateExtra +
+                                               (size_t)(i - kStages) * kStageBytes);
+    if (threadIdx.x == 0) {
+      epoch_next = *reinterpret_cast<volatile uint32_t*>(f.ctl + 2) + 1u;
+      for (int i = 0; i < kSlots; ++i) mbar_init(&gbar[i], 1);
+      fence_mbar_init();
+    }
+    __syncthreads();
+    uint32_t gseq = 0;
+    const int rows = p.B * p.Hkv;
+    for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+      gate_row<Shape::kThreads, kMathWarps, kSlots, kMathThreads, 64>(
+          f.gate, row / p.Hkv, row % p.Hkv, gring, gbar, gseq, gs);
+      __syncthreads();  // the row's indices, kbar row and appended K/V are written
+      if (threadIdx.x == 0) {
+        __threadfence();
+        fence_proxy_async_global();  // the appended rows are read by TMA elsewhere
+        st_release_gpu(f.row_flag + row, epoch_next);
+      }
+    }
+    __syncthreads();  // ring and merge area belong to the decode from here on
+  }
+
   if (warp == kMathWarps + 1) {
     // =============================================================== scheduler
     // Runs ahead of the copies: resolves each item's block indices and pages
@@ -191,12 +247,30 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     // while another runs dry and the CTAs finish together.
     const bool dyn = p.work_counter != nullptr;
     constexpr uint32_t kClaimAhead = 4;
+    // single-launch step: a row's indices are read only once its gate row has
+    // published them (bounded wait on the row flag, acquire)
+    auto row_ready = [&](int bh) {
+      if constexpr (FUSED) {
+        if (lane == 0 && ok) {
+          const long long t0 = clock64();
+          while (ld_acquire_gpu(f.row_flag + bh) != epoch_next) {
+            if (clock64() - t0 > (1ll << 31)) {
+              flag_status(p.status, SEER_DEV_TIMEOUT);
+              ok = 0;
+              break;
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+    };
     int item = (int)blockIdx.x;
     int L_cur = 0, n_cur = 0;
     if (item < p.num_items) {
       const int bh = item_bh(p, item);
+      row_ready(bh);
       L_cur = __ldg(p.seqlens + bh / p.Hkv);
-      n_cur = __ldg(p.n_sel + bh);
+      n_cur = ld_row_data<FUSED>(p.n_sel + bh);
     }
     int it_no = 0;
     for (; item < p.num_items && ok; ++it_no) {
@@ -204,8 +278,9 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       if (!dyn && item + (int)gridDim.x < p.num_items) {
         nxt = item + (int)gridDim.x;
         const int bh = item_bh(p, nxt);
+        row_ready(bh);
         L_nxt = __ldg(p.seqlens + bh / p.Hkv);
-        n_nxt = __ldg(p.n_sel + bh);
+        n_nxt = ld_row_data<FUSED>(p.n_sel + bh);
       }
       const ItemCoord ic = item_coord(p, item, L_cur, n_cur);
 
@@ -215,7 +290,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         const int i = base + lane;
         int cnt = 0;
         if (i < ic.hi) {
-          const int j = __ldg(p.idx + ic.row + i);
+          const int j = ld_row_data<FUSED>(p.idx + ic.row + i);
           if (j >= 0 && j < ic.nb) cnt = ceil_div_i(min(p.bs, ic.L - j * p.bs), kTileTokens);
           if (base == ic.lo) j0 = j;
         }
@@ -245,7 +320,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         const int i = base + lane;
         int j = -1, pg = 0, ne = 0;
         if (i < ic.hi) {
-          j = (base == ic.lo) ? j0 : __ldg(p.idx + ic.row + i);
+          j = (base == ic.lo) ? j0 : ld_row_data<FUSED>(p.idx + ic.row + i);
           if (j < 0 || j >= ic.nb) {
             flag_status(p.status, SEER_DEV_BAD_INDEX);
             j = -1;
@@ -311,8 +386,9 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         if (v < (unsigned)p.num_items) {
           nxt = (int)v;
           const int bh = item_bh(p, nxt);
+          row_ready(bh);
           L_nxt = __ldg(p.seqlens + bh / p.Hkv);
-          n_nxt = __ldg(p.n_sel + bh);
+          n_nxt = ld_row_data<FUSED>(p.n_sel + bh);
         }
       }
       item = nxt;
@@ -336,6 +412,9 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       if (atomicAdd(p.work_counter + 1, 1u) == gridDim.x - 1) {
         atomicExch(p.work_counter, 0u);
         atomicExch(p.work_counter + 1, 0u);
+        // every CTA read the epoch before its gate rows: the next launch's
+        // flags use the next value
+        if constexpr (FUSED) atomicAdd(f.ctl + 2, 1u);
       }
     }
     // terminator (the copy thread stops on a negative page)
@@ -386,6 +465,8 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       __threadfence_block();
       st_volatile(ent_head, ++head);
       if (e.x < 0) break;
+      // the newest block may hold a row appended by another CTA's gate row
+      if constexpr (FUSED) if (f.gate.k_new != nullptr) fence_proxy_async_global();
       const int slot = issued % kStages;
       const uint32_t phase = (issued / kStages) & 1;
       if (!mbar_wait(&empty_bar[slot], phase ^ 1)) {
@@ -732,19 +813,60 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     last_it = it_no;
   }
   if (last_it >= 0) merge_share(last_it);
+
+  // ---- single-launch step, phase C: the LSE combine of this CTA's rows by
+  // the math warps, once every math warp of the grid has written its last
+  // partials.  (Split-major items put every row's last split among the last
+  // items, so waiting for the whole grid costs little over waiting per row,
+  // and it takes one fence per warp instead of one per item.)
+  if constexpr (FUSED) {
+    __syncwarp();
+    if (lane == 0) __threadfence();  // this warp's partials are out
+    named_barrier_sync(1, kMathThreads);
+    if (threadIdx.x == 0) {  // one arrival per CTA
+      __threadfence();
+      atomicAdd(f.ctl + 3, 1u);
+      const uint32_t want = gridDim.x;
+      const long long t0 = clock64();
+      while (ld_acquire_gpu(f.ctl + 3) < want) {
+        __nanosleep(64);
+        if (clock64() - t0 > (1ll << 31)) {
+          flag_status(p.status, SEER_DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    named_barrier_sync(1, kMathThreads);
+    // one warp per (b, query head) row, spread over every math warp of the grid
+    const int qrows = p.B * p.Hq;
+    for (int q = blockIdx.x * kMathWarps + warp; q < qrows; q += gridDim.x * kMathWarps)
+      combine_row_warp(p.lse_part + (int64_t)q * p.S, p.o_part + (int64_t)q * p.S * kHeadDim,
+                       p.S, f.out + (int64_t)q * kHeadDim,
+                       f.lse_out != nullptr ? f.lse_out + q : nullptr, Load4L2{});
+    // the last CTA through its combine puts the two counters back to zero
+    // (every CTA has passed the wait above by then)
+    if (threadIdx.x == 0 && atomicAdd(f.ctl + 4, 1u) == gridDim.x - 1) {
+      atomicExch(f.ctl + 3, 0u);
+      atomicExch(f.ctl + 4, 0u);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ launcher
-template <int NT, int STAGES, int MSLOTS, bool MASS>
+template <int NT, int STAGES, int MSLOTS, bool MASS, bool FUSED>
 static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
-                                 const DecodeParams& p, int num_sms, cudaStream_t stream,
-                                 bool pdl) {
+                                 const DecodeParams& p, const FusedParams& f, int num_sms,
+                                 cudaStream_t stream, bool pdl) {
   using Shape = DecodeShape<NT, STAGES, MSLOTS>;
-  const size_t smem = Shape::smem_bytes(p.G);
-  auto kern = sparse_decode_kernel<NT, STAGES, MSLOTS, MASS>;
+  const size_t smem = FUSED ? Shape::smem_bytes_fused(p.G) : Shape::smem_bytes(p.G);
+  auto kern = sparse_decode_kernel<NT, STAGES, MSLOTS, MASS, FUSED>;
   static std::atomic<uint64_t> smem_set{0};
   cudaError_t e = ensure_smem_limit(kern, smem_set);
   if (e != cudaSuccess) return e;
+  // at most one CTA per SM and no more CTAs than items (there are never more
+  // gate rows than items); the single-launch step's CTAs wait on one another,
+  // so its grid must be co-resident: a cooperative launch fails rather than
+  // start one that is not
   const int grid = p.num_items < num_sms ? p.num_items : num_sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -752,11 +874,16 @@ static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  if (FUSED) {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tk, tv, p, f);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -770,15 +897,31 @@ cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, cons
       cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     optin = 227 * 1024;
   const bool mass = p.block_lse != nullptr;
+  const FusedParams none = {};
   if (p.G <= 8) {
-    if (DecodeShape<1, 4, 2>::smem_bytes(p.G) <= (size_t)optin)
-      return mass ? launch_decode<1, 4, 2, true>(tk, tv, p, num_sms, stream, pdl)
-                  : launch_decode<1, 4, 2, false>(tk, tv, p, num_sms, stream, pdl);
-    return mass ? launch_decode<1, 4, 1, true>(tk, tv, p, num_sms, stream, pdl)
-                : launch_decode<1, 4, 1, false>(tk, tv, p, num_sms, stream, pdl);
+    if (DecodeShape<1, 4, 2>::smem_bytes(p.G) + 256 <= (size_t)optin)  // + static shared
+      return mass ? launch_decode<1, 4, 2, true, false>(tk, tv, p, none, num_sms, stream, pdl)
+                  : launch_decode<1, 4, 2, false, false>(tk, tv, p, none, num_sms, stream, pdl);
+    return mass ? launch_decode<1, 4, 1, true, false>(tk, tv, p, none, num_sms, stream, pdl)
+                : launch_decode<1, 4, 1, false, false>(tk, tv, p, none, num_sms, stream, pdl);
   }
-  return mass ? launch_decode<2, 4, 1, true>(tk, tv, p, num_sms, stream, pdl)
-              : launch_decode<2, 4, 1, false>(tk, tv, p, num_sms, stream, pdl);
+  return mass ? launch_decode<2, 4, 1, true, false>(tk, tv, p, none, num_sms, stream, pdl)
+              : launch_decode<2, 4, 1, false, false>(tk, tv, p, none, num_sms, stream, pdl);
+}
+
+// The single-launch step (gate rows, decode, combine in one cooperative grid).
+cudaError_t run_fused_step(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                           const FusedParams& f, int num_sms, cudaStream_t stream) {
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    optin = 227 * 1024;
+  if (p.G <= 8) {
+    if (DecodeShape<1, 4, 2>::smem_bytes_fused(p.G) + 256 <= (size_t)optin)
+      return launch_decode<1, 4, 2, false, true>(tk, tv, p, f, num_sms, stream, false);
+    return launch_decode<1, 4, 1, false, true>(tk, tv, p, f, num_sms, stream, false);
+  }
+  return launch_decode<2, 4, 1, false, true>(tk, tv, p, f, num_sms, stream, false);
 }
 
 }  // namespace seer

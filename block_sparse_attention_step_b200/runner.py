@@ -48,6 +48,8 @@ class StepBuffers:
         self.kbar = torch.empty((B, Hkv, self.nb_max, D), dtype=torch.float32, device=dev)
         ws = seer.seer_step_workspace_bytes(self.dims, self.k_max, self.num_splits)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+        # control words of the single-launch step start at zero
+        seer.seer_step_workspace_init(self.dims, self.k_max, self.num_splits, self.workspace)
         self.out = torch.empty((B, w.q_heads, D), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((B, w.q_heads), dtype=torch.float32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -74,7 +76,9 @@ class StepBuffers:
                             ("idx", B * Hkv * self.k_max, torch.int32),
                             ("n_sel", B * Hkv, torch.int32),
                             ("o_part", B * Hq * S * D, torch.float32),
-                            ("lse_part", B * Hq * S, torch.float32)):
+                            ("lse_part", B * Hq * S, torch.float32),
+                            ("ctl", 8, torch.int32),
+                            ("row_flag", B * Hkv, torch.int32)):
             nbytes = n * 4
             out[name] = self.workspace[off:off + nbytes].view(dt)
             off += r256(nbytes)
@@ -90,7 +94,8 @@ class StepBuffers:
         seer.seer_pool_keys(self.dims, d["k_pool"], self.page_table, d["seqlens"], 0, self.kbar,
                             self.status, stream)
 
-    def args(self, update_kbar: int = 0, q=None) -> "seer.seer_step_args":
+    def args(self, update_kbar: int = 0, q=None, k_new=None,
+             v_new=None) -> "seer.seer_step_args":
         d = self.data
         return seer.step_args(d["q"] if q is None else q, d["k_pool"], d["v_pool"], self.page_table,
                               d["seqlens"], d["w_gate"], self.kbar, self.k_per_seq,
@@ -99,7 +104,8 @@ class StepBuffers:
                               softmax_scale=self.scale, workspace=self.workspace, out=self.out,
                               lse_out=self.lse, dev_status=self.status,
                               block_lse=self.block_lse, block_mass=self.block_mass,
-                              unified_heads=self.unified)
+                              unified_heads=self.unified, k_new=k_new, v_new=v_new)
 
-    def step(self, update_kbar: int = 0, stream=None, args=None):
-        seer.seer_decode_step(self.dims, args if args is not None else self.args(update_kbar), stream)
+    def step(self, update_kbar: int = 0, stream=None, args=None, fused: bool = False):
+        call = seer.seer_decode_step_fused if fused else seer.seer_decode_step
+        call(self.dims, args if args is not None else self.args(update_kbar), stream)

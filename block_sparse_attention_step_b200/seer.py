@@ -19,6 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libseer.so")
 
 SEER_OK = 0
+SEER_ERR_CUDA = 3
 STATUS_NAMES = {0: "SEER_OK", 1: "SEER_ERR_INVALID_ARG", 2: "SEER_ERR_UNSUPPORTED",
                 3: "SEER_ERR_CUDA", 4: "SEER_ERR_WORKSPACE"}
 DEV_NONFINITE_SCORE = 1
@@ -28,11 +29,13 @@ DEV_K_CLAMPED = 8
 DEV_TIMEOUT = 16
 
 EXPORTS = (
-    "seer_version", "seer_status_string", "seer_dims_default", "seer_k_from_sparsity",
+    "seer_version", "seer_status_string", "seer_last_cuda_error", "seer_dims_default",
+    "seer_k_from_sparsity",
     "seer_k_from_budget", "seer_fill_k", "seer_default_splits", "seer_step_workspace_bytes",
     "seer_pool_keys", "seer_gate_scores", "seer_block_select", "seer_block_select_unified",
     "seer_sparse_decode",
     "seer_combine", "seer_decode_step", "seer_decode_step_host", "seer_decode_step_noalloc",
+    "seer_decode_step_fused", "seer_step_workspace_init",
     "seer_block_lse_elems", "seer_sparse_decode_mass", "seer_block_mass",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -41,8 +44,10 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 class SeerError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} "
-                         f"({_lib().seer_status_string(status).decode()})")
+        detail = _lib().seer_status_string(status).decode()
+        if status == SEER_ERR_CUDA:
+            detail += ": " + _lib().seer_last_cuda_error().decode()
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
 class seer_dims(ctypes.Structure):
@@ -64,7 +69,8 @@ class seer_step_args(ctypes.Structure):
                 ("workspace_bytes", ctypes.c_size_t), ("out", ctypes.c_void_p),
                 ("lse_out", ctypes.c_void_p), ("dev_status", ctypes.c_void_p),
                 ("block_lse", ctypes.c_void_p), ("block_mass", ctypes.c_void_p),
-                ("unified_heads", ctypes.c_int32)]
+                ("unified_heads", ctypes.c_int32), ("k_new", ctypes.c_void_p),
+                ("v_new", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -73,6 +79,7 @@ _I = ctypes.c_int32
 _SIGS = {
     "seer_version": (_I, []),
     "seer_status_string": (ctypes.c_char_p, [_I]),
+    "seer_last_cuda_error": (ctypes.c_char_p, []),
     "seer_dims_default": (_I, [_I, _I, _I, _I, _I, _I, ctypes.c_int64, _D]),
     "seer_k_from_sparsity": (_I, [_I, _I, ctypes.POINTER(_I)]),
     "seer_k_from_budget": (_I, [_I, _I, _I, ctypes.POINTER(_I)]),
@@ -89,6 +96,8 @@ _SIGS = {
     "seer_decode_step": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_decode_step_host": (_I, [_D, ctypes.POINTER(seer_step_args), _P, _P, _P, _P]),
     "seer_decode_step_noalloc": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
+    "seer_decode_step_fused": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
+    "seer_step_workspace_init": (_I, [_D, _I, _I, _P, ctypes.c_size_t, _P]),
     "seer_block_lse_elems": (ctypes.c_size_t, [_D]),
     "seer_sparse_decode_mass": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P,
                                      _P, _P, _P, _P]),
@@ -245,7 +254,7 @@ def seer_combine(d, o_part, lse_part, num_splits, out, lse_out=None, stream=None
 def step_args(q, k_pool, v_pool, page_table, seqlens, w_gate, kbar, k_per_seq, *, update_kbar,
               force_newest, k_max, num_splits, gate_scale, softmax_scale, workspace, out,
               lse_out=None, dev_status=None, block_lse=None, block_mass=None,
-              unified_heads=False) -> seer_step_args:
+              unified_heads=False, k_new=None, v_new=None) -> seer_step_args:
     a = seer_step_args()
     a.q = _ptr(q, torch.bfloat16, "q", allow_none=True)
     a.k_pool = _ptr(k_pool, torch.bfloat16, "k_pool")
@@ -269,12 +278,26 @@ def step_args(q, k_pool, v_pool, page_table, seqlens, w_gate, kbar, k_per_seq, *
     a.block_lse = _ptr(block_lse, torch.float32, "block_lse", allow_none=True)
     a.block_mass = _ptr(block_mass, torch.float32, "block_mass", allow_none=True)
     a.unified_heads = int(bool(unified_heads))
+    a.k_new = _ptr(k_new, torch.bfloat16, "k_new", allow_none=True)
+    a.v_new = _ptr(v_new, torch.bfloat16, "v_new", allow_none=True)
     return a
 
 
 def seer_decode_step(d, args: seer_step_args, stream=None):
     _check("seer_decode_step", _lib().seer_decode_step(ctypes.byref(d), ctypes.byref(args),
                                                        _stream(stream)))
+
+
+def seer_decode_step_fused(d, args: seer_step_args, stream=None):
+    _check("seer_decode_step_fused", _lib().seer_decode_step_fused(ctypes.byref(d),
+                                                                   ctypes.byref(args),
+                                                                   _stream(stream)))
+
+
+def seer_step_workspace_init(d, k_max, num_splits, workspace, stream=None):
+    _check("seer_step_workspace_init", _lib().seer_step_workspace_init(
+        ctypes.byref(d), int(k_max), int(num_splits), _ptr(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream)))
 
 
 def seer_decode_step_host(d, args: seer_step_args, q_host, q_dev, out_host, stream=None):

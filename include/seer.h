@@ -115,6 +115,11 @@ SEER_API int32_t seer_version(void);
 /* Static text for a status code. */
 SEER_API const char *seer_status_string(seer_status s);
 
+/* The CUDA runtime's message for the error behind the last SEER_ERR_CUDA
+ * returned on the calling host thread ("no error" if there was none); a
+ * static string, owned by the runtime. */
+SEER_API const char *seer_last_cuda_error(void);
+
 /* Fill a seer_dims for the default pool layout [P][bs][Hkv][D]. */
 SEER_API seer_status seer_dims_default(int32_t batch, int32_t num_q_heads,
                               int32_t num_kv_heads, int32_t head_dim,
@@ -144,8 +149,11 @@ SEER_API int32_t seer_default_splits(const seer_dims *d, int32_t k_max,
                             int32_t num_sms);
 
 /* Bytes of caller workspace seer_decode_step needs (scores, idx, n_sel,
- * o_part, lse_part and the decode grid's 2-word item counter, each 256-byte
- * aligned).  The step initialises all of it; its contents need not be zero. */
+ * o_part, lse_part, then the control words: the decode grid's item counter,
+ * the single-launch step's epoch and phase counters, and its [B][Hkv] u32
+ * row flags;
+ * each part 256-byte aligned).  seer_decode_step initialises what it uses;
+ * seer_decode_step_fused needs seer_step_workspace_init once. */
 SEER_API size_t seer_step_workspace_bytes(const seer_dims *d, int32_t k_max,
                                  int32_t num_splits);
 
@@ -260,6 +268,13 @@ typedef struct seer_step_args {
   /* 0: each KV head selects its own blocks (seer_block_select); 1: one block
    * set per sequence shared by all its KV heads (seer_block_select_unified). */
   int32_t unified_heads;
+  /* Optional KV append (both NULL, or both [B][Hkv][D] bf16, 8-byte aligned):
+   * the step first writes the new token's K and V rows at position
+   * seqlens[b] - 1 of k_pool and v_pool (through the page table), then pools,
+   * gates and attends with them.  seqlens already counts the new token.  The
+   * pools are written only in this case. */
+  const uint16_t *k_new;
+  const uint16_t *v_new;
 } seer_step_args;
 
 SEER_API seer_status seer_decode_step(const seer_dims *d, const seer_step_args *a,
@@ -337,6 +352,35 @@ SEER_API seer_status seer_block_mass(const seer_dims *d, const int32_t *idx,
 
 SEER_API seer_status seer_decode_step_noalloc(const seer_dims *d,
                                               const seer_step_args *a,
+                                              seer_stream stream);
+
+/* ------------------------------------------------------ single-launch step
+ * The whole step in one cooperative launch (the persistent decode grid runs
+ * the gate rows first and the LSE combine last; next to the per-stage path,
+ * it removes the launch boundaries between gate + select, decode and
+ * combine): same arguments, same results bit for bit as seer_decode_step --
+ * including the optional KV append -- except that unified_heads and the block
+ * mass are not offered here (SEER_ERR_UNSUPPORTED; use seer_decode_step).
+ *   - The grid holds one CTA per SM and every CTA must be resident at once:
+ *     the launch fails with SEER_ERR_CUDA if they cannot be (other work
+ *     holding SMs).  CTAs wait on each other only through bounded waits on
+ *     flags in the workspace (SEER_DEV_TIMEOUT when one runs out).
+ *   - The workspace's control words must be zero before the first call:
+ *     seer_step_workspace_init once after allocating it (and again after a
+ *     call that flagged SEER_DEV_TIMEOUT).  Every completed call leaves them
+ *     ready for the next; calls that share a workspace must not overlap.
+ *   - update_kbar = 2 runs the full key pooling as its own launch first. */
+SEER_API seer_status seer_decode_step_fused(const seer_dims *d,
+                                            const seer_step_args *a,
+                                            seer_stream stream);
+
+/* Zeroes the control words of a step workspace (bytes from
+ * seer_step_workspace_bytes with the same k_max and num_splits); enqueued on
+ * `stream`.  Needed once before seer_decode_step_fused uses the workspace;
+ * seer_decode_step itself needs no initialised workspace. */
+SEER_API seer_status seer_step_workspace_init(const seer_dims *d, int32_t k_max,
+                                              int32_t num_splits, void *workspace,
+                                              size_t workspace_bytes,
                                               seer_stream stream);
 
 #ifdef __cplusplus

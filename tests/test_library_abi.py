@@ -106,7 +106,7 @@ def test_workspace_and_default_splits(lib):
     ws = seer.seer_step_workspace_bytes(d, 52, 8)
     r = lambda x: (x + 255) // 256 * 256
     expect = (r(16 * 8 * 512 * 4) + r(16 * 8 * 52 * 4) + r(16 * 8 * 4) +
-              r(16 * 40 * 8 * 128 * 4) + r(16 * 40 * 8 * 4) + r(2 * 4))
+              r(16 * 40 * 8 * 128 * 4) + r(16 * 40 * 8 * 4) + r(8 * 4) + r(16 * 8 * 4))
     assert ws == expect
     assert seer.seer_step_workspace_bytes(d, 0, 8) == 0
     s = seer.seer_default_splits(d, 52, 148)
