@@ -64,6 +64,11 @@ __all__ = [
     "unified_scores",
     "unified_scores_f32",
     "select_blocks_unified",
+    "pool_queries",
+    "prefill_gate_scores",
+    "prefill_select",
+    "prefill_attention",
+    "prefill_row",
 ]
 
 
@@ -361,3 +366,101 @@ def select_blocks_unified(per_head_scores, k: int, force_newest: bool) -> np.nda
     order, forced block and ascending output as ``select_blocks``; every KV
     head of the sequence then attends these blocks."""
     return select_blocks(unified_scores(per_head_scores), k, force_newest)
+
+
+# ---------------------------------------------------------------- prefill with query pooling
+#
+# SeerAttention-R removes query pooling to decode token by token (paper
+# summary page, Abstract: it extends SeerAttention, whose gate pools queries).
+# The prefill path here is that pooled form, in the notation of the decode
+# step.  Readings (the pages give no formula for it): query block i holds the
+# query tokens [i*bs, min((i+1)*bs, L)); its pooled query is the mean over
+# those tokens and over the G heads of the group; block j scores
+# gate_scale * (W qbar_i) . kbar_j for j <= i only (a query never sees later
+# keys); block i itself is always selected (it holds the query's own recent
+# keys, the prefill form of the forced newest block) and counts toward k;
+# every query token then attends, causally, the tokens of its block's chosen
+# blocks that do not come after it.
+
+
+def pool_queries(Q_group: np.ndarray, seqlen: int, block_size: int) -> np.ndarray:
+    """Pooled queries of one (sequence, KV head): Q_group [>= L][G][D];
+    returns qbar [NB][D], the mean over the valid tokens of query block i and
+    over the group's G heads."""
+    L = int(seqlen)
+    nb = num_blocks(L, block_size)
+    qbar = np.zeros((nb, Q_group.shape[2]), dtype=np.float64)
+    for i in range(nb):
+        lo, hi = i * block_size, min((i + 1) * block_size, L)
+        rows = Q_group[lo:hi].reshape(-1, Q_group.shape[2])
+        qbar[i] = rows.sum(axis=0) / float(rows.shape[0])
+    return qbar
+
+
+def prefill_gate_scores(Q_group: np.ndarray, W: np.ndarray, kbar: np.ndarray, seqlen: int,
+                        block_size: int, scale: float) -> np.ndarray:
+    """Block-to-block gate scores [NB][NB] of one (sequence, KV head): entry
+    (i, j) is scale * (W qbar_i) . kbar_j for j <= i and -inf above the
+    diagonal.  Written token by token and head by head and averaged last (the
+    mean of the per-query scores equals the score of the pooled query), not
+    in the order a GPU would use."""
+    L = int(seqlen)
+    nb = num_blocks(L, block_size)
+    out = np.full((nb, nb), -np.inf, dtype=np.float64)
+    for i in range(nb):
+        lo, hi = i * block_size, min((i + 1) * block_size, L)
+        acc = np.zeros(i + 1, dtype=np.float64)
+        count = 0
+        for t in range(lo, hi):
+            for g in range(Q_group.shape[1]):
+                acc += kbar[: i + 1] @ (W @ Q_group[t, g])
+                count += 1
+        out[i, : i + 1] = acc / count * float(scale)
+    return out
+
+
+def prefill_select(scores: np.ndarray, k_of_block) -> list:
+    """Per query block i: the top-k_i of row i over blocks 0..i with block i
+    forced (``select_blocks`` with the forced newest block on the causal
+    prefix).  k_of_block(i) gives k_i.  Returns a list of ascending arrays."""
+    return [select_blocks(scores[i, : i + 1], k_of_block(i), True) for i in range(scores.shape[0])]
+
+
+def prefill_attention(Q_group: np.ndarray, K: np.ndarray, V: np.ndarray, seqlen: int,
+                      selected: list, block_size: int, scale: float):
+    """Causal softmax attention of every query token over its query block's
+    selected key blocks: token t of block i, head g attends the keys s of the
+    blocks in selected[i] with s <= t (Agent Skill page, Step 4's masked
+    softmax, with the causal mask of a prefill).  Returns (out [L][G][D],
+    lse [L][G])."""
+    L = int(seqlen)
+    G, D = Q_group.shape[1], V.shape[1]
+    out = np.zeros((L, G, D), dtype=np.float64)
+    lse = np.full((L, G), -np.inf, dtype=np.float64)
+    for i, blocks in enumerate(selected):
+        keep = np.zeros(L, dtype=bool)
+        for j in blocks:
+            keep[int(j) * block_size:min((int(j) + 1) * block_size, L)] = True
+        for t in range(i * block_size, min((i + 1) * block_size, L)):
+            mask = keep.copy()
+            mask[t + 1:] = False
+            keys = np.nonzero(mask)[0]
+            x = (Q_group[t] @ K[keys].T) * float(scale)          # [G][n]
+            m = x.max(axis=1, keepdims=True)
+            e = np.exp(x - m)
+            tot = e.sum(axis=1, keepdims=True)
+            out[t] = (e / tot) @ V[keys]
+            lse[t] = (m + np.log(tot))[:, 0]
+    return out, lse
+
+
+def prefill_row(Q_group, W, K, V, seqlen, block_size, k_of_block, gate_scale, softmax_scale):
+    """The prefill path for one (sequence, KV head): pooled keys, gate scores
+    of the pooled queries, per-block selection, causal block-sparse attention.
+    Returns a dict with kbar, scores, selected, out, lse."""
+    kbar = pool_keys(K, seqlen, block_size)
+    scores = prefill_gate_scores(Q_group, W, kbar, seqlen, block_size, gate_scale)
+    selected = prefill_select(scores, k_of_block)
+    out, lse = prefill_attention(Q_group, K, V, seqlen, selected, block_size, softmax_scale)
+    return {"kbar": kbar, "scores": scores, "selected": selected, "out": out, "lse": lse}
+

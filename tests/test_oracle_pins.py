@@ -382,3 +382,75 @@ def test_unified_f32_aggregate_is_the_in_order_fp32_sum():
     # within fp32 rounding of the fp64 sum
     np.testing.assert_allclose(got, O.unified_scores(ph), rtol=0, atol=4e-6)
 
+
+# ---------------------------------------------------------------- prefill with query pooling
+
+def test_prefill_dense_equals_library_causal_attention():
+    """Every block selected: the prefill path is causal attention, checked
+    against torch's fp64 scaled_dot_product_attention(is_causal=True)."""
+    import torch
+    rng = np.random.default_rng(21)
+    L, G, D, bs = 150, 3, 16, 32
+    Q, K, V = rng.standard_normal((L, G, D)), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    nb = O.num_blocks(L, bs)
+    sel = [np.arange(i + 1) for i in range(nb)]
+    out, lse = O.prefill_attention(Q, K, V, L, sel, bs, 0.25)
+    q = torch.from_numpy(Q).permute(1, 0, 2)[None]            # [1][G][L][D]
+    k = torch.from_numpy(K)[None, None].expand(1, G, L, D)
+    v = torch.from_numpy(V)[None, None].expand(1, G, L, D)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, scale=0.25)
+    np.testing.assert_allclose(out, ref[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+    x = np.einsum("tgd,sd->gts", Q, K) * 0.25
+    x[:, np.triu(np.ones((L, L), bool), 1)] = -np.inf
+    from scipy.special import logsumexp
+    np.testing.assert_allclose(lse, logsumexp(x, axis=2).T, rtol=1e-12)
+
+
+def test_prefill_sparse_equals_library_masked_attention():
+    import torch
+    rng = np.random.default_rng(22)
+    L, G, D, bs = 200, 2, 8, 32
+    Q, K, V = rng.standard_normal((L, G, D)), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    nb = O.num_blocks(L, bs)
+    sel = [np.array(sorted(set(rng.choice(i + 1, size=min(i + 1, 2), replace=False).tolist()) | {i}))
+           for i in range(nb)]
+    out, _ = O.prefill_attention(Q, K, V, L, sel, bs, 0.3)
+    allowed = np.zeros((L, L), bool)
+    for i, blocks in enumerate(sel):
+        rows = slice(i * bs, min((i + 1) * bs, L))
+        for j in blocks:
+            allowed[rows, j * bs:min((j + 1) * bs, L)] = True
+    allowed &= ~np.triu(np.ones((L, L), bool), 1)
+    q = torch.from_numpy(Q).permute(1, 0, 2)[None]
+    k = torch.from_numpy(K)[None, None].expand(1, G, L, D)
+    v = torch.from_numpy(V)[None, None].expand(1, G, L, D)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(allowed),
+                                                           scale=0.3)
+    np.testing.assert_allclose(out, ref[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_closed_forms_and_hand_case():
+    rng = np.random.default_rng(23)
+    L, G, D, bs = 70, 2, 4, 32
+    Q, K, V = rng.standard_normal((L, G, D)), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    # token 0 sees only itself; the first token of any block with only its own
+    # block selected sees only itself too
+    out, lse = O.prefill_attention(Q, K, V, L, [np.array([0]), np.array([1]), np.array([2])], bs, 1.0)
+    np.testing.assert_allclose(out[0], np.stack([V[0]] * G), rtol=0, atol=0)
+    np.testing.assert_allclose(out[32], np.stack([V[32]] * G), rtol=0, atol=0)
+    np.testing.assert_allclose(lse[0], Q[0] @ K[0], rtol=1e-14)
+    # pooled queries: the mean over the block's tokens and the group's heads
+    qbar = O.pool_queries(Q, L, bs)
+    np.testing.assert_allclose(qbar[2], Q[64:70].reshape(-1, D).mean(axis=0), rtol=1e-14)
+    # gate by hand: W = I, kbar = e_j: score(i, j) = qbar_i[j] * scale, -inf above the diagonal
+    kb = np.eye(3, D)
+    sc = O.prefill_gate_scores(Q, np.eye(D), kb, L, bs, 0.5)
+    np.testing.assert_allclose(sc[2, :3], qbar[2, :3] * 0.5, rtol=1e-13)
+    assert np.isneginf(sc[0, 1]) and np.isneginf(sc[1, 2])
+    # selection: the diagonal block is always in and counts toward k
+    s = np.array([[0, -np.inf, -np.inf], [5, 1, -np.inf], [5, 9, -3]], float)
+    got = O.prefill_select(s, lambda i: 1)
+    assert [g.tolist() for g in got] == [[0], [1], [2]]
+    got = O.prefill_select(s, lambda i: 2)
+    assert [g.tolist() for g in got] == [[0], [0, 1], [1, 2]]
+
