@@ -647,6 +647,75 @@ seer_status seer_decode_step_fused(const seer_dims* d, const seer_step_args* a,
   return SEER_OK;
 }
 
+int32_t seer_prefill_k_max(const seer_dims* d, int32_t sparsity_permille, int32_t budget_tokens) {
+  if (check_dims(d) != SEER_OK) return 0;
+  int32_t k = 0;
+  const seer_status st = budget_tokens > 0
+                             ? seer_k_from_budget(d->max_blocks, budget_tokens, d->block_size, &k)
+                             : seer_k_from_sparsity(d->max_blocks, sparsity_permille, &k);
+  return st == SEER_OK ? k : 0;
+}
+
+size_t seer_prefill_workspace_bytes(const seer_dims* d, int32_t k_max) {
+  if (check_dims(d) != SEER_OK || k_max < 1) return 0;
+  const size_t rows = (size_t)d->batch * d->num_kv_heads * d->max_blocks;
+  return round256(rows * k_max * sizeof(int32_t)) + round256(rows * sizeof(int32_t));
+}
+
+seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_stream stream) {
+  SEER_TRY(check_dims(d));
+  if (a == nullptr || !a->q || !a->k_pool || !a->v_pool || !a->seqlens || !a->w_gate || !a->kbar ||
+      !a->out)
+    return SEER_ERR_INVALID_ARG;
+  if (a->sparsity_permille < 0 || a->sparsity_permille > 1000 || a->budget_tokens < 0)
+    return SEER_ERR_INVALID_ARG;
+  if (a->k_max < 1 || a->k_max > d->max_blocks) return SEER_ERR_INVALID_ARG;
+  if (a->workspace == nullptr || !aligned(a->workspace, 256) ||
+      a->workspace_bytes < seer_prefill_workspace_bytes(d, a->k_max))
+    return SEER_ERR_WORKSPACE;
+  if (!aligned(a->q, 16) || !aligned(a->out, 16) || !aligned(a->w_gate, 16) || !aligned(a->kbar, 16))
+    return SEER_ERR_UNSUPPORTED;
+  SEER_TRY(check_pool(d, a->k_pool));
+  SEER_TRY(check_pool(d, a->v_pool));
+  const int token_inner = d->stride_token < d->stride_head ? 1 : 0;
+  CUtensorMap tk, tv;
+  SEER_TRY(make_kv_map(a->k_pool, d, token_inner, &tk));
+  SEER_TRY(make_kv_map(a->v_pool, d, token_inner, &tv));
+  const size_t rows = (size_t)d->batch * d->num_kv_heads * d->max_blocks;
+  PrefillParams p = {};
+  p.q = a->q;
+  p.w_gate = a->w_gate;
+  p.kbar = a->kbar;
+  p.page_table = a->page_table;
+  p.seqlens = a->seqlens;
+  p.scores = a->scores_out;
+  p.idx = reinterpret_cast<int32_t*>(a->workspace);
+  p.n_sel = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a->workspace) +
+                                       round256(rows * a->k_max * sizeof(int32_t)));
+  p.out = a->out;
+  p.lse = a->lse_out;
+  p.status = a->dev_status;
+  p.B = d->batch;
+  p.Hq = d->num_q_heads;
+  p.Hkv = d->num_kv_heads;
+  p.G = d->num_q_heads / d->num_kv_heads;
+  p.bs = d->block_size;
+  p.max_blocks = d->max_blocks;
+  p.k_max = a->k_max;
+  p.sparsity_permille = a->sparsity_permille;
+  p.budget_tokens = a->budget_tokens;
+  p.token_inner = token_inner;
+  p.num_pages = d->num_pages;
+  p.gate_scale = a->gate_scale;
+  p.scale_log2 = a->softmax_scale * kLog2e;
+  if (a->pool_keys)
+    SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
+                            stream));
+  SEER_CUDA(run_prefill_gate_select(p, stream));
+  SEER_CUDA(run_prefill_attention(tk, tv, p, stream));
+  return SEER_OK;
+}
+
 seer_status seer_decode_step_host(const seer_dims* d, const seer_step_args* a,
                                   const uint16_t* q_host, uint16_t* q_dev, uint16_t* out_host,
                                   seer_stream stream) {

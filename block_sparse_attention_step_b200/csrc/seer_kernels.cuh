@@ -82,6 +82,33 @@ struct DecodeParams {
   uint32_t* work_counter;
 };
 
+// Prefill with query pooling: query block i (bs tokens) is gated with the
+// mean of its queries over tokens and the group's heads against the pooled
+// keys of blocks 0..i, block i is always selected, and every query token
+// attends causally over its block's selection.
+struct PrefillParams {
+  const uint16_t* q;        // [B][Lq][Hq][D], Lq = max_blocks * bs
+  const float* w_gate;      // [Hkv][D][D]
+  const float* kbar;        // [B][Hkv][max_blocks][D] pooled keys
+  const int32_t* page_table;
+  const int32_t* seqlens;
+  float* scores;            // optional [B][Hkv][max_blocks][max_blocks]
+  int32_t* idx;             // [B][Hkv][max_blocks][k_max]
+  int32_t* n_sel;           // [B][Hkv][max_blocks]
+  uint16_t* out;            // [B][Lq][Hq][D]
+  float* lse;               // optional [B][Hq][Lq]
+  int32_t* status;
+  int B, Hq, Hkv, G, bs, max_blocks, k_max;
+  int sparsity_permille, budget_tokens;  // k_i from a budget when budget_tokens > 0
+  int token_inner;
+  int64_t num_pages;
+  float gate_scale, scale_log2;
+};
+
+cudaError_t run_prefill_gate_select(const PrefillParams& p, cudaStream_t stream);
+cudaError_t run_prefill_attention(const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const PrefillParams& p, cudaStream_t stream);
+
 // The single-launch step: the decode kernel with the gate rows before it and
 // the combine after it, in one cooperative grid.  Control words (zero before
 // the first launch; every completed launch leaves them ready for the next):

@@ -109,3 +109,51 @@ class StepBuffers:
     def step(self, update_kbar: int = 0, stream=None, args=None, fused: bool = False):
         call = seer.seer_decode_step_fused if fused else seer.seer_decode_step
         call(self.dims, args if args is not None else self.args(update_kbar), stream)
+
+
+class PrefillBuffers:
+    """Device buffers for the prefill path over a drawn workload: prompt
+    queries (seeded), pooled keys, workspace, output, lse, gate scores."""
+
+    def __init__(self, w, data: dict, q, sparsity_permille: Optional[int] = None,
+                 budget_tokens: Optional[int] = None, keep_scores: bool = False):
+        from .workloads import pool_strides
+        self.w, self.data, self.q = w, data, q
+        dev = q.device
+        B, Hkv, D = w.batch, w.kv_heads, w.head_dim
+        self.nb_max = data["nb_max"]
+        sp, st, sh = pool_strides(data)
+        self.dims = seer.make_dims(B, w.q_heads, Hkv, D, w.block_size, self.nb_max,
+                                   data["num_pages"], sp, st, sh)
+        self.budget = (w.budget_tokens if budget_tokens is None else budget_tokens) or 0
+        self.permille = (w.sparsity_permille if sparsity_permille is None else sparsity_permille) or 0
+        self.k_max = max(1, seer.seer_prefill_k_max(self.dims, self.permille, self.budget))
+        self.kbar = torch.empty((B, Hkv, self.nb_max, D), dtype=torch.float32, device=dev)
+        ws = seer.seer_prefill_workspace_bytes(self.dims, self.k_max)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+        Lq = self.nb_max * w.block_size
+        self.out = torch.zeros((B, Lq, w.q_heads, D), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, w.q_heads, Lq), dtype=torch.float32, device=dev)
+        self.scores = (torch.empty((B, Hkv, self.nb_max, self.nb_max), dtype=torch.float32,
+                                   device=dev) if keep_scores else None)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.scale = 1.0 / math.sqrt(D)
+        self.page_table = data["page_table"] if w.paged else None
+
+    def selection(self):
+        rows = self.w.batch * self.w.kv_heads * self.nb_max
+        idx = self.workspace[:rows * self.k_max * 4].view(torch.int32).view(
+            self.w.batch, self.w.kv_heads, self.nb_max, self.k_max)
+        off = (rows * self.k_max * 4 + 255) // 256 * 256
+        n_sel = self.workspace[off:off + rows * 4].view(torch.int32).view(
+            self.w.batch, self.w.kv_heads, self.nb_max)
+        return idx, n_sel
+
+    def run(self, pool_keys: bool = True, stream=None):
+        d = self.data
+        seer.seer_prefill(self.dims, self.q, d["k_pool"], d["v_pool"], self.page_table,
+                          d["seqlens"], d["w_gate"], self.kbar, pool_keys=pool_keys,
+                          sparsity_permille=self.permille, budget_tokens=self.budget,
+                          k_max=self.k_max, gate_scale=self.scale, softmax_scale=self.scale,
+                          workspace=self.workspace, out=self.out, lse_out=self.lse,
+                          scores_out=self.scores, dev_status=self.status, stream=stream)

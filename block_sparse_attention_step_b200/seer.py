@@ -36,6 +36,7 @@ EXPORTS = (
     "seer_sparse_decode",
     "seer_combine", "seer_decode_step", "seer_decode_step_host", "seer_decode_step_noalloc",
     "seer_decode_step_fused", "seer_step_workspace_init",
+    "seer_prefill_k_max", "seer_prefill_workspace_bytes", "seer_prefill",
     "seer_block_lse_elems", "seer_sparse_decode_mass", "seer_block_mass",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -73,6 +74,18 @@ class seer_step_args(ctypes.Structure):
                 ("v_new", ctypes.c_void_p)]
 
 
+class seer_prefill_args(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+                ("page_table", ctypes.c_void_p), ("seqlens", ctypes.c_void_p),
+                ("w_gate", ctypes.c_void_p), ("kbar", ctypes.c_void_p),
+                ("pool_keys", ctypes.c_int32), ("sparsity_permille", ctypes.c_int32),
+                ("budget_tokens", ctypes.c_int32), ("k_max", ctypes.c_int32),
+                ("gate_scale", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("out", ctypes.c_void_p), ("lse_out", ctypes.c_void_p),
+                ("scores_out", ctypes.c_void_p), ("dev_status", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _D = ctypes.POINTER(seer_dims)
 _I = ctypes.c_int32
@@ -98,6 +111,9 @@ _SIGS = {
     "seer_decode_step_noalloc": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_decode_step_fused": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_step_workspace_init": (_I, [_D, _I, _I, _P, ctypes.c_size_t, _P]),
+    "seer_prefill_k_max": (_I, [_D, _I, _I]),
+    "seer_prefill_workspace_bytes": (ctypes.c_size_t, [_D, _I]),
+    "seer_prefill": (_I, [_D, ctypes.POINTER(seer_prefill_args), _P]),
     "seer_block_lse_elems": (ctypes.c_size_t, [_D]),
     "seer_sparse_decode_mass": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P,
                                      _P, _P, _P, _P]),
@@ -339,3 +355,38 @@ def seer_block_mass(d, idx, n_sel, k_max, seqlens, block_lse, lse, mass, stream=
         int(k_max), _ptr(seqlens, torch.int32, "seqlens"),
         _ptr(block_lse, torch.float32, "block_lse"), _ptr(lse, torch.float32, "lse"),
         _ptr(mass, torch.float32, "mass"), _stream(stream)))
+
+
+def seer_prefill_k_max(d, sparsity_permille, budget_tokens):
+    return _lib().seer_prefill_k_max(ctypes.byref(d), int(sparsity_permille), int(budget_tokens))
+
+
+def seer_prefill_workspace_bytes(d, k_max):
+    return _lib().seer_prefill_workspace_bytes(ctypes.byref(d), int(k_max))
+
+
+def seer_prefill(d, q, k_pool, v_pool, page_table, seqlens, w_gate, kbar, *, pool_keys,
+                 sparsity_permille, budget_tokens, k_max, gate_scale, softmax_scale, workspace,
+                 out, lse_out=None, scores_out=None, dev_status=None, stream=None):
+    a = seer_prefill_args()
+    a.q = _ptr(q, torch.bfloat16, "q")
+    a.k_pool = _ptr(k_pool, torch.bfloat16, "k_pool")
+    a.v_pool = _ptr(v_pool, torch.bfloat16, "v_pool")
+    a.page_table = _ptr(page_table, torch.int32, "page_table", allow_none=True)
+    a.seqlens = _ptr(seqlens, torch.int32, "seqlens")
+    a.w_gate = _ptr(w_gate, torch.float32, "w_gate")
+    a.kbar = _ptr(kbar, torch.float32, "kbar")
+    a.pool_keys = int(bool(pool_keys))
+    a.sparsity_permille = int(sparsity_permille)
+    a.budget_tokens = int(budget_tokens)
+    a.k_max = int(k_max)
+    a.gate_scale = float(gate_scale)
+    a.softmax_scale = float(softmax_scale)
+    a.workspace = _ptr(workspace, torch.uint8, "workspace")
+    a.workspace_bytes = workspace.numel()
+    a.out = _ptr(out, torch.bfloat16, "out")
+    a.lse_out = _ptr(lse_out, torch.float32, "lse_out", allow_none=True)
+    a.scores_out = _ptr(scores_out, torch.float32, "scores_out", allow_none=True)
+    a.dev_status = _ptr(dev_status, torch.int32, "dev_status", allow_none=True)
+    _check("seer_prefill", _lib().seer_prefill(ctypes.byref(d), ctypes.byref(a), _stream(stream)))
+

@@ -199,3 +199,13 @@ def gather_rows(pool: torch.Tensor, page_table: torch.Tensor, b: int, h: int,
     else:                                 # [P][Hkv][bs][D]
         rows = picked[:, h, :, :]
     return rows.reshape(nb * block_size, -1)[:seqlen].cpu()
+
+
+def prefill_queries(w: Workload, seed: int, max_blocks: int, device="cpu") -> torch.Tensor:
+    """Prompt queries for the prefill path: [B][max_blocks * bs][Hq][D] bf16,
+    N(0, 1) rounded to nearest, drawn from their own seeded generator (the
+    decode draw of the same seed is left unchanged)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 7919 + 17)
+    shape = (w.batch, max_blocks * w.block_size, w.q_heads, w.head_dim)
+    return torch.randn(shape, generator=g, device=device).to(torch.bfloat16)

@@ -354,6 +354,51 @@ SEER_API seer_status seer_decode_step_noalloc(const seer_dims *d,
                                               const seer_step_args *a,
                                               seer_stream stream);
 
+/* ------------------------------------------------ prefill with query pooling
+ * The SeerAttention form that SeerAttention-R drops to decode token by token
+ * (paper summary page, Abstract), for a whole prompt: query block i (the
+ * query tokens [i*bs, (i+1)*bs)) is gated with its pooled query -- the mean
+ * over its tokens and the group's G heads -- against the pooled keys of the
+ * blocks j <= i (gate_scale * (W qbar_i) . kbar_j); block i is always chosen
+ * and counts toward k_i (k_i from the sparsity over i + 1 candidates, or
+ * min(i + 1, budget / bs)); every query token then attends causally over the
+ * tokens of its block's chosen blocks up to itself.  q and out are
+ * [B][max_blocks * block_size][Hq][D] bf16 (16-byte aligned); K/V come from
+ * the paged pools; lse_out is [B][Hq][max_blocks * block_size] fp32 or NULL;
+ * scores_out, if not NULL, receives the block gate scores
+ * [B][Hkv][max_blocks][max_blocks] (-inf above the diagonal).  The workspace
+ * (seer_prefill_workspace_bytes) receives the chosen indices
+ * [B][Hkv][max_blocks][k_max] (ascending, -1 padded) and their counts
+ * [B][Hkv][max_blocks] int32.  pool_keys != 0 rebuilds kbar first. */
+typedef struct seer_prefill_args {
+  const uint16_t *q;
+  const uint16_t *k_pool;
+  const uint16_t *v_pool;
+  const int32_t *page_table; /* may be NULL (identity) */
+  const int32_t *seqlens;
+  const float *w_gate;
+  float *kbar;
+  int32_t pool_keys;
+  int32_t sparsity_permille;
+  int32_t budget_tokens;     /* > 0: budget rule */
+  int32_t k_max;             /* >= every k_i: seer_prefill_k_max */
+  float gate_scale;
+  float softmax_scale;
+  void *workspace;
+  size_t workspace_bytes;
+  uint16_t *out;
+  float *lse_out;
+  float *scores_out;
+  int32_t *dev_status;
+} seer_prefill_args;
+
+/* k of the last query block, which bounds every k_i (0 on bad dims). */
+SEER_API int32_t seer_prefill_k_max(const seer_dims *d, int32_t sparsity_permille,
+                                    int32_t budget_tokens);
+SEER_API size_t seer_prefill_workspace_bytes(const seer_dims *d, int32_t k_max);
+SEER_API seer_status seer_prefill(const seer_dims *d, const seer_prefill_args *a,
+                                  seer_stream stream);
+
 /* ------------------------------------------------------ single-launch step
  * The whole step in one cooperative launch (the persistent decode grid runs
  * the gate rows first and the LSE combine last; next to the per-stage path,

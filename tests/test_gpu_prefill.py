@@ -1,0 +1,134 @@
+"""Prefill with query pooling against the fp64 oracle: pooled keys, the
+block-to-block gate scores of the pooled queries, the diagonal-forced
+selection of every query block (bit-exact where the fp64 margin is clear,
+valid otherwise) and the causal block-sparse attention of every query token
+over the GPU's own selection; paged and contiguous caches, bs 64 and 128,
+ragged lengths, sparsity and budget rules, and the dense case (every block
+chosen) as plain causal attention."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_step_b200 import workloads as W
+from block_sparse_attention_step_b200.runner import PrefillBuffers
+from oracle import seer_oracle as O
+
+from gpu_util import MARGIN, assert_out_close, f64, require_gpu, scale_of
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+CASES = {
+    "paged_bs64_s80": (W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(
+        batch=2, q_heads=8, kv_heads=2, seqlen_range=(300, 1100)), 800, 0),
+    "contig_bs64_dense": (W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(
+        batch=2, q_heads=8, kv_heads=2, seqlen=450), 0, 0),
+    "contig_bs128_budget": (W.WORKLOADS["b16_h40_L32k_bs128_budget4k_newest"].replace(
+        batch=1, q_heads=10, kv_heads=2, seqlen=1500, budget_tokens=512), 0, 512),
+    "paged_bs64_s95_g8": (W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(
+        batch=1, q_heads=16, kv_heads=2, seqlen_range=(2000, 2600)), 950, 0),
+}
+
+
+def _k_of(permille, budget, bs):
+    if budget > 0:
+        return lambda i: O.k_from_budget(i + 1, budget, bs)
+    return lambda i: O.k_from_sparsity(i + 1, permille)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_matches_oracle(name):
+    w, permille, budget = CASES[name]
+    data = W.generate(w, 61, DEV)
+    q = W.prefill_queries(w, 61, data["nb_max"], DEV)
+    run = PrefillBuffers(w, data, q, sparsity_permille=permille, budget_tokens=budget,
+                         keep_scores=True)
+    run.run(pool_keys=True)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    idx, n_sel = (t.cpu().numpy() for t in run.selection())
+    kbar, scores = f64(run.kbar), f64(run.scores)
+    out, lse = f64(run.out), f64(run.lse)
+    G, bs = w.group, w.block_size
+    k_of = _k_of(permille, budget, bs)
+    exact = near = 0
+    for b in range(w.batch):
+        L = int(data["seqlens"][b])
+        nb = O.num_blocks(L, bs)
+        for h in range(w.kv_heads):
+            Qg = f64(q[b, :L, h * G:(h + 1) * G])
+            K = f64(W.gather_rows(data["k_pool"], data["page_table"], b, h, L, bs))
+            V = f64(W.gather_rows(data["v_pool"], data["page_table"], b, h, L, bs))
+            ref_kbar = O.pool_keys(K, L, bs)
+            np.testing.assert_allclose(kbar[b, h, :nb], ref_kbar, rtol=1e-5, atol=2e-6)
+            ref_sc = O.prefill_gate_scores(Qg, f64(data["w_gate"][h]), ref_kbar, L, bs, scale_of(w))
+            got_sel = []
+            for i in range(nb):
+                row = ref_sc[i, : i + 1]
+                bound = 1e-5 * max(1e-3, float(np.abs(row).max()))
+                assert np.abs(scores[b, h, i, : i + 1] - row).max() <= bound + 2e-6, (b, h, i)
+                assert np.isneginf(scores[b, h, i, i + 1:]).all()
+                k = k_of(i)
+                got = idx[b, h, i, : n_sel[b, h, i]]
+                assert (idx[b, h, i, n_sel[b, h, i]:] == -1).all()
+                if O.selection_margin(row, k, True) > MARGIN:
+                    assert got.tolist() == O.select_blocks(row, k, True).tolist(), (b, h, i)
+                    exact += 1
+                else:
+                    assert O.selection_is_valid(row, got, k, True, MARGIN), (b, h, i)
+                    near += 1
+                got_sel.append(got)
+            ref_out, ref_lse = O.prefill_attention(Qg, K, V, L, got_sel, bs, scale_of(w))
+            for g in range(G):
+                assert_out_close(out[b, :L, h * G + g], ref_out[:, g], (b, h, g))
+                np.testing.assert_allclose(lse[b, h * G + g, :L], ref_lse[:, g], atol=1e-3)
+    assert exact > 0
+
+
+def test_prefill_dense_is_causal_attention():
+    """Sparsity 0: every block is chosen, so each output row is plain causal
+    attention (checked against torch's fp64 SDPA, not the oracle)."""
+    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=1, q_heads=4, kv_heads=1,
+                                                           seqlen=333)
+    data = W.generate(w, 63, DEV)
+    q = W.prefill_queries(w, 63, data["nb_max"], DEV)
+    run = PrefillBuffers(w, data, q, sparsity_permille=0, budget_tokens=0)
+    run.run(pool_keys=True)
+    torch.cuda.synchronize()
+    L = 333
+    Q = q[0, :L].double().permute(1, 0, 2)[None]                  # [1][4][L][D]
+    K = W.gather_rows(data["k_pool"], data["page_table"], 0, 0, L, 64).double()
+    V = W.gather_rows(data["v_pool"], data["page_table"], 0, 0, L, 64).double()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.cpu(), K.cpu()[None, None].expand(1, 4, L, 128), V.cpu()[None, None].expand(1, 4, L, 128),
+        is_causal=True, scale=scale_of(w))[0].permute(1, 0, 2).numpy()
+    assert_out_close(f64(run.out[0, :L]), ref, "dense")
+
+
+def test_prefill_tail_garbage_never_matters():
+    """NaN in the cache slots past each sequence's end changes nothing."""
+    w, permille, budget = CASES["paged_bs64_s80"]
+    data = W.generate(w, 65, DEV)
+    q = W.prefill_queries(w, 65, data["nb_max"], DEV)
+    a = PrefillBuffers(w, data, q, sparsity_permille=permille)
+    a.run()
+    torch.cuda.synchronize()
+    out_a = a.out.clone()
+    table = data["page_table"]
+    for b in range(w.batch):
+        L = int(data["seqlens"][b])
+        if L % w.block_size:
+            page = int(table[b, L // w.block_size])
+            data["k_pool"][page, L % w.block_size:] = float("nan")
+            data["v_pool"][page, L % w.block_size:] = float("nan")
+    b_run = PrefillBuffers(w, data, q, sparsity_permille=permille)
+    b_run.kbar.copy_(a.kbar)
+    b_run.run(pool_keys=False)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a, b_run.out)
