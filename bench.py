@@ -36,6 +36,7 @@ UNIT = "tokens/s"
 KERNELS_PER_STEP = 3   # gate+select (with the incremental pooled-key update), decode, combine
 NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal, for the second roofline denominator
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0  # dense bf16 burst measured earlier on this machine's B200s
 
 
 def measured_peaks():
@@ -43,7 +44,7 @@ def measured_peaks():
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             return json.load(f), "measured"
     except (OSError, ValueError):
-        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS}, "fallback"
 
 
 def decode_source_hash():
@@ -400,6 +401,98 @@ def run_ours(args):
     return 0
 
 
+def prefill_flops(run, w):
+    """Algorithmic FLOPs of the prefill attention: 4 D per (query token, head,
+    attended key), the attended keys being the valid tokens of the query
+    block's chosen blocks up to the query itself (counted from the selection
+    the input actually produces)."""
+    import torch
+    idx, n_sel = run.selection()
+    bs, G = w.block_size, w.group
+    L = run.data["seqlens"].long()
+    total = 0
+    for b in range(w.batch):
+        Lb = int(L[b])
+        nb = -(-Lb // bs)
+        sel = idx[b, :, :nb].long()                       # [Hkv][nb][k_max]
+        live = torch.arange(sel.shape[-1], device=sel.device)[None, None] < n_sel[b, :, :nb, None]
+        qi = torch.arange(nb, device=sel.device)[None, :, None]
+        # full earlier blocks: every query token of block i sees all their valid keys
+        start = sel.clamp(min=0) * bs
+        valid = (Lb - start).clamp(min=0, max=bs)
+        q_in = (Lb - qi * bs).clamp(min=0, max=bs)          # query tokens in block i
+        earlier = (live & (sel < qi)) * valid * q_in
+        # the diagonal block: token u of the block sees u + 1 keys
+        diag = (live & (sel == qi)) * (q_in * (q_in + 1) // 2)
+        total += int((earlier + diag).sum().item())
+    return 4 * w.head_dim * G * total
+
+
+def run_prefill(args):
+    """Prefill with query pooling on the headline shapes at batch 2 and a
+    16K-token prompt: one JSON line (prompt tokens/s, tensor roofline)."""
+    import torch
+    from block_sparse_attention_step_b200 import workloads as W
+    from block_sparse_attention_step_b200.runner import PrefillBuffers
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = W.WORKLOADS[W.HEADLINE].replace(batch=2, seqlen=16384)
+    if args.sparsity is not None:
+        w = w.replace(sparsity_permille=args.sparsity)
+    runs = []
+    for r in range(2):
+        data = W.generate(w, args.seed + r, dev)
+        q = W.prefill_queries(w, args.seed + r, data["nb_max"], dev)
+        pr = PrefillBuffers(w, data, q)
+        pr.run(pool_keys=True)
+        runs.append(pr)
+    torch.cuda.synchronize()
+    flops = prefill_flops(runs[0], w)
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(0)
+
+    def timed(pool):
+        for i in range(args.warmup):
+            runs[i % 2].run(pool_keys=pool)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(args.steps):
+            runs[i % 2].run(pool_keys=pool)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    ms_full = timed(True)
+    ms_attn_gate = timed(False)
+    clock_info = clocks.stop()
+    peaks, kind = measured_peaks()
+    tflops = flops / (ms_attn_gate * 1e-3) / 1e12
+    line = {
+        "metric": "prefill prompt tokens/s (query-pooled block gate + causal block-sparse attention)",
+        "value": w.batch * w.seqlen / (ms_full * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_full,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"prefill_b{w.batch}_h{w.q_heads}_L{w.seqlen}_bs{w.block_size}_"
+                               f"s{w.sparsity_permille // 10}", "batch": w.batch,
+                   "seq_len": w.seqlen, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+                   "block_size": w.block_size, "sparsity_permille": w.sparsity_permille,
+                   "step": "seer_prefill with the full key pooling"},
+        "stage_ms": {"prefill_with_pooling": ms_full, "gate_select_attention": ms_attn_gate},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "prefill gate+select and attention (algorithmic attention FLOPs "
+                               "over both launches)", "flops_per_step": flops,
+                     "peak_source": f"{kind} bf16_tflops (burst)"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clock_info,
+        "device_status": [int(r.status.item()) for r in runs],
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def max_over_ranks(ms: float, device) -> float:
     """The slowest rank's time: every rank contributes its own elapsed time
     and all receive the maximum (the job is as fast as its slowest replica)."""
@@ -613,11 +706,15 @@ def main(argv=None):
                    help="one block set per sequence shared by all KV heads (cross-head ranking)")
     p.add_argument("--fused", action="store_true",
                    help="the whole step as one cooperative launch (seer_decode_step_fused)")
+    p.add_argument("--prefill", action="store_true",
+                   help="measure the prefill path with query pooling instead of the decode step")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.prefill:
+        return run_prefill(args)
     return run_ours(args)
 
 

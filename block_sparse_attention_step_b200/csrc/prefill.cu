@@ -230,19 +230,27 @@ __global__ void __launch_bounds__(kPAThreads, 2)
         ++issued;
       }
     }
+    bool marked = false;
     if (ok) {  // end marker: a stage with no data
       const int slot = issued % kPAStages;
       if (mbar_wait(&empty[slot], ((issued / kPAStages) & 1) ^ 1)) {
         meta[slot] = make_int2(0, -1);
         mbar_arrive(&full[slot]);
+        marked = true;
       } else {
         flag_status(p.status, SEER_DEV_TIMEOUT);
       }
     }
-    // let every copy this CTA started land before it retires
-    for (uint32_t k = 0; k < kPAStages && k < issued; ++k) {
+    // Let every copy this CTA started land before it retires.  With the end
+    // marker posted, the stage that last used the marker's slot was released
+    // by every math warp (so its copy landed), and its full barrier has moved
+    // on by the marker's phase: a parity wait on it could not tell the two
+    // apart, so it is left out.
+    const uint32_t in_flight = marked ? kPAStages - 1 : kPAStages;
+    for (uint32_t k = 0; k < in_flight && k < issued; ++k) {
       const uint32_t s = issued - 1 - k;
-      mbar_wait(&full[s % kPAStages], (s / kPAStages) & 1);
+      if (!mbar_wait(&full[s % kPAStages], (s / kPAStages) & 1))
+        flag_status(p.status, SEER_DEV_TIMEOUT);
     }
     return;
   }

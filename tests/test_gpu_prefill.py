@@ -101,6 +101,7 @@ def test_prefill_dense_is_causal_attention():
     run = PrefillBuffers(w, data, q, sparsity_permille=0, budget_tokens=0)
     run.run(pool_keys=True)
     torch.cuda.synchronize()
+    assert run.status.item() == 0   # also: no wait ran out (every tile streams several stages)
     L = 333
     Q = q[0, :L].double().permute(1, 0, 2)[None]                  # [1][4][L][D]
     K = W.gather_rows(data["k_pool"], data["page_table"], 0, 0, L, 64).double()
@@ -131,4 +132,5 @@ def test_prefill_tail_garbage_never_matters():
     b_run.kbar.copy_(a.kbar)
     b_run.run(pool_keys=False)
     torch.cuda.synchronize()
+    assert a.status.item() == 0 and b_run.status.item() == 0
     assert torch.equal(out_a, b_run.out)
