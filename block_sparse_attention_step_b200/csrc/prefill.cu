@@ -26,7 +26,7 @@ constexpr int kPGWarps = kPGThreads / 32;  // 8: 16 W rows and 8 kbar rows per w
 
 struct PrefillGateSmem {
   float scores[kMaxBlocks];
-  float qpart[2][kHeadDim];
+  float qpart[kPGWarps][kHeadDim];
   float qbar[kHeadDim];
   float gvec[kHeadDim];
   SelectSmem sel;
@@ -43,7 +43,7 @@ __device__ __forceinline__ int prefill_k(const PrefillParams& p, int n_cand) {
   return (int)(k < 1 ? 1 : k);
 }
 
-__global__ void __launch_bounds__(kPGThreads) prefill_gate_select_kernel(const PrefillParams p) {
+__global__ void __launch_bounds__(kPGThreads, 3) prefill_gate_select_kernel(const PrefillParams p) {
   __shared__ __align__(16) PrefillGateSmem sm;
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -60,18 +60,25 @@ __global__ void __launch_bounds__(kPGThreads) prefill_gate_select_kernel(const P
     if (tid == 0) p.n_sel[row] = 0;
     return;
   }
-  // pooled query: thread (half, d) adds tokens lo + half, lo + half + 2, ...
-  // over the group's heads, the two halves are added last
+  // pooled query: the block's (token, head) rows of the group, row r to warp
+  // r % 8 (a row is 256 contiguous bytes; lane l takes dims 4l .. 4l+3), eight
+  // rows in flight per warp; the eight warp partials are added in warp order
   const int lo = i * p.bs, hi = min(lo + p.bs, L);
   {
-    const int d = tid & (kHeadDim - 1), half = tid >> 7;
-    float s = 0.f;
-    for (int t = lo + half; t < hi; t += 2) {
-      const uint16_t* qt = p.q + (((int64_t)b * p.max_blocks * p.bs + t) * p.Hq + (int64_t)h * p.G) *
-                                     kHeadDim + d;
-      for (int g = 0; g < p.G; ++g) s += __uint_as_float((uint32_t)__ldg(qt + g * kHeadDim) << 16);
+    const int nrows = (hi - lo) * p.G;
+    const uint16_t* q0 = p.q + (((int64_t)b * p.max_blocks * p.bs + lo) * p.Hq + (int64_t)h * p.G) *
+                                   kHeadDim + 4 * lane;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+    for (int rr = warp; rr < nrows; rr += kPGWarps) {
+      const int t = rr / p.G, g = rr - t * p.G;
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(q0 + ((int64_t)t * p.Hq + g) * kHeadDim));
+      a0 += __uint_as_float(v.x << 16);
+      a1 += __uint_as_float(v.x & 0xffff0000u);
+      a2 += __uint_as_float(v.y << 16);
+      a3 += __uint_as_float(v.y & 0xffff0000u);
     }
-    sm.qpart[half][d] = s;
+    *reinterpret_cast<float4*>(&sm.qpart[warp][4 * lane]) = make_float4(a0, a1, a2, a3);
   }
   // this warp's W rows warp + 8 r (16 of them), in flight meanwhile
   float4 wrow[kHeadDim / kPGWarps];
@@ -82,8 +89,12 @@ __global__ void __launch_bounds__(kPGThreads) prefill_gate_select_kernel(const P
       wrow[r] = __ldg(reinterpret_cast<const float4*>(W + (warp + r * kPGWarps) * kHeadDim + 4 * lane));
   }
   __syncthreads();
-  if (tid < kHeadDim)
-    sm.qbar[tid] = (sm.qpart[0][tid] + sm.qpart[1][tid]) / (float)((hi - lo) * p.G);
+  if (tid < kHeadDim) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kPGWarps; ++w) s += sm.qpart[w][tid];
+    sm.qbar[tid] = s / (float)((hi - lo) * p.G);
+  }
   __syncthreads();
   {
     const float4 qv = *reinterpret_cast<const float4*>(&sm.qbar[4 * lane]);
