@@ -11,8 +11,8 @@
 //     TMA (the decode's tensor maps, 64 tokens x 64 dims per box), and four
 //     math warps (16 query tokens each) run S = Q K^T, the causal and tail
 //     masks, the online softmax and O += P V on the tensor cores
-//     (mma.sync m16n8k16 bf16, P as a bf16 hi + lo pair), writing bf16 out
-//     and the natural-log lse.
+//     (mma.sync m16n8k16 bf16, P rounded to bf16 as in FlashAttention),
+//     writing bf16 out and the natural-log lse.
 // Every wait is bounded (SEER_DEV_TIMEOUT); nothing traps.
 #include "block_mean.cuh"
 #include "seer_kernels.cuh"
@@ -359,14 +359,14 @@ __global__ void __launch_bounds__(kPAThreads, 2)
       o[dt][2] *= alpha_b;
       o[dt][3] *= alpha_b;
     }
-    // ---- O += P V: P (from the S accumulators) as a bf16 hi + lo pair, V by ldmatrix.trans
+    // ---- O += P V: P (from the S accumulators) rounded to bf16, V by ldmatrix.trans
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-      uint32_t ph[4], pl[4];
-      split_bf16x2(s[2 * kk][0], s[2 * kk][1], ph[0], pl[0]);
-      split_bf16x2(s[2 * kk][2], s[2 * kk][3], ph[1], pl[1]);
-      split_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1], ph[2], pl[2]);
-      split_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3], ph[3], pl[3]);
+      uint32_t ph[4];
+      ph[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
+      ph[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
+      ph[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      ph[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
       // tail keys (past the sequence) may hold anything: zero their V
       const int k0 = 16 * kk + 2 * c;
       const uint32_t m0 = (k0 < valid ? 0x0000ffffu : 0u) | (k0 + 1 < valid ? 0xffff0000u : 0u);
@@ -385,9 +385,7 @@ __global__ void __launch_bounds__(kPAThreads, 2)
         v2 &= m0;
         v3 &= m1;
         mma_bf16_16816(o[2 * dp], ph, v0, v1);
-        mma_bf16_16816(o[2 * dp], pl, v0, v1);
         mma_bf16_16816(o[2 * dp + 1], ph, v2, v3);
-        mma_bf16_16816(o[2 * dp + 1], pl, v2, v3);
       }
     }
     fence_proxy_async_smem();
