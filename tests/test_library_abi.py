@@ -114,3 +114,28 @@ def test_workspace_and_default_splits(lib):
     d1 = seer.make_dims(1, 4, 1, 128, 64, 64, 64)
     assert seer.seer_default_splits(d1, 8, 148) == 4     # capped at k_max / 2
     assert seer.seer_default_splits(d1, 1, 148) == 1
+
+
+def test_prefill_and_fused_host_checks(lib):
+    d = seer.make_dims(2, 8, 2, 128, 64, 256, 2 * 256)
+    # k of the last query block bounds every k_i: 10 % of 256 blocks, or 4096 / 64
+    assert seer.seer_prefill_k_max(d, 900, 0) == O.k_from_sparsity(256, 900) == 26
+    assert seer.seer_prefill_k_max(d, 0, 4096) == O.k_from_budget(256, 4096, 64) == 64
+    rows = 2 * 2 * 256
+    r = lambda x: (x + 255) // 256 * 256
+    assert seer.seer_prefill_workspace_bytes(d, 26) == r(rows * 26 * 4) + r(rows * 4)
+    null = None
+    a = seer.seer_prefill_args()
+    assert lib.seer_prefill(ctypes.byref(d), ctypes.byref(a), null) == 1      # no inputs
+    fake = ctypes.c_void_p(4096)
+    b = seer.seer_step_args()
+    b.k_per_seq = b.kbar = fake
+    b.k_max, b.num_splits, b.unified_heads = 4, 1, 1
+    assert lib.seer_decode_step_fused(ctypes.byref(d), ctypes.byref(b), null) == 2   # unified
+    b.unified_heads, b.k_new = 0, fake                                             # k_new alone
+    assert lib.seer_decode_step_fused(ctypes.byref(d), ctypes.byref(b), null) == 1
+    assert lib.seer_step_workspace_init(ctypes.byref(d), 4, 1, null, 0, null) == 4
+    assert lib.seer_block_select_unified(ctypes.byref(d), null, null, null, 0, 4, null, null,
+                                         null, null) == 1
+    assert lib.seer_last_cuda_error().decode() == "no error"
+
