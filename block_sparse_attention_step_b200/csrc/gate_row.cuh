@@ -70,15 +70,16 @@ struct ChunkRing {
 
 // THREADS: the CTA (every thread calls this; it synchronises the CTA).
 // WORKERS: warps 0 .. WORKERS-1 form g and the scores (8 W rows and 8 kbar
-// rows per warp at a time).  CHUNK_ROWS = 8 * WORKERS kbar rows per buffer.
+// rows per warp at a time, R8 such groups of kbar rows per chunk).
+// CHUNK_ROWS = 8 * R8 * WORKERS kbar rows per buffer.
 // Threads QFIRST .. QFIRST + QTHREADS - 1 form the mean query.  Thread 0
 // issues the copies.  `seq` counts the chunks this CTA consumed before (slot
 // and parity of the ring), so a persistent CTA's rows share one ring.
 // Returns false when a wait ran out (SEER_DEV_TIMEOUT is flagged).
-template <int THREADS, int WORKERS, int NBUF, int QFIRST, int QTHREADS>
+template <int THREADS, int WORKERS, int NBUF, int QFIRST, int QTHREADS, int R8 = 1>
 __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRing<NBUF>& ring,
                          uint64_t* bars, uint32_t& seq, GateRowScratch& gs) {
-  constexpr int CHUNK_ROWS = 8 * WORKERS;
+  constexpr int CHUNK_ROWS = 8 * R8 * WORKERS;
   constexpr int kWRows = kHeadDim / WORKERS;  // W rows per worker warp
   static_assert(THREADS % 32 == 0 && THREADS / 32 >= kPoolWarps, "pooling uses 8 warps");
   static_assert(WORKERS * 32 <= THREADS && kWRows % 8 == 0, "8 W rows per reduction");
@@ -191,24 +192,27 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
     }
     const int rows = min(CHUNK_ROWS, nb - c * CHUNK_ROWS);
     const float* buf = ring.slot[slot];
-    if (warp < WORKERS) {  // this warp's 8 rows warp + WORKERS * i, one reduction
-      float4 v[8];
+    if (warp < WORKERS) {  // this warp's rows warp + WORKERS * i, 8 per reduction
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = warp + i * WORKERS;
-        const int j = c * CHUNK_ROWS + r;
-        v[i] = (r >= rows) ? make_float4(0.f, 0.f, 0.f, 0.f)
-               : (refresh && j == nb - 1)
-                   ? *reinterpret_cast<const float4*>(&gs.newest[4 * lane])
-                   : *reinterpret_cast<const float4*>(&buf[r * kHeadDim + 4 * lane]);
-      }
-      const float sc = warp_dot4_x8(v, gv);
-      const int r = warp + ((lane >> 2) & 7) * WORKERS;
-      if ((lane & 3) == 0 && r < rows) {
-        const int j = c * CHUNK_ROWS + r;
-        gs.scores[j] = sc;
-        scores_out[j] = sc;
-        bad |= !isfinite(sc);
+      for (int g8 = 0; g8 < R8; ++g8) {
+        float4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = warp + (g8 * 8 + i) * WORKERS;
+          const int j = c * CHUNK_ROWS + r;
+          v[i] = (r >= rows) ? make_float4(0.f, 0.f, 0.f, 0.f)
+                 : (refresh && j == nb - 1)
+                     ? *reinterpret_cast<const float4*>(&gs.newest[4 * lane])
+                     : *reinterpret_cast<const float4*>(&buf[r * kHeadDim + 4 * lane]);
+        }
+        const float sc = warp_dot4_x8(v, gv);
+        const int r = warp + (g8 * 8 + ((lane >> 2) & 7)) * WORKERS;
+        if ((lane & 3) == 0 && r < rows) {
+          const int j = c * CHUNK_ROWS + r;
+          gs.scores[j] = sc;
+          scores_out[j] = sc;
+          bad |= !isfinite(sc);
+        }
       }
     }
     fence_proxy_async_smem();

@@ -74,16 +74,18 @@ struct DecodeShape {
   static constexpr size_t kO = kML + kMSlots * kMLBytes;
   __host__ __device__ static size_t o_slot_floats(int G) { return (size_t)kMathWarps * G * kOStride; }
   static size_t smem_bytes(int G) { return 1024 + kO + kMSlots * o_slot_floats(G) * 4; }
-  // The single-launch step's gate rows stream kbar through the stage ring
-  // plus one or two more 32 KB slots (192 KB in flight when they fit), and
-  // keep their scratch and chunk mbarriers in the merge area -- all idle
-  // until the decode starts.
+  // The single-launch step's gate rows stream kbar in 64 KB chunks (two
+  // stage slots each) through the stage ring plus one more 64 KB slot when it
+  // fits (192 KB in flight), else 32 KB chunks through the ring and one more
+  // 32 KB slot; their scratch and chunk mbarriers sit in the merge area -- all
+  // idle until the decode starts.
   static constexpr size_t kGateBars = (kML + sizeof(GateRowScratch) + 7) & ~size_t(7);
   static constexpr size_t kGateExtra = (kGateBars + 8 * (kStages + 2) + 127) & ~size_t(127);
-  static constexpr int kGateSlots =
-      (1024 + kGateExtra + 2 * kStageBytes + 512 <= 227 * 1024) ? kStages + 2 : kStages + 1;
+  static constexpr bool kGateWide = 1024 + kGateExtra + 2 * kStageBytes + 512 <= 227 * 1024;
+  static constexpr int kGateR8 = kGateWide ? 2 : 1;                  // 8-row groups per warp
+  static constexpr int kGateSlots = kGateWide ? kStages / 2 + 1 : kStages + 1;
   static size_t smem_bytes_fused(int G) {
-    const size_t gate = 1024 + kGateExtra + (size_t)(kGateSlots - kStages) * kStageBytes;
+    const size_t gate = 1024 + kGateExtra + (size_t)(kGateWide ? 2 : 1) * kStageBytes;
     return smem_bytes(G) > gate ? smem_bytes(G) : gate;
   }
   static_assert(kRing % 1024 == 0 && kStageBytes % 1024 == 0, "swizzled TMA tiles need 1 KB");
@@ -203,13 +205,13 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     static_assert(kStageBytes == 8 * kMathWarps * kHeadDim * 4, "a stage holds one kbar chunk");
     GateRowScratch& gs = *reinterpret_cast<GateRowScratch*>(smem + Shape::kML);
     uint64_t* gbar = reinterpret_cast<uint64_t*>(smem + Shape::kGateBars);
+    constexpr int kR8 = Shape::kGateR8;
+    constexpr size_t kChunkBytes = (size_t)kR8 * kStageBytes;  // 8 * R8 * 8 warps rows
     ChunkRing<kSlots> gring;
 #pragma unroll
-    for (int i = 0; i < kStages; ++i) gring.slot[i] = reinterpret_cast<float*>(ring + i * kStageBytes);
-#pragma unroll
-    for (int i = kStages; i < kSlots; ++i)
-      gring.slot[i] = reinterpret_cast<float*>(smem + Shape::kGateExtra +
-                                               (size_t)(i - kStages) * kStageBytes);
+    for (int i = 0; i < kSlots - 1; ++i)
+      gring.slot[i] = reinterpret_cast<float*>(ring + i * kChunkBytes);
+    gring.slot[kSlots - 1] = reinterpret_cast<float*>(smem + Shape::kGateExtra);
     if (threadIdx.x == 0) {
       epoch_next = *reinterpret_cast<volatile uint32_t*>(f.ctl + 2) + 1u;
       for (int i = 0; i < kSlots; ++i) mbar_init(&gbar[i], 1);
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     uint32_t gseq = 0;
     const int rows = p.B * p.Hkv;
     for (int row = blockIdx.x; row < rows; row += gridDim.x) {
-      gate_row<Shape::kThreads, kMathWarps, kSlots, kMathThreads, 64>(
+      gate_row<Shape::kThreads, kMathWarps, kSlots, kMathThreads, 64, kR8>(
           f.gate, row / p.Hkv, row % p.Hkv, gring, gbar, gseq, gs);
       __syncthreads();  // the row's indices, kbar row and appended K/V are written
       if (threadIdx.x == 0) {
