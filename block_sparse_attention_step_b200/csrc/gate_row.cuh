@@ -75,10 +75,16 @@ struct ChunkRing {
 // Threads QFIRST .. QFIRST + QTHREADS - 1 form the mean query.  Thread 0
 // issues the copies.  `seq` counts the chunks this CTA consumed before (slot
 // and parity of the ring), so a persistent CTA's rows share one ring.
+// A CTA that gates several rows streams them as one chunk sequence: `ahead`
+// enters as the number of this row's chunks already issued by the previous
+// row, and leaves as the number of the next row's chunks issued here (next_b
+// < 0: no next row), so the next row's data is on its way while this row
+// finishes and selects.
 // Returns false when a wait ran out (SEER_DEV_TIMEOUT is flagged).
 template <int THREADS, int WORKERS, int NBUF, int QFIRST, int QTHREADS, int R8 = 1>
 __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRing<NBUF>& ring,
-                         uint64_t* bars, uint32_t& seq, GateRowScratch& gs) {
+                         uint64_t* bars, uint32_t& seq, GateRowScratch& gs, int next_b = -1,
+                         int next_h = 0, uint32_t* ahead = nullptr) {
   constexpr int CHUNK_ROWS = 8 * R8 * WORKERS;
   constexpr int kWRows = kHeadDim / WORKERS;  // W rows per worker warp
   static_assert(THREADS % 32 == 0 && THREADS / 32 >= kPoolWarps, "pooling uses 8 warps");
@@ -93,17 +99,33 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
   float* kb_row = p.kbar + bh * p.max_blocks * kHeadDim;
   const int k_row = __ldg(p.k_per_seq + b);
   bool ok = true;
-
-  // the first chunks of the row go out before anything else
-  if (tid == 0) {
-    for (int c = 0; c < NBUF && c < nchunks; ++c) {
-      const uint32_t slot = (seq + c) % NBUF;
-      const uint32_t bytes = (uint32_t)min(CHUNK_ROWS, nb - c * CHUNK_ROWS) * kHeadDim * 4;
-      mbar_arrive_expect_tx(&bars[slot], bytes);
-      bulk_copy_g2s(ring.slot[slot], kb_row + (int64_t)c * CHUNK_ROWS * kHeadDim, bytes,
-                    &bars[slot]);
-    }
+  // the chunk stream: this row's chunks, then the next row's
+  int next_nb = 0;
+  const float* next_kb = nullptr;
+  if (next_b >= 0) {
+    const int Ln = max(0, min(__ldg(p.seqlens + next_b), p.max_blocks * p.bs));
+    next_nb = ceil_div_i(Ln, p.bs);
+    next_kb = p.kbar + ((int64_t)next_b * p.Hkv + next_h) * p.max_blocks * kHeadDim;
   }
+  const int stream_len = nchunks + ceil_div_i(next_nb, CHUNK_ROWS);
+  const uint32_t first = ahead != nullptr ? *ahead : 0u;  // already issued
+  uint32_t issued = first;
+  auto issue = [&](int u) {  // position u of the stream into slot (seq + u) % NBUF
+    const uint32_t slot = (seq + u) % NBUF;
+    const bool own = u < nchunks;
+    const int c = own ? u : u - nchunks;
+    const int rows_c = min(CHUNK_ROWS, (own ? nb : next_nb) - c * CHUNK_ROWS);
+    const uint32_t bytes = (uint32_t)rows_c * kHeadDim * 4;
+    mbar_arrive_expect_tx(&bars[slot], bytes);
+    bulk_copy_g2s(ring.slot[slot], (own ? kb_row : next_kb) + (int64_t)c * CHUNK_ROWS * kHeadDim,
+                  bytes, &bars[slot]);
+  };
+
+  // the first chunks go out before anything else (free slots: this row's
+  // own chunks, then, if the row is short, the next row's)
+  if (tid == 0)
+    for (int u = (int)first; u < NBUF && u < stream_len; ++u) issue(u);
+  issued = (uint32_t)max((int)first, min(NBUF, stream_len));
 
   // KV append: the new token's K and V rows of head h at position L - 1
   const bool append = p.k_new != nullptr && L > 0;
@@ -217,15 +239,13 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
     }
     fence_proxy_async_smem();
     __syncthreads();  // every warp is done with this buffer
-    if (tid == 0 && ok && c + NBUF < nchunks) {
-      const int cn = c + NBUF;
-      const uint32_t bytes = (uint32_t)min(CHUNK_ROWS, nb - cn * CHUNK_ROWS) * kHeadDim * 4;
-      mbar_arrive_expect_tx(&bars[slot], bytes);
-      bulk_copy_g2s(ring.slot[slot], kb_row + (int64_t)cn * CHUNK_ROWS * kHeadDim, bytes,
-                    &bars[slot]);
+    if (c + NBUF < stream_len) {
+      if (tid == 0 && ok) issue(c + NBUF);
+      issued = max(issued, (uint32_t)(c + NBUF + 1));
     }
   }
   seq += (uint32_t)nchunks;
+  if (ahead != nullptr) *ahead = issued > (uint32_t)nchunks ? issued - (uint32_t)nchunks : 0u;
   if (bad) flag_status(p.status, SEER_DEV_NONFINITE_SCORE);
   for (int j = nb + tid; j < p.max_blocks; j += THREADS) scores_out[j] = -INFINITY;
   if (p.scores_only) return ok;  // uniform: the cross-head select runs next

@@ -54,6 +54,67 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
   gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(p, b, h, ring, sm.bar, seq, sm.row);
 }
 
+// The same rows for batches with more (b, h) rows than SMs: one persistent
+// CTA per SM gates row after row, claiming the next row (a counter zeroed
+// before the launch) while it starts the current one, and keeps one kbar
+// chunk stream across its rows -- the next row's first chunks are in flight
+// while this one finishes and selects, and no CTA start-up or drain sits
+// between rows.
+__global__ void __launch_bounds__(kGSThreads, 1)
+    gate_select_rows_kernel(const GateSelectParams p) {
+  extern __shared__ uint8_t gs_raw[];
+  GateSelectSmem& sm = *reinterpret_cast<GateSelectSmem*>(
+      (reinterpret_cast<uintptr_t>(gs_raw) + 127) & ~uintptr_t(127));
+  __shared__ int next_row;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGSBuffers; ++i) mbar_init(&sm.bar[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait();
+  pdl_launch_dependents();
+  if (p.work_counter != nullptr && blockIdx.x == 0 && threadIdx.x < 2)
+    p.work_counter[threadIdx.x] = 0u;
+  const int rows = p.B * p.Hkv;
+  const ChunkRing<kGSBuffers> ring = {{sm.buf[0], sm.buf[1], sm.buf[2]}};
+  uint32_t seq = 0, ahead = 0;
+  int row = blockIdx.x;
+  while (row < rows) {
+    if (threadIdx.x == 0) {
+      const unsigned v = atomicAdd(p.row_counter, 1u) + gridDim.x;
+      next_row = v < (unsigned)rows ? (int)v : -1;
+    }
+    __syncthreads();
+    const int nxt = next_row;
+    gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(
+        p, row / p.Hkv, row % p.Hkv, ring, sm.bar, seq, sm.row, nxt >= 0 ? nxt / p.Hkv : -1,
+        nxt >= 0 ? nxt % p.Hkv : 0, &ahead);
+    __syncthreads();  // next_row is rewritten for the following row
+    row = nxt >= 0 ? nxt : rows;
+  }
+}
+
+cudaError_t run_gate_select_rows(const GateSelectParams& p, int num_sms, cudaStream_t stream,
+                                 bool pdl) {
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = ensure_smem_limit(gate_select_rows_kernel, smem_set);
+  if (e != cudaSuccess) return e;
+  const int rows = p.B * p.Hkv;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows < num_sms ? rows : num_sms);
+  cfg.blockDim = dim3(kGSThreads);
+  cfg.dynamicSmemBytes = sizeof(GateSelectSmem) + 128;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gate_select_rows_kernel, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream, bool pdl) {
   static std::atomic<uint64_t> smem_set{0};
   cudaError_t e = ensure_smem_limit(gate_select_kernel, smem_set);

@@ -531,7 +531,16 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   g.gate_scale = a->gate_scale;
   g.work_counter = w.work_counter;  // zeroed by the gate grid for the decode grid
   g.scores_only = a->unified_heads ? 1 : 0;
-  SEER_CUDA(run_gate_select(g, d->batch, stream, true));
+  g.B = d->batch;
+  g.row_counter = w.work_counter + 5;
+  const int num_sms = num_sms_current();
+  if ((int64_t)d->batch * d->num_kv_heads > num_sms) {
+    // more rows than SMs: persistent row-claiming gate (its counter starts at 0)
+    SEER_CUDA(cudaMemsetAsync(g.row_counter, 0, sizeof(uint32_t), stream));
+    SEER_CUDA(run_gate_select_rows(g, num_sms, stream, true));
+  } else {
+    SEER_CUDA(run_gate_select(g, d->batch, stream, true));
+  }
   if (a->unified_heads) {  // one block set per sequence, shared by its KV heads
     SelectParams u;
     u.scores = w.scores;

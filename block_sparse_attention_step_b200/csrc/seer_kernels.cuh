@@ -58,6 +58,8 @@ struct GateSelectParams {
   float gate_scale;
   int scores_only;          // 1: stop after the scores (the unified select follows)
   uint32_t* work_counter;  // optional: zeroed for the decode grid that follows
+  int B;
+  uint32_t* row_counter;   // the row-claiming gate grid's counter (zero before it starts)
 };
 
 struct DecodeParams {
@@ -145,6 +147,8 @@ cudaError_t run_pool_keys(const PoolParams& p, int B, cudaStream_t stream);
 cudaError_t run_gate_scores(const GateParams& p, int B, cudaStream_t stream);
 cudaError_t run_block_select(const SelectParams& p, int B, cudaStream_t stream);
 cudaError_t run_gate_select(const GateSelectParams& p, int B, cudaStream_t stream, bool pdl);
+cudaError_t run_gate_select_rows(const GateSelectParams& p, int num_sms, cudaStream_t stream,
+                                 bool pdl);
 cudaError_t run_unified_select(const SelectParams& p, int B, cudaStream_t stream, bool pdl);
 cudaError_t run_fill_k(const int32_t* seqlens, int B, int bs, int permille, int budget,
                        int32_t* k_out, cudaStream_t stream);

@@ -218,11 +218,13 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       fence_mbar_init();
     }
     __syncthreads();
-    uint32_t gseq = 0;
+    uint32_t gseq = 0, gahead = 0;
     const int rows = p.B * p.Hkv;
     for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+      const int nxt = row + (int)gridDim.x;  // this CTA's next row: its kbar streams in early
       gate_row<Shape::kThreads, kMathWarps, kSlots, kMathThreads, 64, kR8>(
-          f.gate, row / p.Hkv, row % p.Hkv, gring, gbar, gseq, gs);
+          f.gate, row / p.Hkv, row % p.Hkv, gring, gbar, gseq, gs, nxt < rows ? nxt / p.Hkv : -1,
+          nxt < rows ? nxt % p.Hkv : 0, &gahead);
       __syncthreads();  // the row's indices, kbar row and appended K/V are written
       if (threadIdx.x == 0) {
         __threadfence();
