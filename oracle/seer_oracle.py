@@ -66,8 +66,10 @@ __all__ = [
     "select_blocks_unified",
     "pool_queries",
     "prefill_gate_scores",
+    "prefill_gate_row",
     "prefill_select",
     "prefill_attention",
+    "prefill_attention_token",
     "prefill_row",
 ]
 
@@ -408,15 +410,23 @@ def prefill_gate_scores(Q_group: np.ndarray, W: np.ndarray, kbar: np.ndarray, se
     nb = num_blocks(L, block_size)
     out = np.full((nb, nb), -np.inf, dtype=np.float64)
     for i in range(nb):
-        lo, hi = i * block_size, min((i + 1) * block_size, L)
-        acc = np.zeros(i + 1, dtype=np.float64)
-        count = 0
-        for t in range(lo, hi):
-            for g in range(Q_group.shape[1]):
-                acc += kbar[: i + 1] @ (W @ Q_group[t, g])
-                count += 1
-        out[i, : i + 1] = acc / count * float(scale)
+        out[i, : i + 1] = prefill_gate_row(Q_group, W, kbar, L, block_size, scale, i)
     return out
+
+
+def prefill_gate_row(Q_group: np.ndarray, W: np.ndarray, kbar: np.ndarray, seqlen: int,
+                     block_size: int, scale: float, i: int) -> np.ndarray:
+    """Row i of ``prefill_gate_scores`` on its causal prefix: [i + 1] scores
+    of query block i against key blocks 0..i (each query token and head of
+    block i scored on its own, the mean taken last)."""
+    lo, hi = i * block_size, min((i + 1) * block_size, int(seqlen))
+    acc = np.zeros(i + 1, dtype=np.float64)
+    count = 0
+    for t in range(lo, hi):
+        for g in range(Q_group.shape[1]):
+            acc += kbar[: i + 1] @ (W @ Q_group[t, g])
+            count += 1
+    return acc / count * float(scale)
 
 
 def prefill_select(scores: np.ndarray, k_of_block) -> list:
@@ -438,20 +448,27 @@ def prefill_attention(Q_group: np.ndarray, K: np.ndarray, V: np.ndarray, seqlen:
     out = np.zeros((L, G, D), dtype=np.float64)
     lse = np.full((L, G), -np.inf, dtype=np.float64)
     for i, blocks in enumerate(selected):
-        keep = np.zeros(L, dtype=bool)
-        for j in blocks:
-            keep[int(j) * block_size:min((int(j) + 1) * block_size, L)] = True
         for t in range(i * block_size, min((i + 1) * block_size, L)):
-            mask = keep.copy()
-            mask[t + 1:] = False
-            keys = np.nonzero(mask)[0]
-            x = (Q_group[t] @ K[keys].T) * float(scale)          # [G][n]
-            m = x.max(axis=1, keepdims=True)
-            e = np.exp(x - m)
-            tot = e.sum(axis=1, keepdims=True)
-            out[t] = (e / tot) @ V[keys]
-            lse[t] = (m + np.log(tot))[:, 0]
+            out[t], lse[t] = prefill_attention_token(Q_group, K, V, L, t, blocks, block_size,
+                                                     scale)
     return out, lse
+
+
+def prefill_attention_token(Q_group: np.ndarray, K: np.ndarray, V: np.ndarray, seqlen: int,
+                            t: int, blocks, block_size: int, scale: float):
+    """One query token t of ``prefill_attention``: its G heads attend the keys
+    s <= t of the given blocks.  Returns (out [G][D], lse [G])."""
+    L = int(seqlen)
+    keep = np.zeros(L, dtype=bool)
+    for j in blocks:
+        keep[int(j) * block_size:min((int(j) + 1) * block_size, L)] = True
+    keep[t + 1:] = False
+    keys = np.nonzero(keep)[0]
+    x = (Q_group[t] @ K[keys].T) * float(scale)          # [G][n]
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    tot = e.sum(axis=1, keepdims=True)
+    return (e / tot) @ V[keys], (m + np.log(tot))[:, 0]
 
 
 def prefill_row(Q_group, W, K, V, seqlen, block_size, k_of_block, gate_scale, softmax_scale):

@@ -158,3 +158,25 @@ def test_fused_step_edge_cases():
     torch.cuda.synchronize()
     assert run.status.item() == 0
     _assert_same(ref, _snapshot(run))
+
+
+@pytest.mark.parametrize("name", ["b16_h40_L32k_bs64_s90", "b16_h40_L32k_bs128_budget4k_newest"])
+def test_fused_step_full_size_equals_per_stage_step(name):
+    """At full size with the benchmark's seed and incremental pooled-key
+    update, the single launch gives the per-stage step's bits (the per-stage
+    step is checked against the oracle at full size on sampled rows)."""
+    w = W.WORKLOADS[name]
+    data = W.generate(w, 1, DEV)
+    run = StepBuffers(w, data)
+    run.pool_full()
+    kbar0 = run.kbar.clone()
+    run.step(update_kbar=1)
+    torch.cuda.synchronize()
+    ref = _snapshot(run)
+    run.kbar.copy_(kbar0)
+    run.out.zero_()
+    run.lse.zero_()
+    run.step(update_kbar=1, fused=True)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    _assert_same(ref, _snapshot(run))

@@ -134,3 +134,52 @@ def test_prefill_tail_garbage_never_matters():
     torch.cuda.synchronize()
     assert a.status.item() == 0 and b_run.status.item() == 0
     assert torch.equal(out_a, b_run.out)
+
+
+def test_prefill_full_size_sampled():
+    """The prefill at the size and seeds the benchmark times (batch 2, 16K-token
+    prompt, 40/8 heads, bs 64, 90 %): every pooled key, and for sampled query
+    blocks (first, second, middle, last and seeded picks) the gate row, the
+    selection and the output and lse of sampled query tokens against the
+    oracle computed one by one."""
+    w = W.WORKLOADS[W.HEADLINE].replace(batch=2, seqlen=16384)
+    seed = 1
+    data = W.generate(w, seed, DEV)
+    q = W.prefill_queries(w, seed, data["nb_max"], DEV)
+    run = PrefillBuffers(w, data, q, keep_scores=True)
+    run.run(pool_keys=True)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    idx, n_sel = (t.cpu().numpy() for t in run.selection())
+    kbar, scores = f64(run.kbar), f64(run.scores)
+    G, bs, scale = w.group, w.block_size, scale_of(w)
+    rng = np.random.default_rng(7)
+    exact = 0
+    for b in range(w.batch):
+        L = int(data["seqlens"][b])
+        nb = O.num_blocks(L, bs)
+        for h in range(w.kv_heads):
+            K = f64(W.gather_rows(data["k_pool"], data["page_table"], b, h, L, bs))
+            ref_kbar = O.pool_keys(K, L, bs)
+            np.testing.assert_allclose(kbar[b, h, :nb], ref_kbar, rtol=1e-5, atol=2e-6)
+            V = f64(W.gather_rows(data["v_pool"], data["page_table"], b, h, L, bs))
+            Qg = f64(q[b, :L, h * G:(h + 1) * G])
+            blocks = sorted({0, 1, nb // 2, nb - 1, *rng.integers(0, nb, 2).tolist()})
+            for i in blocks:
+                row = O.prefill_gate_row(Qg, f64(data["w_gate"][h]), ref_kbar, L, bs, scale, i)
+                bound = 1e-5 * max(1e-3, float(np.abs(row).max()))
+                assert np.abs(scores[b, h, i, : i + 1] - row).max() <= bound + 2e-6, (b, h, i)
+                k = O.k_from_sparsity(i + 1, w.sparsity_permille)
+                got = idx[b, h, i, : n_sel[b, h, i]]
+                if O.selection_margin(row, k, True) > MARGIN:
+                    assert got.tolist() == O.select_blocks(row, k, True).tolist(), (b, h, i)
+                    exact += 1
+                else:
+                    assert O.selection_is_valid(row, got, k, True, MARGIN), (b, h, i)
+                lo, hi = i * bs, min((i + 1) * bs, L)
+                for t in sorted({lo, hi - 1, int(rng.integers(lo, hi))}):
+                    ref_o, ref_l = O.prefill_attention_token(Qg, K, V, L, t, got, bs, scale)
+                    assert_out_close(f64(run.out[b, t, h * G:(h + 1) * G]), ref_o, (b, h, t))
+                    np.testing.assert_allclose(f64(run.lse[b, h * G:(h + 1) * G, t]), ref_l,
+                                               atol=1e-3)
+    assert exact > 0

@@ -238,9 +238,9 @@ FULL = [
 def test_step_full_size_sampled(name, over):
     w = W.WORKLOADS[name].replace(**over)
     data = W.generate(w, 1, DEV)
-    run = StepBuffers(w, data)          # the benchmark's launch configuration
-    run.pool_full()
-    run.step(update_kbar=0)
+    run = StepBuffers(w, data)          # the benchmark's launch configuration:
+    run.pool_full()                     # full pooling once, then the step with the
+    run.step(update_kbar=1)             # incremental newest-block refresh
     torch.cuda.synchronize()
     assert run.status.item() == 0
     rng = np.random.default_rng(0)

@@ -454,3 +454,11 @@ def test_prefill_closed_forms_and_hand_case():
     got = O.prefill_select(s, lambda i: 2)
     assert [g.tolist() for g in got] == [[0], [0, 1], [1, 2]]
 
+    # the one-row and one-token forms the full-size tests sample
+    np.testing.assert_allclose(O.prefill_gate_row(Q, np.eye(D), kb, L, bs, 0.5, 2),
+                               qbar[2, :3] * 0.5, rtol=1e-13)
+    o, l = O.prefill_attention_token(Q, K, V, L, 40, [1], bs, 0.7)
+    x = Q[40] @ K[32:41].T * 0.7                                # keys 32..40 of block 1
+    from scipy.special import logsumexp, softmax
+    np.testing.assert_allclose(o, softmax(x, axis=1) @ V[32:41], rtol=1e-12)
+    np.testing.assert_allclose(l, logsumexp(x, axis=1), rtol=1e-13)
