@@ -180,7 +180,7 @@ static seer_status decode_prepare(const seer_dims* d, const uint16_t* q, const u
   if (!q || !seqlens || !idx || !n_sel || !o_part || !lse_part) return SEER_ERR_INVALID_ARG;
   if (k_max < 1 || k_max > d->max_blocks || num_splits < 1 || num_splits > kMaxSplits)
     return SEER_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(o_part, 8) || !aligned(work_counter, 8))
+  if (!aligned(q, 16) || !aligned(o_part, 16) || !aligned(work_counter, 8))
     return SEER_ERR_UNSUPPORTED;
   const int64_t items = (int64_t)d->batch * d->num_kv_heads * num_splits;
   if (items > INT_MAX / 2) return SEER_ERR_UNSUPPORTED;  // item ids carry a flag bit

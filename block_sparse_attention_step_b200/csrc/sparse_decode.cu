@@ -45,10 +45,20 @@ constexpr int kItemSlots = 3;
 constexpr int kOStride = kHeadDim + 4;                 // padded merge row (floats)
 constexpr int kEntries = 256;                          // stage entries in flight (power of 2)
 
-template <int NT, int STAGES, int MSLOTS>
+// The per-stage kernel with two merge slots hands each finished item's merge
+// to warps of their own; the single-launch step (whose gate phase is sized
+// for 10 warps) and the one-slot shapes keep the merge in the math warps.
+constexpr int kMergeWarpsPerCta = 2;
+constexpr int merge_warps(int mslots, bool fused) {
+  return (!fused && mslots == 2) ? kMergeWarpsPerCta : 0;
+}
+
+template <int NT, int STAGES, int MSLOTS, int MW = 0>
 struct DecodeShape {
   static constexpr int kMathWarps = 8;
-  static constexpr int kThreads = (kMathWarps + 2) * 32;  // + copy warp + scheduler warp
+  static constexpr int kMergeWarps = MW;
+  // + copy warp + scheduler warp (+ merge warp)
+  static constexpr int kThreads = (kMathWarps + 2 + MW) * 32;
   static constexpr int kGroups = 2;
   // Stage k goes to group k % kGroups and slot k % kStages.  The ring depth
   // must be a multiple of the group count so that every slot is always
@@ -138,11 +148,13 @@ __device__ __forceinline__ int ld_row_data(const int32_t* ptr) {
 }
 
 template <int NT, int STAGES, int MSLOTS, bool MASS, bool FUSED>
-__global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
+__global__ void __launch_bounds__(
+    DecodeShape<NT, STAGES, MSLOTS, merge_warps(MSLOTS, FUSED)>::kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const DecodeParams p,
                          const FusedParams f) {
-  using Shape = DecodeShape<NT, STAGES, MSLOTS>;
+  using Shape = DecodeShape<NT, STAGES, MSLOTS, merge_warps(MSLOTS, FUSED)>;
+  constexpr bool kMergeWarp = Shape::kMergeWarps > 0;
   static_assert(Shape::kMathWarps == 8 && Shape::kGroups == 2, "merge order assumes 2 x 4 warps");
   constexpr int kStages = Shape::kStages;
   constexpr int kQSlotBytes = Shape::kQSlotBytes;
@@ -174,6 +186,99 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
   const int G = p.G;
   const size_t o_slot = Shape::o_slot_floats(G);
 
+  // Item number u's merge: every math warp's (m, l, O) of that item is in
+  // merge slot u % MSLOTS once state_full completes (the caller has waited
+  // for that when `waited`); threads tid = 0 .. nthr - 1 of the merging
+  // warps take outputs e = tid, tid + nthr, ... of the G x D block, write
+  // o_part / lse_part and free the slot.  Group (item's first stage's parity)
+  // first, then the other group: the sums then run in the same order
+  // whichever group took the item's first stage, so an item's partials do
+  // not depend on which CTA ran it, what that CTA ran before, or which warps
+  // merge it.  Merge warps take one head's row per pass (the head's weights
+  // worked out once), math warps one output per pass: the same values in the
+  // same order either way.
+  auto merge_item = [&](int u, int tid, int nthr, bool waited, bool& okr) {
+    const int ms = u % MSLOTS;
+    const uint32_t use = (uint32_t)(u / MSLOTS);
+    if (!waited && okr && !mbar_wait(&state_full[ms], use & 1)) {
+      flag_status(p.status, SEER_DEV_TIMEOUT);
+      okr = false;
+    }
+    const int mitem = slot_item[ms] >> 1;
+    if (okr && mitem >= 0 && mitem < p.num_items) {
+      const int first = slot_item[ms] & 1;
+      const int bh = item_bh(p, mitem);
+      const int s = mitem / (p.B * p.Hkv);
+      const int b = bh / p.Hkv;
+      const int h = bh - b * p.Hkv;
+      const float* mls = ml_base + (size_t)ms * (Shape::kMLBytes / 4);
+      const float* os = o_base + (size_t)ms * o_slot;
+      if (waited) {
+        // merge warps: one head's row per warp and pass, 4 outputs per lane
+        // (d = 4 lane .. 4 lane + 3, float4 loads), the head's weights once
+        const int d0 = 4 * lane;
+        for (int g = tid; g < G; g += nthr) {
+          float mt = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kMathWarps; ++w) mt = fmaxf(mt, mls[w * 2 * kMaxGroup + g]);
+          const int64_t orow = ((int64_t)b * p.Hq + (int64_t)h * G + g) * p.S + s;
+          float4* dst = reinterpret_cast<float4*>(p.o_part + orow * kHeadDim + d0);
+          if (mt == -INFINITY) {
+            *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (lane == 0) p.lse_part[orow] = -INFINITY;
+            continue;
+          }
+          float fw[kMathWarps], lt = 0.f;
+#pragma unroll
+          for (int wr = 0; wr < kMathWarps; ++wr) {
+            const int w = wr ^ (first << 2);  // kMathWarps == 8, groups of 4
+            fw[wr] = fast_exp2(mls[w * 2 * kMaxGroup + g] - mt);
+            lt = __fmaf_rn(mls[w * 2 * kMaxGroup + kMaxGroup + g], fw[wr], lt);
+          }
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int wr = 0; wr < kMathWarps; ++wr) {
+            const int w = wr ^ (first << 2);
+            const float4 v =
+                *reinterpret_cast<const float4*>(os + ((size_t)w * G + g) * kOStride + d0);
+            acc.x = __fmaf_rn(v.x, fw[wr], acc.x);
+            acc.y = __fmaf_rn(v.y, fw[wr], acc.y);
+            acc.z = __fmaf_rn(v.z, fw[wr], acc.z);
+            acc.w = __fmaf_rn(v.w, fw[wr], acc.w);
+          }
+          *dst = make_float4(acc.x / lt, acc.y / lt, acc.z / lt, acc.w / lt);
+          if (lane == 0) p.lse_part[orow] = (mt + log2f(lt)) * kLn2;
+        }
+      } else {
+        // the math warps: one output per thread and pass, weights on the fly
+        for (int e = tid; e < G * kHeadDim; e += nthr) {
+          const int g = e / kHeadDim, d = e - g * kHeadDim;
+          float mt = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kMathWarps; ++w) mt = fmaxf(mt, mls[w * 2 * kMaxGroup + g]);
+          const int64_t orow = ((int64_t)b * p.Hq + (int64_t)h * G + g) * p.S + s;
+          if (mt == -INFINITY) {
+            p.o_part[orow * kHeadDim + d] = 0.f;
+            if (d == 0) p.lse_part[orow] = -INFINITY;
+            continue;
+          }
+          float lt = 0.f, acc = 0.f;
+#pragma unroll
+          for (int wr = 0; wr < kMathWarps; ++wr) {
+            const int w = wr ^ (first << 2);
+            const float f = fast_exp2(mls[w * 2 * kMaxGroup + g] - mt);
+            lt = __fmaf_rn(mls[w * 2 * kMaxGroup + kMaxGroup + g], f, lt);
+            acc = __fmaf_rn(os[((size_t)w * G + g) * kOStride + d], f, acc);
+          }
+          p.o_part[orow * kHeadDim + d] = acc / lt;
+          if (d == 0) p.lse_part[orow] = (mt + log2f(lt)) * kLn2;
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&state_empty[ms]);
+  };
+
   if (threadIdx.x == 0) {
     *ent_tail = 0;
     *ent_head = 0;
@@ -186,8 +291,9 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       mbar_init(&item_empty[i], kMathWarps);
     }
     for (int i = 0; i < MSLOTS; ++i) {
+      // every merge warp waits on state_full; whoever merges frees the slot
       mbar_init(&state_full[i], kMathWarps);
-      mbar_init(&state_empty[i], kMathWarps);
+      mbar_init(&state_empty[i], kMergeWarp ? Shape::kMergeWarps : kMathWarps);
     }
     fence_mbar_init();
   }
@@ -233,6 +339,24 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
       }
     }
     __syncthreads();  // ring and merge area belong to the decode from here on
+  }
+
+  if (kMergeWarp && warp >= kMathWarps + 2) {
+    // =========================================================== merge warps
+    // Merge each item the math warps drop into a merge slot, one item behind
+    // them, each warp its share of the item's head rows; an item id of -1 in
+    // a slot ends the run.
+    bool mok = true;
+    for (int u = 0; mok; ++u) {
+      const int ms = u % MSLOTS;
+      if (!mbar_wait(&state_full[ms], (u / MSLOTS) & 1)) {
+        flag_status(p.status, SEER_DEV_TIMEOUT);
+        break;
+      }
+      if (slot_item[ms] < 0) break;
+      merge_item(u, warp - (kMathWarps + 2), Shape::kMergeWarps, true, mok);
+    }
+    return;
   }
 
   if (warp == kMathWarps + 1) {
@@ -508,54 +632,6 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
   bool ok = true;
   int last_it = -1;
 
-  // This warp's 1/8 of item number u's merge: every warp's (m, l, O) of that
-  // item is in slot u % MSLOTS once state_full completes; thread (warp, lane)
-  // takes outputs e = warp * 32 + lane, + 256, ... of the G x D block.
-  auto merge_share = [&](int u) {
-    const int ms = u % MSLOTS;
-    const uint32_t use = (uint32_t)(u / MSLOTS);
-    if (ok && !mbar_wait(&state_full[ms], use & 1)) {
-      flag_status(p.status, SEER_DEV_TIMEOUT);
-      ok = false;
-    }
-    // Group (item's first stage's parity) first, then the other group: the
-    // sum then runs in the same order whichever group took the item's first
-    // stage, so an item's partials do not depend on which CTA ran it or what
-    // that CTA ran before.
-    const int mitem = slot_item[ms] >> 1;
-    const int first = slot_item[ms] & 1;
-    const int bh = item_bh(p, mitem);
-    const int s = mitem / (p.B * p.Hkv);
-    const int b = bh / p.Hkv;
-    const int h = bh - b * p.Hkv;
-    const float* mls = ml_base + (size_t)ms * (Shape::kMLBytes / 4);
-    const float* os = o_base + (size_t)ms * o_slot;
-    for (int e = warp * 32 + lane; e < G * kHeadDim; e += kMathThreads) {
-      const int g = e / kHeadDim, d = e - g * kHeadDim;
-      float mt = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kMathWarps; ++w) mt = fmaxf(mt, mls[w * 2 * kMaxGroup + g]);
-      const int64_t orow = ((int64_t)b * p.Hq + (int64_t)h * G + g) * p.S + s;
-      if (mt == -INFINITY) {
-        p.o_part[orow * kHeadDim + d] = 0.f;
-        if (d == 0) p.lse_part[orow] = -INFINITY;
-        continue;
-      }
-      float lt = 0.f, acc = 0.f;
-#pragma unroll
-      for (int wr = 0; wr < kMathWarps; ++wr) {
-        const int w = wr ^ (first << 2);  // kMathWarps == 8, groups of 4
-        const float f = fast_exp2(mls[w * 2 * kMaxGroup + g] - mt);
-        lt += mls[w * 2 * kMaxGroup + kMaxGroup + g] * f;
-        acc += os[((size_t)w * G + g) * kOStride + d] * f;
-      }
-      p.o_part[orow * kHeadDim + d] = acc / lt;
-      if (d == 0) p.lse_part[orow] = (mt + log2f(lt)) * kLn2;
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&state_empty[ms]);
-  };
-
   for (int it_no = 0; ok; ++it_no) {
     const int islot = it_no % kItemSlots;
     const uint32_t iphase = (it_no / kItemSlots) & 1;
@@ -776,7 +852,7 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
         l[nt][e] = v;
       }
     }
-    if (it_no > 0) merge_share(it_no - 1);
+    if (!kMergeWarp && it_no > 0) merge_item(it_no - 1, warp * 32 + lane, kMathThreads, false, ok);
     {
       const int ms = it_no % MSLOTS;
       const uint32_t use = (uint32_t)(it_no / MSLOTS);
@@ -816,7 +892,20 @@ __global__ void __launch_bounds__(DecodeShape<NT, STAGES, MSLOTS>::kThreads, 1)
     }
     last_it = it_no;
   }
-  if (last_it >= 0) merge_share(last_it);
+  if constexpr (kMergeWarp) {
+    // end-of-items mark for the merge warp, in the slot after the last item
+    const int u = last_it + 1;
+    const int ms = u % MSLOTS;
+    if (ok && !mbar_wait(&state_empty[ms], ((u / MSLOTS) & 1) ^ 1)) {
+      flag_status(p.status, SEER_DEV_TIMEOUT);
+      ok = false;
+    }
+    if (warp == 0 && lane == 0) slot_item[ms] = -1;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&state_full[ms]);
+  } else if (last_it >= 0) {
+    merge_item(last_it, warp * 32 + lane, kMathThreads, false, ok);
+  }
 
   // ---- single-launch step, phase C: the LSE combine of this CTA's rows by
   // the math warps, once every math warp of the grid has written its last
@@ -861,7 +950,7 @@ template <int NT, int STAGES, int MSLOTS, bool MASS, bool FUSED>
 static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
                                  const DecodeParams& p, const FusedParams& f, int num_sms,
                                  cudaStream_t stream, bool pdl) {
-  using Shape = DecodeShape<NT, STAGES, MSLOTS>;
+  using Shape = DecodeShape<NT, STAGES, MSLOTS, merge_warps(MSLOTS, FUSED)>;
   const size_t smem = FUSED ? Shape::smem_bytes_fused(p.G) : Shape::smem_bytes(p.G);
   auto kern = sparse_decode_kernel<NT, STAGES, MSLOTS, MASS, FUSED>;
   static std::atomic<uint64_t> smem_set{0};

@@ -56,7 +56,8 @@
  *   scores     [B][Hkv][max_blocks] fp32 (-inf at j >= NB_b)
  *   idx        [B][Hkv][k_max] int32, ascending, -1 after the n_sel entries
  *   n_sel      [B][Hkv] int32
- *   o_part     [B][Hq][num_splits][D] fp32, lse_part [B][Hq][num_splits] fp32
+ *   o_part     [B][Hq][num_splits][D] fp32 (16-byte aligned),
+ *              lse_part [B][Hq][num_splits] fp32
  *   out        [B][Hq][D] bf16 (round-to-nearest-even), lse_out [B][Hq] fp32
  *              natural-log log-sum-exp of the scaled scores (-inf if empty)
  */

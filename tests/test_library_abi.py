@@ -85,6 +85,9 @@ def test_invalid_arguments_fail_before_any_launch(lib):
     odd = ctypes.c_void_p(4096 + 2)
     assert lib.seer_sparse_decode(ctypes.byref(d), fake, odd, fake, null, fake, fake, fake, 4, 1,
                                   0.1, fake, fake, null, null, null) == 2
+    # o_part not 16-byte aligned (the merge writes float4 rows)
+    assert lib.seer_sparse_decode(ctypes.byref(d), fake, fake, fake, null, fake, fake, fake, 4, 1,
+                                  0.1, ctypes.c_void_p(4096 + 8), fake, null, null, null) == 2
     # misaligned item counter
     assert lib.seer_sparse_decode(ctypes.byref(d), fake, fake, fake, null, fake, fake, fake, 4, 1,
                                   0.1, fake, fake, ctypes.c_void_p(4096 + 4), null, null) == 2
