@@ -262,7 +262,15 @@ def run_ours(args):
     # replicas: enough that one rotation reads > 4x L2
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
     probe = W.generate(w, args.seed + 1000 * rank, dev, layout=args.layout)
-    run0 = StepBuffers(w, probe, num_splits=args.splits, mass=args.mass, unified=args.unified)
+    k_cap = None
+    if w.seqlen_range is not None:
+        # the other replicas draw other lengths: size the index rows for the
+        # longest sequence the workload allows, so that no replica's k is clamped
+        nb = -(-w.seqlen_range[1] // w.block_size)
+        k_cap = (seer.seer_k_from_budget(nb, w.budget_tokens, w.block_size) if w.budget_tokens
+                 else seer.seer_k_from_sparsity(nb, w.sparsity_permille))
+    run0 = StepBuffers(w, probe, num_splits=args.splits, k_max=k_cap, mass=args.mass,
+                       unified=args.unified)
     run0.pool_full()
     torch.cuda.synchronize()
     sel_bytes, sel_tokens = selected_bytes(run0, probe, w)

@@ -29,10 +29,11 @@
 //   * online softmax per head column in the exp2 domain; P^T enters the
 //     tensor cores through movmatrix as a bf16 hi + lo pair (weights kept to
 //     ~16 bits); tail tokens past seqlen are masked in registers;
-//   * at the end of an item each warp drops its (m, l, O) into a shared-memory
-//     slot (mbarrier-counted) and, one item later, merges 1/8 of that item's
-//     outputs into o_part / lse_part: with two slots no warp waits for
-//     another at item boundaries.
+//   * at the end of an item each math warp drops its (m, l, O) into a
+//     shared-memory slot (mbarrier-counted) and goes on; two merge warps merge
+//     the item's head rows into o_part / lse_part and free the slot, so the
+//     math warps never stop at item boundaries (the single-launch step and
+//     the one-slot shapes merge in the math warps instead, one item later).
 // Every mbarrier wait is bounded (SEER_DEV_TIMEOUT); nothing traps.
 #include "gate_row.cuh"
 #include "combine_core.cuh"
