@@ -19,7 +19,9 @@ __global__ void __launch_bounds__(kHeadDim) combine_kernel(const CombineParams p
   float lse;
   const float v = combine_element(p.lse_part + row * p.S, p.o_part + row * p.S * kHeadDim + d,
                                   p.S, &lse, LoadReadOnly{});
-  p.out[row * kHeadDim + d] = to_bf16_bits(v);
+  const uint16_t bits = to_bf16_bits(v);
+  p.out[row * kHeadDim + d] = bits;
+  if (p.out_host != nullptr) p.out_host[row * kHeadDim + d] = bits;
   if (p.lse_out != nullptr && d == 0) p.lse_out[row] = lse;
 }
 

@@ -168,14 +168,25 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
       wrow[r] = __ldg(reinterpret_cast<const float4*>(W + (warp + r * WORKERS) * kHeadDim +
                                                       4 * lane));
   }
-  // mean query of the group
+  // mean query of the group (q in mapped host memory: read through L2 and
+  // copied to q_copy for the decode)
   if (tid >= QFIRST && tid < QFIRST + QTHREADS) {
 #pragma unroll
     for (int m = 0; m < kHeadDim / QTHREADS; ++m) {
       const int d = tid - QFIRST + m * QTHREADS;
-      const uint16_t* qg = p.q + ((int64_t)b * p.Hq + (int64_t)h * p.G) * kHeadDim + d;
+      const int64_t off = ((int64_t)b * p.Hq + (int64_t)h * p.G) * kHeadDim + d;
       float s = 0.f;
-      for (int g = 0; g < p.G; ++g) s += __uint_as_float((uint32_t)__ldg(qg + g * kHeadDim) << 16);
+      if (p.q_copy != nullptr) {
+        for (int g = 0; g < p.G; ++g) {
+          const unsigned short v = __ldcg(reinterpret_cast<const unsigned short*>(p.q) + off +
+                                          g * kHeadDim);
+          p.q_copy[off + g * kHeadDim] = v;
+          s += __uint_as_float((uint32_t)v << 16);
+        }
+      } else {
+        for (int g = 0; g < p.G; ++g)
+          s += __uint_as_float((uint32_t)__ldg(p.q + off + g * kHeadDim) << 16);
+      }
       gs.qbar[d] = s / (float)p.G;
     }
   }

@@ -462,7 +462,7 @@ seer_status seer_combine(const seer_dims* d, const float* o_part, const float* l
   SEER_TRY(check_dims(d));
   if (!o_part || !lse_part || !out) return SEER_ERR_INVALID_ARG;
   if (num_splits < 1 || num_splits > kMaxSplits) return SEER_ERR_INVALID_ARG;
-  CombineParams p;
+  CombineParams p = {};
   p.o_part = o_part;
   p.lse_part = lse_part;
   p.out = out;
@@ -472,7 +472,12 @@ seer_status seer_combine(const seer_dims* d, const float* o_part, const float* l
   return SEER_OK;
 }
 
-seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_stream stream) {
+// The step; q_mapped / out_mapped (optional): host memory mapped into the
+// device, read by the gate (which fills a->q for the decode) / written by the
+// combine besides a->out.
+static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
+                                    seer_stream stream, const uint16_t* q_mapped,
+                                    uint16_t* out_mapped) {
   SEER_TRY(check_dims(d));
   if (a == nullptr || a->k_per_seq == nullptr || a->kbar == nullptr) return SEER_ERR_INVALID_ARG;
   if (a->update_kbar < 0 || a->update_kbar > 2) return SEER_ERR_INVALID_ARG;
@@ -499,7 +504,8 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
                             stream));
   // a0 (incremental) + a1 + a2 in one kernel; same results as the three calls
   GateSelectParams g = {};
-  g.q = a->q;
+  g.q = q_mapped != nullptr ? q_mapped : a->q;
+  g.q_copy = q_mapped != nullptr ? const_cast<uint16_t*>(a->q) : nullptr;
   g.w_gate = a->w_gate;
   g.kbar = a->kbar;
   g.seqlens = a->seqlens;
@@ -558,12 +564,13 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
   }
   // a3, then a4; each grid launches early and waits for its predecessor
   SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, true));
-  CombineParams c;
+  CombineParams c = {};
   c.o_part = w.o_part;
   c.lse_part = w.lse_part;
   c.out = a->out;
   c.lse_out = a->lse_out;
   c.S = a->num_splits;
+  c.out_host = out_mapped;
   SEER_CUDA(run_combine(c, d->batch, d->num_q_heads, stream, true));
   if (mass) {
     MassParams m;
@@ -582,6 +589,10 @@ seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_s
     SEER_CUDA(run_block_mass(m, d->batch, stream));
   }
   return SEER_OK;
+}
+
+seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_stream stream) {
+  return decode_step_impl(d, a, stream, nullptr, nullptr);
 }
 
 seer_status seer_step_workspace_init(const seer_dims* d, int32_t k_max, int32_t num_splits,
@@ -725,6 +736,21 @@ seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_st
   return SEER_OK;
 }
 
+// Device address of host memory that is pinned and mapped into the device's
+// address space, else NULL (pageable memory, or not a host pointer).
+static void* mapped_host_ptr(const void* host) {
+  cudaPointerAttributes at;
+  if (host == nullptr || cudaPointerGetAttributes(&at, host) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
+int32_t seer_host_ptr_mapped(const void* host_ptr) {
+  return mapped_host_ptr(host_ptr) != nullptr ? 1 : 0;
+}
+
 seer_status seer_decode_step_host(const seer_dims* d, const seer_step_args* a,
                                   const uint16_t* q_host, uint16_t* q_dev, uint16_t* out_host,
                                   seer_stream stream) {
@@ -733,11 +759,17 @@ seer_status seer_decode_step_host(const seer_dims* d, const seer_step_args* a,
       a->out == nullptr)
     return SEER_ERR_INVALID_ARG;
   const size_t bytes = (size_t)d->batch * d->num_q_heads * d->head_dim * sizeof(uint16_t);
-  SEER_CUDA(cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, stream));
+  // mapped buffers are read and written by the step's own kernels; others
+  // go through a copy on the stream
+  const uint16_t* q_map = static_cast<const uint16_t*>(mapped_host_ptr(q_host));
+  uint16_t* out_map = static_cast<uint16_t*>(mapped_host_ptr(out_host));
+  if (q_map == nullptr)
+    SEER_CUDA(cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, stream));
   seer_step_args b = *a;
   b.q = q_dev;
-  SEER_TRY(seer_decode_step(d, &b, stream));
-  SEER_CUDA(cudaMemcpyAsync(out_host, a->out, bytes, cudaMemcpyDeviceToHost, stream));
+  SEER_TRY(decode_step_impl(d, &b, stream, q_map, out_map));
+  if (out_map == nullptr)
+    SEER_CUDA(cudaMemcpyAsync(out_host, a->out, bytes, cudaMemcpyDeviceToHost, stream));
   return SEER_OK;
 }
 

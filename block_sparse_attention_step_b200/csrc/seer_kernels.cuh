@@ -60,6 +60,10 @@ struct GateSelectParams {
   uint32_t* work_counter;  // optional: zeroed for the decode grid that follows
   int B;
   uint32_t* row_counter;   // the row-claiming gate grid's counter (zero before it starts)
+  // optional: q is then host memory mapped into the device's address space,
+  // and each gate row copies its group's query rows into q_copy (device) for
+  // the decode grid
+  uint16_t* q_copy;
 };
 
 struct DecodeParams {
@@ -141,6 +145,7 @@ struct CombineParams {
   uint16_t* out;
   float* lse_out;
   int S;
+  uint16_t* out_host;  // optional: host memory mapped into the device, written besides out
 };
 
 cudaError_t run_pool_keys(const PoolParams& p, int B, cudaStream_t stream);

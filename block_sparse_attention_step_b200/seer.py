@@ -34,7 +34,8 @@ EXPORTS = (
     "seer_k_from_budget", "seer_fill_k", "seer_default_splits", "seer_step_workspace_bytes",
     "seer_pool_keys", "seer_gate_scores", "seer_block_select", "seer_block_select_unified",
     "seer_sparse_decode",
-    "seer_combine", "seer_decode_step", "seer_decode_step_host", "seer_decode_step_noalloc",
+    "seer_combine", "seer_decode_step", "seer_decode_step_host", "seer_host_ptr_mapped",
+    "seer_decode_step_noalloc",
     "seer_decode_step_fused", "seer_step_workspace_init",
     "seer_prefill_k_max", "seer_prefill_workspace_bytes", "seer_prefill",
     "seer_block_lse_elems", "seer_sparse_decode_mass", "seer_block_mass",
@@ -108,6 +109,7 @@ _SIGS = {
     "seer_combine": (_I, [_D, _P, _P, _I, _P, _P, _P]),
     "seer_decode_step": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_decode_step_host": (_I, [_D, ctypes.POINTER(seer_step_args), _P, _P, _P, _P]),
+    "seer_host_ptr_mapped": (_I, [_P]),
     "seer_decode_step_noalloc": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_decode_step_fused": (_I, [_D, ctypes.POINTER(seer_step_args), _P]),
     "seer_step_workspace_init": (_I, [_D, _I, _I, _P, ctypes.c_size_t, _P]),
@@ -321,6 +323,14 @@ def seer_decode_step_host(d, args: seer_step_args, q_host, q_dev, out_host, stre
         ctypes.byref(d), ctypes.byref(args), _ptr(q_host, torch.bfloat16, "q_host", device=False),
         _ptr(q_dev, torch.bfloat16, "q_dev"), _ptr(out_host, torch.bfloat16, "out_host", device=False),
         _stream(stream)))
+
+
+def seer_host_ptr_mapped(t) -> bool:
+    """True if seer_decode_step_host accesses this host tensor directly from
+    its kernels (pinned and mapped into the device), False if it copies."""
+    if t.is_cuda:
+        raise ValueError("expected a host tensor")
+    return bool(_lib().seer_host_ptr_mapped(ctypes.c_void_p(t.data_ptr())))
 
 
 def seer_decode_step_noalloc(d, args: seer_step_args, stream=None):

@@ -281,14 +281,24 @@ typedef struct seer_step_args {
 SEER_API seer_status seer_decode_step(const seer_dims *d, const seer_step_args *a,
                              seer_stream stream);
 
-/* End-to-end form for callers holding q and out in host memory: enqueues the
- * copy q_host -> q_dev (B*Hq*D bf16), the step with a->q replaced by q_dev,
- * and the copy a->out -> out_host.  Asynchronous: with pinned host buffers
- * the copies overlap nothing else on `stream`, and out_host is valid after
- * the stream is synchronised. */
+/* End-to-end form for callers holding q and out in host memory: the step with
+ * a->q replaced by q_dev, q taken from q_host (B*Hq*D bf16) and the output
+ * delivered to out_host (B*Hq*D bf16) as well as a->out.  A host buffer that
+ * is pinned and mapped into the device's address space (cudaHostAlloc /
+ * cudaMallocHost memory, or cudaHostRegister'ed with the mapped flag; see
+ * seer_host_ptr_mapped) is accessed by the step's kernels directly: the gate
+ * reads q_host and fills q_dev, the combine writes out_host, and no copy is
+ * enqueued.  Any other host buffer goes through cudaMemcpyAsync on `stream`
+ * (before the step for q, after it for out).  Asynchronous either way: q_host
+ * must stay unchanged and out_host is valid only once the stream is
+ * synchronised. */
 SEER_API seer_status seer_decode_step_host(const seer_dims *d, const seer_step_args *a,
                                   const uint16_t *q_host, uint16_t *q_dev,
                                   uint16_t *out_host, seer_stream stream);
+
+/* 1 if seer_decode_step_host reads or writes this host buffer directly
+ * (pinned and mapped into the device's address space), else 0. */
+SEER_API int32_t seer_host_ptr_mapped(const void *host_ptr);
 
 /* ------------------------------------------------- per-block attention mass
  * The dense model's block-level attention distribution is what the

@@ -203,20 +203,44 @@ def test_step_incremental_kbar_matches_full_rebuild():
     assert run.status.item() == 0
 
 
-def test_step_host_entry_point_matches_device_step():
-    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=2, seqlen=1500)
+HOST_CASES = {
+    "per_row_gate": W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=2, seqlen=1500),
+    # more (b, h) rows than SMs: the row-claiming gate grid
+    "row_claiming_gate": W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(
+        batch=80, q_heads=8, kv_heads=2, seqlen_range=(1, 3000)),
+}
+
+
+@pytest.mark.parametrize("pinned_q,pinned_out", [(True, True), (False, False), (True, False),
+                                                 (False, True)])
+@pytest.mark.parametrize("name", list(HOST_CASES))
+def test_step_host_entry_point_matches_device_step(name, pinned_q, pinned_out):
+    """q and out in host memory: pinned (mapped) buffers are read and written
+    by the step's kernels, pageable ones go through copies; either way the
+    same bits as the device step, q_dev filled and a->out written too."""
+    w = HOST_CASES[name]
     data = W.generate(w, 3, DEV)
     run = StepBuffers(w, data)
     run.pool_full()
-    run.step()
-    dev_out = run.out.clone()
-    q_host = data["q"].cpu().pin_memory()
-    out_host = torch.empty(dev_out.shape, dtype=torch.bfloat16).pin_memory()
-    q_dev = torch.empty_like(data["q"])
-    run.out.zero_()
-    seer.seer_decode_step_host(run.dims, run.args(0, q=q_dev), q_host, q_dev, out_host)
+    kbar0 = run.kbar.clone()
+    run.step(update_kbar=1)
     torch.cuda.synchronize()
+    dev_out = run.out.clone()
+    q_host = data["q"].cpu()
+    q_host = q_host.pin_memory() if pinned_q else q_host.clone()
+    out_host = torch.empty(dev_out.shape, dtype=torch.bfloat16)
+    out_host = out_host.pin_memory() if pinned_out else out_host
+    assert seer.seer_host_ptr_mapped(q_host) == pinned_q
+    assert seer.seer_host_ptr_mapped(out_host) == pinned_out
+    q_dev = torch.zeros_like(data["q"])
+    run.kbar.copy_(kbar0)
+    run.out.zero_()
+    seer.seer_decode_step_host(run.dims, run.args(1, q=q_dev), q_host, q_dev, out_host)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    assert torch.equal(q_dev.cpu(), q_host)
     assert torch.equal(out_host, dev_out.cpu())
+    assert torch.equal(run.out, dev_out)
 
 
 # --------------------------------------------------------- full-size, sampled
