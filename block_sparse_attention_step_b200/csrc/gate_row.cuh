@@ -121,11 +121,14 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
                   bytes, &bars[slot]);
   };
 
-  // the first chunks go out before anything else (free slots: this row's
-  // own chunks, then, if the row is short, the next row's)
+  // The first chunk goes out before anything else; the other free slots
+  // (this row's own chunks, then, if the row is short, the next row's) are
+  // filled once the loads that form g below have returned.  One chunk per
+  // row already keeps HBM busy across the grid, and the few loads that g
+  // needs would otherwise queue behind every row's whole first burst.
+  constexpr int kBurst = 1;
   if (tid == 0)
-    for (int u = (int)first; u < NBUF && u < stream_len; ++u) issue(u);
-  issued = (uint32_t)max((int)first, min(NBUF, stream_len));
+    for (int u = (int)first; u < kBurst && u < stream_len; ++u) issue(u);
 
   // KV append: the new token's K and V rows of head h at position L - 1
   const bool append = p.k_new != nullptr && L > 0;
@@ -191,6 +194,9 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
     }
   }
   __syncthreads();
+  if (tid == 0)
+    for (int u = max((int)first, kBurst); u < NBUF && u < stream_len; ++u) issue(u);
+  issued = (uint32_t)max((int)first, min(NBUF, stream_len));
   if (refresh && tid < kHeadDim) {
     float v = 0.f;
     if (!bad_page) v = pool_finish(gs.part, tid, valid_new);
