@@ -46,12 +46,13 @@ constexpr int kItemSlots = 3;
 constexpr int kOStride = kHeadDim + 4;                 // padded merge row (floats)
 constexpr int kEntries = 256;                          // stage entries in flight (power of 2)
 
-// The per-stage kernel with two merge slots hands each finished item's merge
-// to warps of their own; the single-launch step (whose gate phase is sized
-// for 10 warps) and the one-slot shapes keep the merge in the math warps.
+// The two-slot shapes hand each finished item's merge to warps of their own
+// (in the single-launch step they also take part in the gate phase and the
+// final combine); the one-slot shapes keep the merge in the math warps.
 constexpr int kMergeWarpsPerCta = 2;
 constexpr int merge_warps(int mslots, bool fused) {
-  return (!fused && mslots == 2) ? kMergeWarpsPerCta : 0;
+  (void)fused;
+  return mslots == 2 ? kMergeWarpsPerCta : 0;
 }
 
 template <int NT, int STAGES, int MSLOTS, int MW = 0>
@@ -198,6 +199,46 @@ __global__ void __launch_bounds__(
   // merge it.  Merge warps take one head's row per pass (the head's weights
   // worked out once), math warps one output per pass: the same values in the
   // same order either way.
+  // Single-launch step, phase C: the LSE combine of this CTA's rows by the
+  // math warps and merge warps, once every CTA of the grid has written its
+  // last partials.  (Split-major items put every row's last split among the
+  // last items, so waiting for the whole grid costs little over waiting per
+  // row, and it takes one fence per warp instead of one per item.)
+  auto phase_c = [&]() {
+    constexpr int kCombineWarps = kMathWarps + Shape::kMergeWarps;
+    __syncwarp();
+    if (lane == 0) __threadfence();  // this warp's partials are out
+    named_barrier_sync(1, kCombineWarps * 32);
+    if (threadIdx.x == 0) {  // one arrival per CTA
+      __threadfence();
+      atomicAdd(f.ctl + 3, 1u);
+      const uint32_t want = gridDim.x;
+      const long long t0 = clock64();
+      while (ld_acquire_gpu(f.ctl + 3) < want) {
+        __nanosleep(64);
+        if (clock64() - t0 > (1ll << 31)) {
+          flag_status(p.status, SEER_DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    named_barrier_sync(1, kCombineWarps * 32);
+    // one warp per (b, query head) row, spread over the combining warps of
+    // the grid (merge warps follow the math warps)
+    const int cw = warp < kMathWarps ? warp : warp - 2;
+    const int qrows = p.B * p.Hq;
+    for (int q = blockIdx.x * kCombineWarps + cw; q < qrows; q += gridDim.x * kCombineWarps)
+      combine_row_warp(p.lse_part + (int64_t)q * p.S, p.o_part + (int64_t)q * p.S * kHeadDim,
+                       p.S, f.out + (int64_t)q * kHeadDim,
+                       f.lse_out != nullptr ? f.lse_out + q : nullptr, Load4L2{});
+    // the last CTA through its combine puts the two counters back to zero
+    // (every CTA has passed the wait above by then)
+    if (threadIdx.x == 0 && atomicAdd(f.ctl + 4, 1u) == gridDim.x - 1) {
+      atomicExch(f.ctl + 3, 0u);
+      atomicExch(f.ctl + 4, 0u);
+    }
+  };
+
   auto merge_item = [&](int u, int tid, int nthr, bool waited, bool& okr) {
     const int ms = u % MSLOTS;
     const uint32_t use = (uint32_t)(u / MSLOTS);
@@ -357,6 +398,7 @@ __global__ void __launch_bounds__(
       if (slot_item[ms] < 0) break;
       merge_item(u, warp - (kMathWarps + 2), Shape::kMergeWarps, true, mok);
     }
+    if constexpr (FUSED) phase_c();
     return;
   }
 
@@ -908,42 +950,8 @@ __global__ void __launch_bounds__(
     merge_item(last_it, warp * 32 + lane, kMathThreads, false, ok);
   }
 
-  // ---- single-launch step, phase C: the LSE combine of this CTA's rows by
-  // the math warps, once every math warp of the grid has written its last
-  // partials.  (Split-major items put every row's last split among the last
-  // items, so waiting for the whole grid costs little over waiting per row,
-  // and it takes one fence per warp instead of one per item.)
-  if constexpr (FUSED) {
-    __syncwarp();
-    if (lane == 0) __threadfence();  // this warp's partials are out
-    named_barrier_sync(1, kMathThreads);
-    if (threadIdx.x == 0) {  // one arrival per CTA
-      __threadfence();
-      atomicAdd(f.ctl + 3, 1u);
-      const uint32_t want = gridDim.x;
-      const long long t0 = clock64();
-      while (ld_acquire_gpu(f.ctl + 3) < want) {
-        __nanosleep(64);
-        if (clock64() - t0 > (1ll << 31)) {
-          flag_status(p.status, SEER_DEV_TIMEOUT);
-          break;
-        }
-      }
-    }
-    named_barrier_sync(1, kMathThreads);
-    // one warp per (b, query head) row, spread over every math warp of the grid
-    const int qrows = p.B * p.Hq;
-    for (int q = blockIdx.x * kMathWarps + warp; q < qrows; q += gridDim.x * kMathWarps)
-      combine_row_warp(p.lse_part + (int64_t)q * p.S, p.o_part + (int64_t)q * p.S * kHeadDim,
-                       p.S, f.out + (int64_t)q * kHeadDim,
-                       f.lse_out != nullptr ? f.lse_out + q : nullptr, Load4L2{});
-    // the last CTA through its combine puts the two counters back to zero
-    // (every CTA has passed the wait above by then)
-    if (threadIdx.x == 0 && atomicAdd(f.ctl + 4, 1u) == gridDim.x - 1) {
-      atomicExch(f.ctl + 3, 0u);
-      atomicExch(f.ctl + 4, 0u);
-    }
-  }
+  // ---- single-launch step, phase C (math warps and merge warps)
+  if constexpr (FUSED) phase_c();
 }
 
 // ------------------------------------------------------------------ launcher
