@@ -47,11 +47,23 @@ def measured_peaks():
         return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS}, "fallback"
 
 
+def _code_only(src: str) -> str:
+    """C++ source without its comments and with whitespace collapsed: what
+    the compiler sees, so that a comment edit does not mark the kernel as
+    changed."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def decode_source_hash():
+    """Hash of the decode kernel's code (its source and the two headers it
+    takes its parameters and helpers from), comments and layout ignored."""
     h = hashlib.sha256()
     for name in ("sparse_decode.cu", "seer_common.cuh", "seer_kernels.cuh"):
-        with open(os.path.join(ROOT, "block_sparse_attention_step_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "block_sparse_attention_step_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

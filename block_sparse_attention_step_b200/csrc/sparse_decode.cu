@@ -32,8 +32,8 @@
 //   * at the end of an item each math warp drops its (m, l, O) into a
 //     shared-memory slot (mbarrier-counted) and goes on; two merge warps merge
 //     the item's head rows into o_part / lse_part and free the slot, so the
-//     math warps never stop at item boundaries (the single-launch step and
-//     the one-slot shapes merge in the math warps instead, one item later).
+//     math warps never stop at item boundaries (the one-slot shapes merge in
+//     the math warps instead, one item later).
 // Every mbarrier wait is bounded (SEER_DEV_TIMEOUT); nothing traps.
 #include "gate_row.cuh"
 #include "combine_core.cuh"
