@@ -28,7 +28,9 @@
  *   - Pointers named *_host are host memory; every other pointer is device
  *     memory on the current device.  The caller owns every buffer; the library
  *     never allocates, frees or synchronises, and keeps no state between calls
- *     (it caches one driver entry point on first use).
+ *     besides what it sets up once: the driver entry point of the tensor-map
+ *     encoder, each kernel's shared-memory limit, and the fixed device scratch
+ *     array of seer_decode_step_noalloc.
  *   - bf16 tensors are passed as uint16_t bit patterns.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
  *   - Host-side checks return an error before anything is enqueued.
