@@ -365,6 +365,7 @@ def run_ours(args):
     e2e = end_to_end(runs, args.steps, stream, replicas, w)
     clock_info = clocks.stop() if clocks else None
     status = [int(r.status.item()) for r in runs]
+    recall = gate_recall_stats(run0, probe, w) if args.recall else None
 
     graphs.clear()   # release the graphs before the process group goes
     if world > 1:
@@ -415,10 +416,33 @@ def run_ours(args):
         "clocks": clock_info,
         "device_status": status,
     }
+    if recall is not None:
+        line["gate_recall"] = recall
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, runs[0], args)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def gate_recall_stats(run0, data, w):
+    """Gate recall on replica 0 (outside the timed region): a dense step with
+    the block masses (every block selected) and the sparse step on the same
+    inputs; the share of each (b, query head)'s dense attention mass that the
+    sparse selection keeps."""
+    import torch
+    from block_sparse_attention_step_b200.runner import StepBuffers, gate_recall
+    dense = StepBuffers(w, data, sparsity_permille=0, budget_tokens=0, mass=True)
+    dense.step(update_kbar=2)
+    run0.step(update_kbar=0)
+    torch.cuda.synchronize()
+    v = run0.workspace_views()
+    rec = gate_recall(dense.block_mass, v["idx"], v["n_sel"], w.group).flatten().float()
+    return {"mean": float(rec.mean()), "p10": float(torch.quantile(rec, 0.1)),
+            "min": float(rec.min()),
+            "what": "share of the dense attention mass in the blocks the gate selected, per "
+                    "(sequence, query head) of replica 0 (random-init gate: a capability "
+                    "check, not a quality number)",
+            "device_status": [int(dense.status.item()), int(run0.status.item())]}
 
 
 def prefill_flops(run, w):
@@ -726,6 +750,8 @@ def main(argv=None):
     p.add_argument("--no-graph", action="store_true", help="launch each step directly, no CUDA graph")
     p.add_argument("--mass", action="store_true",
                    help="also emit every block's attention mass (dense-mode gate target)")
+    p.add_argument("--recall", action="store_true",
+                   help="also report the gate recall (dense attention mass kept by the selection)")
     p.add_argument("--unified", action="store_true",
                    help="one block set per sequence shared by all KV heads (cross-head ranking)")
     p.add_argument("--fused", action="store_true",

@@ -15,6 +15,23 @@ import torch
 from . import seer
 
 
+def gate_recall(dense_mass: torch.Tensor, idx: torch.Tensor, n_sel: torch.Tensor,
+                group: int) -> torch.Tensor:
+    """Gate recall per (b, query head): the share of the dense attention
+    distribution that a sparse selection keeps, i.e. the sum over the chosen
+    blocks j of mass[b, qh, j], with `dense_mass` the block masses of a step
+    that selected every block (the self-distilled gate's training target) and
+    `idx` / `n_sel` the selection of the sparse step on the same inputs
+    (query head qh reads the row of KV head qh // group).  An analysis
+    metric over the step's outputs (a gather and a sum), not a step of the
+    path.  Returns [B][Hq] fp32; 1 means the selection holds all the mass."""
+    k_max = idx.shape[-1]
+    live = torch.arange(k_max, device=idx.device)[None, None, :] < n_sel[..., None]
+    j = idx.long().clamp(min=0).repeat_interleave(group, dim=1)       # [B][Hq][k_max]
+    live = live.repeat_interleave(group, dim=1)
+    return (torch.gather(dense_mass, 2, j) * live).sum(-1)
+
+
 class StepBuffers:
     def __init__(self, w, data: dict, num_splits: Optional[int] = None,
                  sparsity_permille: Optional[int] = None, budget_tokens: Optional[int] = None,

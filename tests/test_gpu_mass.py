@@ -115,3 +115,35 @@ def test_decode_item_counter_gives_the_same_bits_and_resets():
     assert run.status.item() == 0
     for o, l in outs:
         assert torch.equal(o, v["o_part"]) and torch.equal(l, v["lse_part"])
+
+
+def test_gate_recall_matches_oracle():
+    """Gate recall (the dense block masses kept by the sparse selection) from
+    the GPU's dense-mass step and sparse step against the oracle's dense
+    block masses summed over the GPU's own selection."""
+    from block_sparse_attention_step_b200.runner import gate_recall
+    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=2, seqlen=2500)
+    data = W.generate(w, 43, DEV)
+    dense = StepBuffers(w, data, sparsity_permille=0, budget_tokens=0, mass=True)
+    dense.step(update_kbar=2)
+    sparse = StepBuffers(w, data)
+    sparse.step(update_kbar=2)
+    torch.cuda.synchronize()
+    assert dense.status.item() == 0 and sparse.status.item() == 0
+    v = sparse.workspace_views()
+    rec = gate_recall(dense.block_mass, v["idx"], v["n_sel"], w.group).cpu().numpy()
+    idx, n_sel = v["idx"].cpu().numpy(), v["n_sel"].cpu().numpy()
+    G = w.group
+    for b in range(w.batch):
+        for h in range(w.kv_heads):
+            q, _, K, _, L = row_inputs(w, data, b, h)
+            allb = np.arange(O.num_blocks(L, w.block_size))
+            ref = O.block_mass(q, K, L, allb, w.block_size, scale_of(w))     # [G][nb]
+            chosen = idx[b, h, :n_sel[b, h]]
+            np.testing.assert_allclose(rec[b, h * G:(h + 1) * G], ref[:, chosen].sum(axis=1),
+                                       atol=1e-4, err_msg=str((b, h)))
+    assert (rec <= 1 + 1e-4).all() and (rec > 0).all()
+    # the dense selection keeps everything
+    dv = dense.workspace_views()
+    full = gate_recall(dense.block_mass, dv["idx"], dv["n_sel"], G)
+    assert torch.allclose(full, torch.ones_like(full), atol=1e-4)

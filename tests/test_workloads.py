@@ -70,3 +70,15 @@ def test_head_major_layout_holds_the_same_values():
             x = W.gather_rows(a["v_pool"], a["page_table"], bb, h, L, 64, "nhd")
             y = W.gather_rows(b["v_pool"], b["page_table"], bb, h, L, 64, "hnd")
             assert torch.equal(x, y)
+
+
+def test_gate_recall_hand_case():
+    """Recall = mass of the chosen blocks, per query head, padding ignored;
+    choosing every block keeps all of a normalised row."""
+    from block_sparse_attention_step_b200.runner import gate_recall
+    m = torch.tensor([[[0.1, 0.2, 0.3, 0.4], [0.25, 0.25, 0.25, 0.25],
+                       [0.7, 0.1, 0.1, 0.1], [0.0, 0.0, 0.5, 0.5]]])      # B 1, Hq 4, NB 4
+    idx = torch.tensor([[[3, 1, -1, -1], [0, 1, 2, 3]]], dtype=torch.int32)  # Hkv 2, G 2
+    n_sel = torch.tensor([[2, 4]], dtype=torch.int32)
+    got = gate_recall(m, idx, n_sel, 2)
+    assert torch.allclose(got, torch.tensor([[0.6, 0.5, 1.0, 1.0]]))
