@@ -332,3 +332,36 @@ def test_step_fused_combine_equals_standalone_combine(name):
     assert run.status.item() == 0
     assert torch.equal(out2, run.out)
     assert torch.equal(lse2, run.lse)
+
+
+@pytest.mark.parametrize("bs", [64, 128])
+def test_step_max_context(bs):
+    """The longest context the library takes: 4096 blocks per sequence (the
+    gate's long-row select path in both gate grids), one sequence exactly full
+    and one with a ragged tail; every row against the oracle, and the single
+    launch gives the per-stage step's bits."""
+    nbm = 4096
+    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(
+        batch=2, q_heads=8, kv_heads=2, block_size=bs, seqlen=None,
+        seqlen_range=(nbm * bs - 37, nbm * bs))
+    data = W.generate(w, 29, DEV)
+    data["seqlens"][0] = nbm * bs
+    run = StepBuffers(w, data)
+    assert run.nb_max == nbm
+    run.pool_full()
+    kbar0 = run.kbar.clone()
+    run.step(update_kbar=1)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    report = {"exact": 0, "near_tie": 0}
+    check_rows(w, data, run, [(b, h) for b in range(w.batch) for h in range(w.kv_heads)], report)
+    v = run.workspace_views()
+    ref = [t.clone() for t in (run.kbar, v["scores"], v["idx"], v["n_sel"], run.out, run.lse)]
+    run.kbar.copy_(kbar0)
+    run.step(update_kbar=1, fused=True)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    v = run.workspace_views()
+    got = (run.kbar, v["scores"], v["idx"], v["n_sel"], run.out, run.lse)
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
