@@ -472,6 +472,49 @@ def prefill_flops(run, w):
     return 4 * w.head_dim * G * total
 
 
+def prefill_cpu_baseline(w, data, q, args):
+    """The fp64 oracle's prefill (pooled keys, pooled-query gate, per-block
+    selection, causal block-sparse attention) timed on (b, h) rows of the
+    same inputs until the CPU budget runs out, scaled to the whole batch."""
+    import random
+    import numpy as np
+    from block_sparse_attention_step_b200 import workloads as W
+    from oracle import seer_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    rows = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    random.Random(0).shuffle(rows)
+    G, bs = w.group, w.block_size
+    scale = 1.0 / math.sqrt(w.head_dim)
+    if w.budget_tokens:
+        k_of = lambda i: O.k_from_budget(i + 1, w.budget_tokens, bs)
+    else:
+        k_of = lambda i: O.k_from_sparsity(i + 1, w.sparsity_permille)
+    spent, done = 0.0, 0
+    for (b, h) in rows:
+        L = int(data["seqlens"][b])
+        Qg = q[b, :L, h * G:(h + 1) * G].double().cpu().numpy()
+        Wg = data["w_gate"][h].double().cpu().numpy()
+        K = W.gather_rows(data["k_pool"], data["page_table"], b, h, L, bs).double().numpy()
+        V = W.gather_rows(data["v_pool"], data["page_table"], b, h, L, bs).double().numpy()
+        t0 = time.perf_counter()
+        O.prefill_row(Qg, Wg, K, V, L, bs, k_of, scale, scale)
+        spent += time.perf_counter() - t0
+        done += 1
+        if spent >= args.cpu_budget:
+            break
+    sec_row = spent / max(done, 1)
+    tokens = int(data["seqlens"].sum())
+    return {"value": tokens / (sec_row * len(rows)), "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{done} of {len(rows)} (b, kv-head) rows of this prompt batch, fp64 numpy "
+                      f"oracle prefill (pooled keys, pooled-query gate, selection, causal "
+                      f"attention), {sec_row:.1f} s/row, scaled to the whole batch"}
+
+
 def run_prefill(args):
     """Prefill with query pooling on the headline shapes at batch 2 and a
     16K-token prompt: one JSON line (prompt tokens/s, tensor roofline)."""
@@ -533,6 +576,8 @@ def run_prefill(args):
         "clocks": clock_info,
         "device_status": [int(r.status.item()) for r in runs],
     }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_cpu_baseline(w, runs[0].data, runs[0].q, args)
     print(json.dumps(line), flush=True)
     return 0
 
