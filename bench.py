@@ -274,15 +274,7 @@ def run_ours(args):
     # replicas: enough that one rotation reads > 4x L2
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
     probe = W.generate(w, args.seed + 1000 * rank, dev, layout=args.layout)
-    k_cap = None
-    if w.seqlen_range is not None:
-        # the other replicas draw other lengths: size the index rows for the
-        # longest sequence the workload allows, so that no replica's k is clamped
-        nb = -(-w.seqlen_range[1] // w.block_size)
-        k_cap = (seer.seer_k_from_budget(nb, w.budget_tokens, w.block_size) if w.budget_tokens
-                 else seer.seer_k_from_sparsity(nb, w.sparsity_permille))
-    run0 = StepBuffers(w, probe, num_splits=args.splits, k_max=k_cap, mass=args.mass,
-                       unified=args.unified)
+    run0 = StepBuffers(w, probe, num_splits=args.splits, mass=args.mass, unified=args.unified)
     run0.pool_full()
     torch.cuda.synchronize()
     sel_bytes, sel_tokens = selected_bytes(run0, probe, w)
@@ -293,8 +285,9 @@ def run_ours(args):
     runs = [run0]
     for r in range(1, replicas):
         d = W.generate(w, args.seed + 1000 * rank + r, dev, layout=args.layout)
-        rr = StepBuffers(w, d, num_splits=run0.num_splits, k_max=run0.k_max, mass=args.mass,
-                         unified=args.unified)
+        # each replica sizes its index rows for its own sequences (ragged
+        # replicas draw other lengths, so a shared k_max could clamp their k)
+        rr = StepBuffers(w, d, num_splits=run0.num_splits, mass=args.mass, unified=args.unified)
         rr.pool_full()
         runs.append(rr)
     step_args = [r.args(update_kbar=1) for r in runs]
