@@ -87,88 +87,326 @@ def recorded_traffic(workload):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled every 50 ms while the
+    measurements run, through read-only NVML queries in a thread (nothing is
+    set).  Falls back to ``nvidia-smi -lms 50 -f <file>`` (the tool writes
+    each sample to the file itself, so nothing is lost when it is stopped)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    LOADED_W = 200.0    # power draw above which a sample counts as "under load"
 
-    def __init__(self, device_index):
-        self.proc = None
+    def __init__(self, device_index, period_s=0.05):
+        import threading
+        self.samples = []          # (sm_mhz, sm_max_mhz, power_w, frozenset(reasons))
+        self.source = None
+        self.proc = self.path = None
+        self._stop = threading.Event()
+        self._thread = None
+        uuid = None
         try:
             import torch
-            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            u = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = u if u.startswith("GPU-") else f"GPU-{u}"
         except Exception:
-            target = str(device_index)
+            pass
         try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = (nv.nvmlDeviceGetHandleByUUID(uuid) if uuid else
+                 nv.nvmlDeviceGetHandleByIndex(int(device_index)))
+            smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((sm, smax, pw,
+                                             frozenset(k for k, b in bits.items() if r & b)))
+                    except Exception:
+                        pass
+                    self._stop.wait(period_s)
+            self._thread = threading.Thread(target=loop, daemon=True)
+            self._thread.start()
+            self.source = "nvml"
+            return
+        except Exception:
+            pass
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50", "-i", target], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                text=True)
+                 "-lms", str(int(period_s * 1000)), "-i", uuid or str(device_index),
+                 "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi"
         except OSError:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
+    def _read_smi_file(self):
         try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, loaded, reasons = [], [], [], set()
-        for line in out.strip().splitlines():
+            text = open(self.path).read()
+        except OSError:
+            return
+        for line in text.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                s, m, pw = float(parts[1]), float(parts[2]), float(parts[3])
+                sm, m, pw = float(parts[1]), float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            sm.append(s)
-            smax.append(m)
-            if pw > 200:          # under load
-                loaded.append(s)
-            for name, val in zip(self.NAMES, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
+            self.samples.append((sm, m, pw, frozenset(
+                n for n, v in zip(self.NAMES, parts[5:9]) if v.lower() == "active")))
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.proc.wait()
+            self._read_smi_file()
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"],
+                    "samples": 0}
+        return self.summary(self.samples, self.source)
+
+    @classmethod
+    def summary(cls, samples, source):
+        sm = [s[0] for s in samples]
+        loaded = [s[0] for s in samples if s[2] > cls.LOADED_W]
+        reasons = set()
+        for s in samples:
+            reasons |= s[3]
         use = loaded or sm
         return {"sm_mhz": statistics.median(use) if use else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
+                "sm_max_mhz": max(s[1] for s in samples) if samples else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "samples_under_load": len(loaded),
+                "power_w_max": max((s[2] for s in samples), default=None),
+                "source": source}
 
 
 # ------------------------------------------------------------------ CPU oracle
+#
+# The oracle is timed in parallel over the host cores: one spawned process
+# per core, each held to one BLAS thread, each owning a share of the (b, h)
+# rows balanced by sequence length.  A row's inputs reach its process once,
+# as raw bf16 bits (q, K, V) and fp32 (W), before any timing; a timed pass
+# then runs the oracle's whole step on every row -- the exact bf16 -> fp64
+# conversion, pooled keys, gate scores, selection and masked attention (or
+# the prefill path) -- and the pass's wall time is the slowest process's.
 
-def oracle_rows_timed(w, data, rows, budget_s, k_per_seq, force_newest):
-    """Time the fp64 oracle's whole step on (b, h) rows, one after another,
-    until the row list or the time budget runs out.  Returns (seconds per
-    row, rows timed, threads)."""
+
+def _oracle_run_row(O, np, r):
+    """The oracle's step on one row from its raw inputs (timed part)."""
+    q = O.bf16_bits_to_f64(r["q"])
+    Wg = np.asarray(r["W"], dtype=np.float64)
+    K = O.bf16_bits_to_f64(r["K"])
+    V = O.bf16_bits_to_f64(r["V"])
+    if r["kind"] == "decode":
+        return O.decode_row(q, Wg, K, V, r["L"], r["bs"], r["k"], r["force"], r["scale"],
+                            r["scale"])
+    bs = r["bs"]
+    if r["budget"]:
+        k_of = lambda i: O.k_from_budget(i + 1, r["budget"], bs)
+    else:
+        k_of = lambda i: O.k_from_sparsity(i + 1, r["permille"])
+    return O.prefill_row(q, Wg, K, V, r["L"], bs, k_of, r["scale"], r["scale"])
+
+
+def _oracle_worker(conn):
+    """One host core's share of the oracle step (a spawned process).  Its
+    BLAS is held to one thread: the variables are read when numpy loads its
+    BLAS, which happens here, after they are set."""
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS",
+                "BLIS_NUM_THREADS", "NUMEXPR_NUM_THREADS"):
+        os.environ[var] = "1"
     import numpy as np
-    from block_sparse_attention_step_b200 import workloads as W
-    from oracle import seer_oracle as O
     try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = 1
-    scale = 1.0 / math.sqrt(w.head_dim)
-    G = w.group
-    spent, done = 0.0, 0
-    for (b, h) in rows:
-        L = int(data["seqlens"][b])
-        q = data["q"][b, h * G:(h + 1) * G].double().cpu().numpy()
-        Wg = data["w_gate"][h].double().cpu().numpy()
-        K = W.gather_rows(data["k_pool"], data["page_table"], b, h, L, w.block_size, data.get("layout", "nhd")).double().numpy()
-        V = W.gather_rows(data["v_pool"], data["page_table"], b, h, L, w.block_size, data.get("layout", "nhd")).double().numpy()
-        t0 = time.perf_counter()
-        O.decode_row(q, Wg, K, V, L, w.block_size, int(k_per_seq[b]), force_newest, scale, scale)
-        spent += time.perf_counter() - t0
-        done += 1
-        if spent >= budget_s:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except ImportError:
+        pass
+    from oracle import seer_oracle as O
+    rows = conn.recv()
+    while True:
+        cmd = conn.recv()
+        if cmd == "run":
+            t0 = time.perf_counter()
+            for r in rows:
+                _oracle_run_row(O, np, r)
+            conn.send(time.perf_counter() - t0)
+        elif cmd == "results":
+            conn.send([_oracle_run_row(O, np, r) for r in rows])
+        else:
             break
-    return spent / max(done, 1), done, threads
+    conn.close()
+
+
+def host_cpu_info():
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count() or 1
+    return {"nproc": os.cpu_count(), "usable_cores": usable, "cpu_model": model}
+
+
+class OraclePool:
+    """Spawned oracle processes (spawn, so that none inherits a CUDA
+    context), each with its share of rows; ``step()`` times one parallel pass
+    over all of them."""
+
+    def __init__(self, workers: int):
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
+        self.conns, self.procs = [], []
+        for _ in range(max(1, int(workers))):
+            a, b = ctx.Pipe()
+            proc = ctx.Process(target=_oracle_worker, args=(b,), daemon=True)
+            proc.start()
+            self.conns.append(a)
+            self.procs.append(proc)
+        self.order = []
+
+    def load(self, rows, cost):
+        """Deal the rows out, longest first, each to the least-loaded process."""
+        n = len(self.conns)
+        load = [0.0] * n
+        share = [[] for _ in range(n)]
+        self.order = [[] for _ in range(n)]
+        for i in sorted(range(len(rows)), key=lambda i: -cost[i]):
+            j = min(range(n), key=lambda j: load[j])
+            load[j] += cost[i]
+            share[j].append(rows[i])
+            self.order[j].append(i)
+        for c, part in zip(self.conns, share):
+            c.send(part)
+
+    def step(self) -> float:
+        t0 = time.perf_counter()
+        for c in self.conns:
+            c.send("run")
+        for c in self.conns:
+            c.recv()
+        return time.perf_counter() - t0
+
+    def results(self):
+        """The oracle's outputs per row, in the order the rows were loaded."""
+        for c in self.conns:
+            c.send("results")
+        out = {}
+        for c, idx in zip(self.conns, self.order):
+            for i, r in zip(idx, c.recv()):
+                out[i] = r
+        return [out[i] for i in range(len(out))]
+
+    def close(self):
+        for c in self.conns:
+            try:
+                c.send("stop")
+            except (OSError, BrokenPipeError):
+                pass
+        for proc in self.procs:
+            proc.join(timeout=10)
+            if proc.is_alive():
+                proc.kill()
+
+
+def _bits(t):
+    import torch
+    return t.contiguous().view(torch.int16).cpu().numpy().view("uint16")
+
+
+def oracle_decode_rows(w, data, rows, k_per_seq, force_newest):
+    """Raw per-row inputs of the oracle's decode step (host copies, not timed)."""
+    from block_sparse_attention_step_b200 import workloads as W
+    G, bs = w.group, w.block_size
+    layout = data.get("layout", "nhd")
+    q = _bits(data["q"])
+    wg = data["w_gate"].cpu().numpy()
+    L_all = data["seqlens"].cpu().tolist()
+    out = []
+    for (b, h) in rows:
+        L = int(L_all[b])
+        out.append({"kind": "decode", "q": q[b, h * G:(h + 1) * G], "W": wg[h],
+                    "K": _bits(W.gather_rows(data["k_pool"], data["page_table"], b, h, L, bs,
+                                             layout)),
+                    "V": _bits(W.gather_rows(data["v_pool"], data["page_table"], b, h, L, bs,
+                                             layout)),
+                    "L": L, "bs": bs, "k": int(k_per_seq[b]), "force": bool(force_newest),
+                    "scale": 1.0 / math.sqrt(w.head_dim)})
+    return out
+
+
+def pick_rows(w, seqlens, max_bytes):
+    """Every (b, h) row when their inputs fit in ``max_bytes`` of host
+    copies, else the longest-first sample of rows that does (each row ships
+    its K and V, L x D x 2 bytes each)."""
+    rows = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    per = lambda r: 4 * w.head_dim * int(seqlens[r[0]])
+    if sum(per(r) for r in rows) <= max_bytes:
+        return rows, False
+    import random
+    rng = random.Random(0)
+    rng.shuffle(rows)
+    pick, total = [], 0
+    for r in rows:
+        if total + per(r) > max_bytes and pick:
+            continue
+        pick.append(r)
+        total += per(r)
+    return sorted(pick), True
+
+
+def oracle_parallel_timing(w, data, k_per_seq, force_newest, rows, workers, steps,
+                           warmup=1, budget_s=None):
+    """Mean wall time of one parallel oracle pass over ``rows`` (after
+    ``warmup`` passes), with the pool's processes and the rows' lengths."""
+    seqlens = data["seqlens"].cpu().tolist()
+    inputs = oracle_decode_rows(w, data, rows, k_per_seq, force_newest)
+    pool = OraclePool(min(workers, len(rows)))
+    try:
+        pool.load(inputs, [float(seqlens[b]) for (b, _) in rows])
+        del inputs
+        for _ in range(warmup):
+            pool.step()
+        times = []
+        spent = 0.0
+        for _ in range(steps):
+            t = pool.step()
+            times.append(t)
+            spent += t
+            if budget_s is not None and spent >= budget_s and len(times) >= 1:
+                break
+        return times, len(pool.conns)
+    finally:
+        pool.close()
 
 
 def cpu_k_per_seq(w, seqlens):
@@ -183,68 +421,124 @@ def cpu_k_per_seq(w, seqlens):
     return out
 
 
+def row_share(w, seqlens, rows):
+    """The whole batch's oracle work over the sample's: by row count for
+    fixed lengths, by total length (the oracle's cost grows with L) for a
+    ragged batch."""
+    all_l = sum(int(seqlens[b]) for b in range(w.batch)) * w.kv_heads
+    got = sum(int(seqlens[b]) for (b, _) in rows)
+    return all_l / max(got, 1)
+
+
 def run_reference(args):
-    """The oracle alone on the host cores: each step is a bounded sample of
-    the workload's (b, h) rows, scaled to tokens/s of the whole batch."""
+    """The oracle alone on the host cores, on the same workload draw and the
+    same rows as the CPU baseline of the GPU arm: each step is one parallel
+    pass of the oracle's whole step over every (b, h) row of the batch (a
+    longest-first sample of rows for batches whose inputs exceed the host
+    copy budget, scaled by total length and marked as extrapolated)."""
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     import torch
     from block_sparse_attention_step_b200 import workloads as W
-    w = W.WORKLOADS[args.workload]
-    # rows of a batch-1 draw have the workload's per-row shape (L, G, bs, k)
-    one = w.replace(batch=1) if w.seqlen_range is None else w.replace(batch=2)
-    data = W.generate(one, args.seed, "cpu")
-    kps = cpu_k_per_seq(one, data["seqlens"].tolist())
-    rows = [(b, h) for b in range(one.batch) for h in range(one.kv_heads)]
-    per_step = max(1, min(len(rows), args.ref_rows))
-    times = []
-    for i in range(args.warmup + args.steps):
-        sample = [rows[(i * per_step + r) % len(rows)] for r in range(per_step)]
-        sec, n, threads = oracle_rows_timed(one, data, sample, 1e9, kps, w.force_newest)
-        if i >= args.warmup:
-            times.append(sec)
-    sec_row = sum(times) / len(times)
-    if w.seqlen_range is not None:
-        sec_row *= _ragged_row_scale(w, data)
-    step_s = sec_row * w.batch * w.kv_heads
+    w = resolve_workload(args)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    data = W.generate(w, args.seed if args.seed is not None else w.seed, dev)
+    seqlens = data["seqlens"].cpu().tolist()
+    kps = cpu_k_per_seq(w, seqlens)
+    rows, sampled = pick_rows(w, seqlens, args.cpu_max_bytes)
+    info = host_cpu_info()
+    workers = info["usable_cores"]
+    inputs = oracle_decode_rows(w, data, rows, kps, w.force_newest)
+    pool = OraclePool(min(workers, len(rows)))
+    try:
+        pool.load(inputs, [float(seqlens[b]) for (b, _) in rows])
+        del inputs
+        # the selection the oracle makes (for the config's byte count), untimed
+        res = pool.results()
+        for _ in range(args.warmup):
+            pool.step()
+        times = [pool.step() for _ in range(args.steps)]
+        used = len(pool.conns)
+    finally:
+        pool.close()
+    scale = row_share(w, seqlens, rows)
+    step_s = statistics.mean(times) * scale
     value = w.batch / step_s
+    sel_tokens = 0
+    for (b, _), r in zip(rows, res):
+        L = int(seqlens[b])
+        sel_tokens += sum(min(w.block_size, L - int(j) * w.block_size) for j in r["indices"])
+    sel_bytes = int(round(sel_tokens * scale)) * w.head_dim * 4
+    kbar_bytes = w.batch * w.kv_heads * data["nb_max"] * w.head_dim * 4
+    k_max = max(1, min(max(kps), data["nb_max"]))
+    cfg = workload_config(w, reference_splits(w, data, k_max), k_max,
+                          replica_count(sel_bytes + kbar_bytes, dev, args.max_replicas),
+                          args.layout, args)
+    sample = (f"{'a longest-first sample of ' if sampled else 'all '}{len(rows)} (b, kv-head) "
+              f"rows of this workload draw (seed {args.seed if args.seed is not None else w.seed})"
+              f" per step, fp64 numpy oracle (bf16->f64, pool, gate, select, masked attention), "
+              f"{used} spawned processes with one BLAS thread each"
+              + (f", scaled x{scale:.2f} by total length to the whole batch" if sampled else ""))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w, None),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"{per_step} (b, kv-head) rows of a batch-{one.batch} draw per "
-                                   f"step, fp64 numpy oracle, scaled to {w.batch}x{w.kv_heads} rows"},
+        "data": "synthetic (seeded; random-init gate projection)", "config": cfg,
+        "extrapolated": bool(sampled), "rows_per_step": len(rows),
+        "cpu_baseline": dict({"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                              "sample": sample}, **info),
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def _ragged_row_scale(w, data):
-    """Oracle cost grows with L: scale the sampled rows' mean length to the
-    workload's expected mean length."""
-    lo, hi = w.seqlen_range
-    sampled = float(data["seqlens"].double().mean())
-    return ((lo + hi) / 2.0) / sampled
+def resolve_workload(args):
+    from block_sparse_attention_step_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    if args.sparsity is not None:
+        w = w.replace(sparsity_permille=args.sparsity, budget_tokens=None)
+    return w
 
 
-def workload_config(w, run, replicas=None, touched=None, layout=None):
+def replica_count(touched, dev, max_replicas):
+    """Replicas whose rotation reads more than 4x the L2 (at least 2)."""
+    l2 = 126 * 1024 * 1024
+    if str(dev).startswith("cuda"):
+        import torch
+        l2 = torch.cuda.get_device_properties(torch.device(dev)).L2_cache_size
+    return min(max(2, math.ceil(4 * l2 / max(touched, 1))), max_replicas), touched
+
+
+def reference_splits(w, data, k_max):
+    """The split count the GPU arm launches with on this workload (a host
+    helper of the library: no device work), so both lines name one config."""
+    if w.num_splits:
+        return w.num_splits
+    from block_sparse_attention_step_b200 import seer
+    d = seer.make_dims(w.batch, w.q_heads, w.kv_heads, w.head_dim, w.block_size,
+                       data["nb_max"], data["num_pages"])
+    return seer.seer_default_splits(d, k_max, 0)
+
+
+def workload_config(w, num_splits, k_max, rep, layout, args):
+    """The config object both arms print (the same keys and values for the
+    same workload, split count and selection size)."""
+    replicas, touched = rep
     cfg = {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
            "head_dim": w.head_dim, "block_size": w.block_size,
            "seq_len": w.seqlen if w.seqlen else f"U[{w.seqlen_range[0]},{w.seqlen_range[1]}]",
            "selection": (f"budget {w.budget_tokens} tokens" if w.budget_tokens
                          else f"sparsity {w.sparsity_permille / 10:g}%"),
-           "force_newest": w.force_newest, "paged": w.paged}
-    if layout is not None:
-        cfg["kv_layout"] = layout
-    if run is not None:
-        cfg["num_splits"] = run.num_splits
-        cfg["k_max"] = run.k_max
-    if replicas is not None:
-        cfg["l2"] = (f"inputs larger than L2: {replicas} rotating replicas, "
-                     f"{touched / 1e6:.0f} MB read per step, L2 126 MB")
+           "force_newest": w.force_newest, "paged": w.paged, "kv_layout": layout,
+           "num_splits": int(num_splits), "k_max": int(k_max),
+           "l2": (f"inputs larger than L2: {replicas} rotating replicas, "
+                  f"{touched / 1e6:.0f} MB read per step, L2 126 MB"),
+           "block_mass": bool(args.mass),
+           "selection_scope": ("one block set per sequence (all KV heads)" if args.unified
+                               else "per KV head"),
+           "step_launch": ("single cooperative launch" if args.fused
+                           else "per stage, PDL-chained")}
     return cfg
 
 
@@ -267,24 +561,22 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     seer.library()
-    w = W.WORKLOADS[args.workload]
-    if args.sparsity is not None:
-        w = w.replace(sparsity_permille=args.sparsity, budget_tokens=None)
+    w = resolve_workload(args)
+    seed0 = (args.seed if args.seed is not None else w.seed) + 1000 * rank
 
     # replicas: enough that one rotation reads > 4x L2
-    l2 = torch.cuda.get_device_properties(local).L2_cache_size
-    probe = W.generate(w, args.seed + 1000 * rank, dev, layout=args.layout)
+    probe = W.generate(w, seed0, dev, layout=args.layout)
     run0 = StepBuffers(w, probe, num_splits=args.splits, mass=args.mass, unified=args.unified)
     run0.pool_full()
     torch.cuda.synchronize()
     sel_bytes, sel_tokens = selected_bytes(run0, probe, w)
     kbar_bytes = run0.kbar.numel() * 4
     touched = sel_bytes + kbar_bytes
-    replicas = max(2, math.ceil(4 * l2 / max(touched, 1)))
-    replicas = min(replicas, args.max_replicas)
+    rep = replica_count(touched, dev, args.max_replicas)
+    replicas = rep[0]
     runs = [run0]
     for r in range(1, replicas):
-        d = W.generate(w, args.seed + 1000 * rank + r, dev, layout=args.layout)
+        d = W.generate(w, seed0 + r, dev, layout=args.layout)
         # each replica sizes its index rows for its own sequences (ragged
         # replicas draw other lengths, so a shared k_max could clamp their k)
         rr = StepBuffers(w, d, num_splits=run0.num_splits, mass=args.mass, unified=args.unified)
@@ -384,12 +676,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; random-init gate projection)",
-        "config": dict(workload_config(w, run0, replicas, touched, args.layout),
-                       block_mass=bool(args.mass),
-                       selection_scope="one block set per sequence (all KV heads)"
-                       if args.unified else "per KV head",
-                       step_launch="single cooperative launch" if args.fused
-                       else "per stage, PDL-chained"),
+        "config": workload_config(w, run0.num_splits, run0.k_max, rep, args.layout, args),
         "selected_kv_bytes_per_step": sel_bytes,
         "selected_tokens_per_step": sel_tokens,
         "step_hbm_gbs": (touched / (ms_step * 1e-3)) / 1e9,
@@ -412,7 +699,7 @@ def run_ours(args):
     if recall is not None:
         line["gate_recall"] = recall
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, runs[0], args)
+        line["cpu_baseline"] = cpu_baseline(w, runs[0].data, args, seed0)
     print(json.dumps(line), flush=True)
     return 0
 
@@ -467,45 +754,38 @@ def prefill_flops(run, w):
 
 def prefill_cpu_baseline(w, data, q, args):
     """The fp64 oracle's prefill (pooled keys, pooled-query gate, per-block
-    selection, causal block-sparse attention) timed on (b, h) rows of the
-    same inputs until the CPU budget runs out, scaled to the whole batch."""
-    import random
-    import numpy as np
+    selection, causal block-sparse attention) on every (b, h) row of the
+    prompt batch, one spawned process per usable core with one BLAS thread
+    each, one timed parallel pass."""
     from block_sparse_attention_step_b200 import workloads as W
-    from oracle import seer_oracle as O
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = 1
     rows = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
-    random.Random(0).shuffle(rows)
     G, bs = w.group, w.block_size
-    scale = 1.0 / math.sqrt(w.head_dim)
-    if w.budget_tokens:
-        k_of = lambda i: O.k_from_budget(i + 1, w.budget_tokens, bs)
-    else:
-        k_of = lambda i: O.k_from_sparsity(i + 1, w.sparsity_permille)
-    spent, done = 0.0, 0
+    info = host_cpu_info()
+    seqlens = data["seqlens"].cpu().tolist()
+    wg = data["w_gate"].cpu().numpy()
+    inputs = []
     for (b, h) in rows:
-        L = int(data["seqlens"][b])
-        Qg = q[b, :L, h * G:(h + 1) * G].double().cpu().numpy()
-        Wg = data["w_gate"][h].double().cpu().numpy()
-        K = W.gather_rows(data["k_pool"], data["page_table"], b, h, L, bs).double().numpy()
-        V = W.gather_rows(data["v_pool"], data["page_table"], b, h, L, bs).double().numpy()
-        t0 = time.perf_counter()
-        O.prefill_row(Qg, Wg, K, V, L, bs, k_of, scale, scale)
-        spent += time.perf_counter() - t0
-        done += 1
-        if spent >= args.cpu_budget:
-            break
-    sec_row = spent / max(done, 1)
-    tokens = int(data["seqlens"].sum())
-    return {"value": tokens / (sec_row * len(rows)), "unit": "tokens/s", "cores": threads,
-            "kind": "oracle",
-            "sample": f"{done} of {len(rows)} (b, kv-head) rows of this prompt batch, fp64 numpy "
-                      f"oracle prefill (pooled keys, pooled-query gate, selection, causal "
-                      f"attention), {sec_row:.1f} s/row, scaled to the whole batch"}
+        L = int(seqlens[b])
+        inputs.append({"kind": "prefill", "q": _bits(q[b, :L, h * G:(h + 1) * G]), "W": wg[h],
+                       "K": _bits(W.gather_rows(data["k_pool"], data["page_table"], b, h, L, bs)),
+                       "V": _bits(W.gather_rows(data["v_pool"], data["page_table"], b, h, L, bs)),
+                       "L": L, "bs": bs, "budget": w.budget_tokens or 0,
+                       "permille": w.sparsity_permille or 0,
+                       "scale": 1.0 / math.sqrt(w.head_dim)})
+    pool = OraclePool(min(info["usable_cores"], len(rows)))
+    try:
+        pool.load(inputs, [float(seqlens[b]) for (b, _) in rows])
+        del inputs
+        t = pool.step()
+        used = len(pool.conns)
+    finally:
+        pool.close()
+    tokens = int(sum(seqlens))
+    return dict({"value": tokens / t, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                 "sample": f"all {len(rows)} (b, kv-head) rows of this prompt batch in one "
+                           f"parallel pass ({t:.1f} s), fp64 numpy oracle prefill (pooled keys, "
+                           f"pooled-query gate, selection, causal attention), {used} spawned "
+                           f"processes with one BLAS thread each"}, **info)
 
 
 def run_prefill(args):
@@ -521,8 +801,9 @@ def run_prefill(args):
         w = w.replace(sparsity_permille=args.sparsity)
     runs = []
     for r in range(2):
-        data = W.generate(w, args.seed + r, dev)
-        q = W.prefill_queries(w, args.seed + r, data["nb_max"], dev)
+        seed = (args.seed if args.seed is not None else w.seed) + r
+        data = W.generate(w, seed, dev)
+        q = W.prefill_queries(w, seed, data["nb_max"], dev)
         pr = PrefillBuffers(w, data, q)
         pr.run(pool_keys=True)
         runs.append(pr)
@@ -745,26 +1026,35 @@ def end_to_end(runs, steps, stream, replicas, w):
             "path": f"seer_decode_step_host: {how}; device-timed"}
 
 
-def cpu_baseline(w, run, args):
-    rows = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
-    import random
-    random.Random(0).shuffle(rows)
-    k = run.k_per_seq.cpu().tolist()
-    sec_row, n, threads = oracle_rows_timed(w, run.data, rows, args.cpu_budget, k, run.force_newest)
-    step_s = sec_row * len(rows)
-    out = {"value": w.batch / step_s, "unit": UNIT, "cores": threads, "kind": "oracle",
-           "sample": f"{n} of {len(rows)} (b, kv-head) rows of this workload, fp64 numpy oracle "
-                     f"(pool, gate, select, masked attention), {sec_row * 1e3:.1f} ms/row, scaled "
-                     f"to the whole batch"}
-    try:  # the same oracle held to one BLAS thread, on a shorter sample
-        from threadpoolctl import threadpool_limits
-        with threadpool_limits(limits=1):
-            sec1, n1, _ = oracle_rows_timed(w, run.data, rows, args.cpu_budget / 3, k,
-                                            run.force_newest)
-        out["value_1core"] = w.batch / (sec1 * len(rows))
-        out["sample_1core"] = f"{n1} rows, one BLAS thread, {sec1 * 1e3:.1f} ms/row"
-    except ImportError:
-        pass
+def cpu_baseline(w, data, args, seed):
+    """The oracle on the host cores, on replica 0's draw (the reference arm's
+    draw): every (b, h) row of the batch per parallel pass where the inputs
+    fit the host copy budget, one spawned process per usable core with one
+    BLAS thread each; then the same oracle on one core over a few rows."""
+    seqlens = data["seqlens"].cpu().tolist()
+    kps = cpu_k_per_seq(w, seqlens)
+    info = host_cpu_info()
+    rows, sampled = pick_rows(w, seqlens, args.cpu_max_bytes)
+    times, used = oracle_parallel_timing(w, data, kps, w.force_newest, rows,
+                                         info["usable_cores"], steps=5, warmup=1,
+                                         budget_s=args.cpu_budget)
+    step_s = statistics.mean(times) * row_share(w, seqlens, rows)
+    out = dict({"value": w.batch / step_s, "unit": UNIT, "cores": used, "kind": "oracle",
+                "sample": (f"{'a longest-first sample of ' if sampled else 'all '}{len(rows)} "
+                           f"(b, kv-head) rows of this workload draw (seed {seed}) per pass, "
+                           f"{len(times)} timed passes, fp64 numpy oracle (bf16->f64, pool, "
+                           f"gate, select, masked attention), {used} spawned processes with "
+                           f"one BLAS thread each"
+                           + (", scaled by total length to the whole batch" if sampled else "")),
+                "ms_per_step": step_s * 1e3, "extrapolated": bool(sampled)}, **info)
+    # one core: the longest rows that make about a tenth of the batch
+    few = sorted(rows, key=lambda r: -int(seqlens[r[0]]))[:max(1, len(rows) // 10)]
+    t1, _ = oracle_parallel_timing(w, data, kps, w.force_newest, few, 1, steps=2, warmup=1)
+    step1 = statistics.mean(t1) * row_share(w, seqlens, few)
+    out["value_1core"] = w.batch / step1
+    out["sample_1core"] = (f"{len(few)} rows in one process with one BLAS thread, "
+                           f"{statistics.mean(t1) / len(few) * 1e3:.1f} ms/row, scaled by total "
+                           f"length to the whole batch")
     return out
 
 
@@ -780,10 +1070,13 @@ def main(argv=None):
     p.add_argument("--splits", type=int, default=None)
     p.add_argument("--layout", choices=("nhd", "hnd"), default="nhd",
                    help="KV pool page layout: token-major [P][bs][Hkv][D] or head-major [P][Hkv][bs][D]")
-    p.add_argument("--seed", type=int, default=1)
+    p.add_argument("--seed", type=int, default=None,
+                   help="seed of replica 0 (default: the workload's recorded seed)")
     p.add_argument("--max-replicas", type=int, default=8)
-    p.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time")
-    p.add_argument("--ref-rows", type=int, default=4, help="oracle rows per reference step")
+    p.add_argument("--cpu-budget", type=float, default=15.0,
+                   help="seconds of timed oracle passes for the CPU baseline (at least one)")
+    p.add_argument("--cpu-max-bytes", type=float, default=4e9,
+                   help="host bytes of oracle inputs (K and V rows); a batch above it is sampled")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", action="store_true", help="launch each step directly, no CUDA graph")
     p.add_argument("--mass", action="store_true",

@@ -1,9 +1,11 @@
 // C ABI of libseer: argument checks, launch geometry, tensor maps and the
 // fused step.  Declared in include/seer.h.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <climits>
+#include <cstdlib>
 #include <mutex>
 
 #include "seer_kernels.cuh"
@@ -13,6 +15,29 @@ using namespace seer;
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// NVTX ranges around each step and each stage it enqueues, for profilers
+// (ncu --nvtx-include, nsys): compiled in, off unless the environment has
+// SEER_NVTX=1 when the library first checks (a host-side push/pop only).
+bool nvtx_on() {
+  static const bool on = [] {
+    const char* v = std::getenv("SEER_NVTX");
+    return v != nullptr && v[0] == '1';
+  }();
+  return on;
+}
+
+struct NvtxRange {
+  const bool on;
+  explicit NvtxRange(const char* name) : on(nvtx_on()) {
+    if (on) nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (on) nvtxRangePop();
+  }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -478,6 +503,7 @@ seer_status seer_combine(const seer_dims* d, const float* o_part, const float* l
 static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
                                     seer_stream stream, const uint16_t* q_mapped,
                                     uint16_t* out_mapped) {
+  NvtxRange step_range("seer_decode_step");
   SEER_TRY(check_dims(d));
   if (a == nullptr || a->k_per_seq == nullptr || a->kbar == nullptr) return SEER_ERR_INVALID_ARG;
   if (a->update_kbar < 0 || a->update_kbar > 2) return SEER_ERR_INVALID_ARG;
@@ -499,9 +525,11 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
   if (mass && (!a->block_mass || !a->block_lse || !a->lse_out)) return SEER_ERR_INVALID_ARG;
   L.p.block_lse = mass ? a->block_lse : nullptr;
 
-  if (a->update_kbar == 2)
+  if (a->update_kbar == 2) {
+    NvtxRange r("pool_keys (full rebuild)");
     SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
                             stream));
+  }
   // a0 (incremental) + a1 + a2 in one kernel; same results as the three calls
   GateSelectParams g = {};
   g.q = q_mapped != nullptr ? q_mapped : a->q;
@@ -540,12 +568,15 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
   g.B = d->batch;
   g.row_counter = w.work_counter + 5;
   const int num_sms = num_sms_current();
-  if ((int64_t)d->batch * d->num_kv_heads > num_sms) {
-    // more rows than SMs: persistent row-claiming gate (its counter starts at 0)
-    SEER_CUDA(cudaMemsetAsync(g.row_counter, 0, sizeof(uint32_t), stream));
-    SEER_CUDA(run_gate_select_rows(g, num_sms, stream, true));
-  } else {
-    SEER_CUDA(run_gate_select(g, d->batch, stream, true));
+  {
+    NvtxRange r("gate_select");
+    if ((int64_t)d->batch * d->num_kv_heads > num_sms) {
+      // more rows than SMs: persistent row-claiming gate (its counter starts at 0)
+      SEER_CUDA(cudaMemsetAsync(g.row_counter, 0, sizeof(uint32_t), stream));
+      SEER_CUDA(run_gate_select_rows(g, num_sms, stream, true));
+    } else {
+      SEER_CUDA(run_gate_select(g, d->batch, stream, true));
+    }
   }
   if (a->unified_heads) {  // one block set per sequence, shared by its KV heads
     SelectParams u;
@@ -560,10 +591,14 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
     u.max_blocks = d->max_blocks;
     u.k_max = a->k_max;
     u.force_newest = a->force_newest ? 1 : 0;
+    NvtxRange r("unified_select");
     SEER_CUDA(run_unified_select(u, d->batch, stream, true));
   }
   // a3, then a4; each grid launches early and waits for its predecessor
-  SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, true));
+  {
+    NvtxRange r("sparse_decode");
+    SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, true));
+  }
   CombineParams c = {};
   c.o_part = w.o_part;
   c.lse_part = w.lse_part;
@@ -571,7 +606,10 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
   c.lse_out = a->lse_out;
   c.S = a->num_splits;
   c.out_host = out_mapped;
-  SEER_CUDA(run_combine(c, d->batch, d->num_q_heads, stream, true));
+  {
+    NvtxRange r("combine");
+    SEER_CUDA(run_combine(c, d->batch, d->num_q_heads, stream, true));
+  }
   if (mass) {
     MassParams m;
     m.idx = w.idx;
@@ -586,6 +624,7 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
     m.bs = d->block_size;
     m.max_blocks = d->max_blocks;
     m.k_max = a->k_max;
+    NvtxRange r("block_mass");
     SEER_CUDA(run_block_mass(m, d->batch, stream));
   }
   return SEER_OK;
@@ -609,6 +648,7 @@ seer_status seer_step_workspace_init(const seer_dims* d, int32_t k_max, int32_t 
 
 seer_status seer_decode_step_fused(const seer_dims* d, const seer_step_args* a,
                                    seer_stream stream) {
+  NvtxRange step_range("seer_decode_step_fused");
   SEER_TRY(check_dims(d));
   if (a == nullptr || a->k_per_seq == nullptr || a->kbar == nullptr) return SEER_ERR_INVALID_ARG;
   if (a->update_kbar < 0 || a->update_kbar > 2) return SEER_ERR_INVALID_ARG;
@@ -683,6 +723,7 @@ size_t seer_prefill_workspace_bytes(const seer_dims* d, int32_t k_max) {
 }
 
 seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_stream stream) {
+  NvtxRange prefill_range("seer_prefill");
   SEER_TRY(check_dims(d));
   if (a == nullptr || !a->q || !a->k_pool || !a->v_pool || !a->seqlens || !a->w_gate || !a->kbar ||
       !a->out)
@@ -731,7 +772,11 @@ seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_st
   if (a->pool_keys)
     SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
                             stream));
-  SEER_CUDA(run_prefill_gate_select(p, stream));
+  {
+    NvtxRange r("prefill_gate_select");
+    SEER_CUDA(run_prefill_gate_select(p, stream));
+  }
+  NvtxRange r("prefill_attention");
   SEER_CUDA(run_prefill_attention(tk, tv, p, stream));
   return SEER_OK;
 }

@@ -1,7 +1,7 @@
-// seer_decode_step_noalloc: the fused decode step for callers that cannot
-// allocate device memory.  Its workspace (scores, indices, counts, split
-// partials) lives in one file-scope device array owned by this library
-// instead of a caller buffer.
+// seer_decode_step_noalloc: the per-stage decode step (seer_decode_step) for
+// callers that cannot allocate device memory.  Its workspace (scores,
+// indices, counts, split partials) lives in one file-scope device array owned
+// by this library instead of a caller buffer.
 #include <mutex>
 
 #include "seer_kernels.cuh"
@@ -15,7 +15,8 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) uint8_t g_step_scratch[kScratchBytes];
 
 // Device address of g_step_scratch, looked up once per device with that
-// device current.  In host code the symbol itself is only a host-side
+// device current and kept for the process (valid while the device's primary
+// context lives).  In host code the symbol itself is only a host-side
 // handle, never a device pointer.
 void* scratch_address(int device) {
   static void* addr[kMaxDevices] = {};

@@ -53,6 +53,11 @@ class Workload:
     sparsity_permille: Optional[int] = None
     force_newest: bool = False
     num_splits: Optional[int] = None
+    # seed of the full-size draw; where it is not 1 it was picked by rejection
+    # so that every (b, KV head) row's gate margin at the k / k+1 boundary
+    # exceeds 1e-4 (see ``seed_note``)
+    seed: int = 1
+    seed_note: str = ""
 
     @property
     def group(self) -> int:
@@ -72,7 +77,9 @@ WORKLOADS = {
     "b8_h32_L8k_bs64_s90_newest": Workload(
         "b8_h32_L8k_bs64_s90_newest", batch=8, q_heads=32, kv_heads=8,
         head_dim=128, block_size=64, seqlen=8192, offsets="normal",
-        offset_var=0.5, sparsity_permille=900, force_newest=True),
+        offset_var=0.5, sparsity_permille=900, force_newest=True, seed=2,
+        seed_note="seed 1 draws a row with a 1.6e-6 gate margin; seed 2's smallest "
+                  "margin over all 64 rows is 2.7e-4"),
     # 16 x 40/8 heads, 32K context, 90% sparsity (52 of 512), 8 splits
     "b16_h40_L32k_bs64_s90": Workload(
         "b16_h40_L32k_bs64_s90", batch=16, q_heads=40, kv_heads=8,

@@ -354,8 +354,12 @@ SEER_API seer_status seer_block_mass(const seer_dims *d, const int32_t *idx,
  *     exceeds SEER_NOALLOC_SCRATCH_BYTES the call returns SEER_ERR_WORKSPACE
  *     before anything is enqueued.
  *   - Set-up: the first call on each device looks up the array's device
- *     address (cudaGetSymbolAddress) with that device current and caches it;
- *     make that first call before any stream capture begins.
+ *     address (cudaGetSymbolAddress) with that device current and caches it
+ *     for the rest of the process; make that first call before any stream
+ *     capture begins.  The cached address belongs to the device's primary
+ *     context: after cudaDeviceReset (or from a caller that made another
+ *     context current) it no longer points at the array, so do not call
+ *     this entry point again after a reset.
  *   - Sharing: all calls on a device use the same array, which keeps the last
  *     call's contents.  Nothing in it has to start at zero (every byte the
  *     step reads there is written earlier by the same call), but calls whose

@@ -142,3 +142,13 @@ def test_prefill_and_fused_host_checks(lib):
                                          null, null) == 1
     assert lib.seer_last_cuda_error().decode() == "no error"
 
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    """The binding's copy of the no-allocation array size is the header's."""
+    import re
+    from block_sparse_attention_step_b200 import seer
+    hdr = open(os.path.join(ROOT, "include", "seer.h")).read()
+    m = re.search(r"#define SEER_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
+    assert m, "SEER_NOALLOC_SCRATCH_BYTES not found in include/seer.h"
+    assert seer.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

@@ -462,3 +462,29 @@ def test_prefill_closed_forms_and_hand_case():
     from scipy.special import logsumexp, softmax
     np.testing.assert_allclose(o, softmax(x, axis=1) @ V[32:41], rtol=1e-12)
     np.testing.assert_allclose(l, logsumexp(x, axis=1), rtol=1e-13)
+
+
+def test_prefill_gate_hand_case():
+    """The pooled-query gate on a hand-worked case with a partial last block:
+    pooled queries, pooled keys, the causal score matrix and the per-block
+    selection with the diagonal block forced (tests/golden/prefill_gate_hand.json,
+    derivation in the file)."""
+    c = _load("prefill_gate_hand.json")
+    Q, K, Wm = (np.array(c[n], float) for n in ("Q", "K", "W"))
+    L, bs = c["seqlen"], c["block_size"]
+    np.testing.assert_array_equal(O.pool_queries(Q, L, bs), np.array(c["qbar"], float))
+    kbar = O.pool_keys(K, L, bs)
+    np.testing.assert_array_equal(kbar, np.array(c["kbar"], float))
+    want = np.array([[_f(x) for x in row] for row in c["scores"]])
+    got = O.prefill_gate_scores(Q, Wm, kbar, L, bs, c["scale"])
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-15)
+    for i in range(want.shape[0]):
+        np.testing.assert_allclose(O.prefill_gate_row(Q, Wm, kbar, L, bs, c["scale"], i),
+                                   want[i, :i + 1], rtol=0, atol=1e-15)
+    ks = [O.k_from_sparsity(i + 1, c["sparsity_permille"]) for i in range(want.shape[0])]
+    assert ks == c["k"]
+    sel = O.prefill_select(got, lambda i: ks[i])
+    assert [s.tolist() for s in sel] == c["selected"]
+    # the whole prefill row reaches the same selection
+    row = O.prefill_row(Q, Wm, K, K, L, bs, lambda i: ks[i], c["scale"], 1.0)
+    assert [s.tolist() for s in row["selected"]] == c["selected"]

@@ -3,13 +3,13 @@
 The no-allocation entry point serves callers that cannot allocate device
 memory (a host runtime that owns all GPU memory through its own pool, or a
 decode loop that must never enter the CUDA allocator): it runs the same step
-with the library's fixed 16 MiB device array as workspace.  Two calls in a
-row must each match the caller-workspace step within the output tolerance the
-other tests use, and a size beyond the array must be refused.  This file is
+with the library's fixed 16 MiB device array as workspace.  Both paths run the
+same deterministic kernels on the same inputs, so two calls in a row must
+each give exactly the caller-workspace step's bits (a scratch carve at a wrong
+offset would show), and a size beyond the array must be refused.  This file is
 collected last on purpose, so a failure here comes after every other test has
 run; it also passes alone in a fresh process.
 """
-import numpy as np
 import pytest
 import torch
 
@@ -17,7 +17,7 @@ from block_sparse_attention_step_b200 import seer
 from block_sparse_attention_step_b200 import workloads as W
 from block_sparse_attention_step_b200.runner import StepBuffers
 
-from gpu_util import assert_out_close, f64, require_gpu
+from gpu_util import require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +30,9 @@ def test_noalloc_step_matches_workspace_step_twice():
     run.pool_full()
     run.step(update_kbar=0)
     torch.cuda.synchronize()
-    ref_out, ref_lse = f64(run.out), f64(run.lse)
+    ref_out, ref_lse = run.out.clone(), run.lse.clone()
+    v = run.workspace_views()
+    ref_idx, ref_nsel = v["idx"].clone(), v["n_sel"].clone()
     assert run.status.item() == 0
 
     need = seer.seer_step_workspace_bytes(run.dims, run.k_max, run.num_splits)
@@ -40,11 +42,11 @@ def test_noalloc_step_matches_workspace_step_twice():
         run.lse.fill_(0)
         seer.seer_decode_step_noalloc(run.dims, run.args(update_kbar=0))
         torch.cuda.synchronize()
-        out, lse = f64(run.out), f64(run.lse)
-        for b in range(w.batch):
-            assert_out_close(out[b], ref_out[b], ("call", call, "batch", b))
-        np.testing.assert_allclose(lse, ref_lse, atol=1e-3)
+        assert torch.equal(run.out, ref_out), ("call", call)
+        assert torch.equal(run.lse, ref_lse), ("call", call)
         assert run.status.item() == 0
+    # the caller's workspace was not touched by the no-allocation calls
+    assert torch.equal(v["idx"], ref_idx) and torch.equal(v["n_sel"], ref_nsel)
 
     # a request larger than the fixed array is refused before any work
     big = seer.make_dims(64, 64, 8, 128, 64, 4096, 64 * 4096)
