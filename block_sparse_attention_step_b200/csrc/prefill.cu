@@ -17,6 +17,7 @@
 #include "block_mean.cuh"
 #include "seer_kernels.cuh"
 #include "select_core.cuh"
+#include "tcgen05.cuh"
 
 namespace seer {
 
@@ -154,34 +155,78 @@ cudaError_t run_prefill_gate_select(const PrefillParams& p, cudaStream_t stream)
 }
 
 // ---------------------------------------------------------------- attention
-constexpr int kPAMathWarps = 4;                          // 16 query tokens each
-constexpr int kPAThreads = (kPAMathWarps + 1) * 32;      // + the copy warp
-constexpr int kPAStages = 3;
-constexpr int kPAHalf = kTileTokens * 64 * 2;            // 64 tokens x 64 dims bf16
-constexpr int kPAStageBytes = 4 * kPAHalf;               // K lo, K hi, V lo, V hi
-constexpr size_t kPABars = (size_t)kPAStages * kPAStageBytes;
-constexpr size_t kPASmem = 1024 + kPABars + 16 * kPAStages + 8 * kPAStages;
+//
+// One CTA per (b, KV head h, 64-token query tile, pair of the group's query
+// heads), longest causal prefixes first.  Its 128 query rows (64 tokens x 2
+// heads; a group of odd size repeats its last head in the last pair, whose
+// copy is computed and dropped) form the M = 128 side of the fifth-generation
+// tensor-core MMAs, with both accumulators in tensor memory:
+//   S = Q K^T  (N = 64 keys, K = 128 dims: 8 MMAs of K = 16)
+//   O += P V   (N = 128 dims, K = 64 keys: 4 MMAs of K = 16)
+// Warp roles (192 threads): warp 0 issues the TMA loads (Q once; K and V of
+// every key tile of the selected blocks, 64 keys each, in 3 K and 2 V
+// stages); warp 1 allocates 256 TMEM columns (S double-buffered in 2 x 64,
+// O in 128) and one of its threads issues the MMAs; warps 2-5 (one query row
+// per thread, TMEM lane = row) read S, apply the causal and sequence masks,
+// run the online softmax in the exp2 domain and write P as bf16 into the
+// shared-memory slot the tile's K occupied (S = Q K^T is done with it), in
+// the 128-byte swizzled K-major layout the MMA reads.  The running maximum
+// is a reference that moves only when a row's maximum grows by more than
+// 2^8; O (in TMEM) and l are then rescaled by the same factor, so the
+// result is exact for any reference.  Key rows past the sequence are zeroed
+// in V before P V runs.  Stage hand-offs go through mbarriers; tcgen05.commit
+// arrives on them when the MMAs finish.  Every wait is bounded
+// (SEER_DEV_TIMEOUT); TMEM is freed on every path.
+constexpr int kTCThreads = 192;
+constexpr int kTCRows = 128;                      // MMA M: 64 tokens x 2 heads
+constexpr int kTCKStages = 3, kTCVStages = 2;
+constexpr int kTCBox = 64 * 128;                  // one TMA box: 64 rows x 64 bf16 dims
+constexpr int kTCTile = 2 * kTCBox;               // 64 keys x 128 dims (K or V)
+constexpr int kTCQBytes = kTCRows * kHeadDim * 2; // 2 boxes of 128 rows
+constexpr int kTCData = kTCQBytes + (kTCKStages + kTCVStages) * kTCTile;  // 112 KB
+constexpr size_t kTCSmem = (size_t)kTCData + 1024;  // + barriers and alignment slack
+constexpr uint32_t kTCCols = 256;                 // S0 [0,64), S1 [64,128), O [128,256)
+constexpr float kTCRescale = 8.f;                 // log2 growth that moves the reference
+constexpr uint32_t kIdescS = tc_idesc_bf16(128, 64, 0, 0);    // Q (K-major) x K (K-major)
+constexpr uint32_t kIdescPV = tc_idesc_bf16(128, 128, 0, 1);  // P (K-major) x V (MN-major)
 
-__device__ __forceinline__ uint32_t ld_bf16x2(const uint16_t* p) {
-  return __ldg(reinterpret_cast<const uint32_t*>(p));
-}
+struct TcBars {
+  uint64_t q_full;
+  uint64_t k_full[kTCKStages], k_empty[kTCKStages];
+  uint64_t v_full[kTCVStages], v_empty[kTCVStages];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, pv_done, mma_done;
+  int2 meta[kTCKStages];  // per K stage: (first key token, valid keys) or (0, -1): no more
+  uint32_t tmem_base;
+};
+static_assert(sizeof(TcBars) <= 256, "barrier block");
 
-__global__ void __launch_bounds__(kPAThreads, 2)
-    prefill_attention_kernel(const __grid_constant__ CUtensorMap tm_k,
+__device__ __forceinline__ uint64_t tc_kdesc(uint32_t addr) { return tc_desc_sw128(addr, 16, 1024); }
+
+__global__ void __launch_bounds__(kTCThreads, 2)
+    prefill_attention_kernel(const __grid_constant__ CUtensorMap tm_q,
+                             const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
-  extern __shared__ uint8_t pa_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pa_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPABars);
-  uint64_t* empty = full + kPAStages;
-  int2* meta = reinterpret_cast<int2*>(empty + kPAStages);  // (first key token, valid keys)
+  extern __shared__ uint8_t tc_raw[];
+  // 1024-byte aligned data (the 128-byte swizzle atom); the barriers go into
+  // the slack in front when there are 256 bytes of it, else behind the data
+  const uintptr_t raw = reinterpret_cast<uintptr_t>(tc_raw);
+  uint8_t* data = reinterpret_cast<uint8_t*>((raw + 1023) & ~uintptr_t(1023));
+  TcBars* bars = reinterpret_cast<TcBars*>(
+      (uintptr_t)data - raw >= 256 ? tc_raw : data + kTCData);
+  uint8_t* q_s = data;
+  uint8_t* k_ring = data + kTCQBytes;
+  uint8_t* v_ring = k_ring + kTCKStages * kTCTile;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Lq = p.max_blocks * p.bs;
   const int ntiles = Lq / kTileTokens;
   const int tile = ntiles - 1 - (int)blockIdx.x;  // longest causal prefixes first
-  const int qh = blockIdx.y, b = blockIdx.z, h = qh / p.G;
+  const int npairs = (p.G + 1) >> 1;
+  const int h = (int)blockIdx.y / npairs, pair = (int)blockIdx.y - h * npairs;
+  const int b = blockIdx.z;
+  const int g0 = 2 * pair;
+  const bool two = g0 + 1 < p.G;
   int L = __ldg(p.seqlens + b);
   L = max(0, min(L, Lq));
   const int t0 = tile * kTileTokens;
@@ -189,239 +234,347 @@ __global__ void __launch_bounds__(kPAThreads, 2)
   const int t_last = min(t0 + kTileTokens - 1, L - 1);
   const int qb = t0 / p.bs;  // query block of this tile
   const int64_t row = ((int64_t)b * p.Hkv + h) * p.max_blocks + qb;
+  // after a wait has run out somewhere in the grid, later CTAs do no work
+  // (each run-out wait costs about a second)
+  if (p.status != nullptr &&
+      (*reinterpret_cast<const volatile int32_t*>(p.status) & SEER_DEV_TIMEOUT))
+    return;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPAStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kPAMathWarps);
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kTCKStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
     }
+    for (int s = 0; s < kTCVStages; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->s_free[s], 4);
+    }
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->mma_done, 1);
     fence_mbar_init();
   }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTCCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
 
-  if (warp == kPAMathWarps) {
+  if (warp == 0) {
     // ================================================================ copies
-    if (lane != 0) return;
-    prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
-    const uint64_t policy = policy_evict_first();
-    const int n = max(0, min(__ldg(p.n_sel + row), p.k_max));
-    const int nb = ceil_div_i(L, p.bs);
-    uint32_t issued = 0;
-    bool ok = true;
-    for (int q = 0; q < n && ok; ++q) {
-      const int j = __ldg(p.idx + row * p.k_max + q);
-      if (j < 0 || j >= nb || j > qb) {
-        flag_status(p.status, SEER_DEV_BAD_INDEX);
-        continue;
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      // Q is read by this CTA alone; K and V tiles by every query tile that
+      // selected their block and by the group's other head pairs
+      const uint64_t q_policy = policy_evict_first();
+      const uint64_t policy = policy_evict_normal();
+      // Q: rows 0-63 = tokens t0.. of head g0, rows 64-127 = head g0 + 1;
+      // dims 0-63 in the first 16 KB, 64-127 in the second
+      mbar_arrive_expect_tx(&bars->q_full, kTCQBytes);
+      for (int half = 0; half < 2; ++half)
+        for (int gs = 0; gs < 2; ++gs) {
+          const int qh = h * p.G + (two ? g0 + gs : g0);
+          tma_load_4d(q_s + half * (kTCQBytes / 2) + gs * kTCBox, &tm_q, 64 * half, qh, t0, b,
+                      &bars->q_full, q_policy);
+        }
+      const int n = max(0, min(__ldg(p.n_sel + row), p.k_max));
+      const int nb = ceil_div_i(L, p.bs);
+      uint32_t kn = 0, vn = 0;  // K / V tiles issued
+      bool ok = true;
+      for (int q = 0; q < n && ok; ++q) {
+        const int j = __ldg(p.idx + row * p.k_max + q);
+        if (j < 0 || j >= nb || j > qb) {
+          flag_status(p.status, SEER_DEV_BAD_INDEX);
+          continue;
+        }
+        const int64_t page = page_of(p.page_table, b, j, p.max_blocks);
+        if (page < 0 || page >= p.num_pages) {
+          flag_status(p.status, SEER_DEV_BAD_PAGE);
+          continue;
+        }
+        for (int e = 0; e * kTileTokens < p.bs; ++e) {
+          const int s0 = j * p.bs + e * kTileTokens;
+          if (s0 >= L || s0 > t_last) break;  // nothing a query of this tile may see
+          const int t = e * kTileTokens;
+          const int c1 = p.token_inner ? t : h, c2 = p.token_inner ? h : t;
+          const int ks = kn % kTCKStages;
+          if (!mbar_wait(&bars->k_empty[ks], ((kn / kTCKStages) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          bars->meta[ks] = make_int2(s0, min(kTileTokens, L - s0));
+          mbar_arrive_expect_tx(&bars->k_full[ks], kTCTile);
+          uint8_t* kd = k_ring + ks * kTCTile;
+          tma_load_4d(kd, &tm_k, 0, c1, c2, (int)page, &bars->k_full[ks], policy);
+          tma_load_4d(kd + kTCBox, &tm_k, 64, c1, c2, (int)page, &bars->k_full[ks], policy);
+          ++kn;
+          const int vs = vn % kTCVStages;
+          if (!mbar_wait(&bars->v_empty[vs], ((vn / kTCVStages) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->v_full[vs], kTCTile);
+          uint8_t* vd = v_ring + vs * kTCTile;
+          tma_load_4d(vd, &tm_v, 0, c1, c2, (int)page, &bars->v_full[vs], policy);
+          tma_load_4d(vd + kTCBox, &tm_v, 64, c1, c2, (int)page, &bars->v_full[vs], policy);
+          ++vn;
+        }
       }
-      const int64_t page = page_of(p.page_table, b, j, p.max_blocks);
-      if (page < 0 || page >= p.num_pages) {
-        flag_status(p.status, SEER_DEV_BAD_PAGE);
-        continue;
+      bool marked = false;
+      if (ok) {  // end marker: a K stage with no data
+        const int ks = kn % kTCKStages;
+        if (mbar_wait(&bars->k_empty[ks], ((kn / kTCKStages) & 1) ^ 1)) {
+          bars->meta[ks] = make_int2(0, -1);
+          mbar_arrive(&bars->k_full[ks]);
+          marked = true;
+        }
       }
-      for (int e = 0; e * kTileTokens < p.bs; ++e) {
-        const int s0 = j * p.bs + e * kTileTokens;
-        if (s0 >= L || s0 > t_last) break;  // nothing a query of this tile may see
-        const int slot = issued % kPAStages;
-        if (!mbar_wait(&empty[slot], ((issued / kPAStages) & 1) ^ 1)) {
+      if (!marked) flag_status(p.status, SEER_DEV_TIMEOUT);
+      // Let this CTA's copies land before it retires: the newest copy of
+      // each stage (older ones were consumed before their stage was reused;
+      // with the end marker posted, the marker's stage holds no copy).
+      for (uint32_t k = 1; k <= (uint32_t)kTCKStages && k <= kn; ++k) {
+        const uint32_t c = kn - k;
+        if (marked && c % kTCKStages == kn % kTCKStages) continue;
+        if (!mbar_wait(&bars->k_full[c % kTCKStages], (c / kTCKStages) & 1))
           flag_status(p.status, SEER_DEV_TIMEOUT);
+      }
+      for (uint32_t k = 1; k <= (uint32_t)kTCVStages && k <= vn; ++k) {
+        const uint32_t c = vn - k;
+        if (!mbar_wait(&bars->v_full[c % kTCVStages], (c / kTCVStages) & 1))
+          flag_status(p.status, SEER_DEV_TIMEOUT);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA
+    if (lane == 0) {
+      bool ok = mbar_wait(&bars->q_full, 0);
+      const uint32_t q_addr = smem_u32(q_s);
+      auto issue_pv = [&](uint32_t jj) -> bool {
+        if (!mbar_wait(&bars->p_full, jj & 1)) return false;
+        const int vs = jj % kTCVStages;
+        if (!mbar_wait(&bars->v_full[vs], (jj / kTCVStages) & 1)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(k_ring + (jj % kTCKStages) * kTCTile);
+        const uint32_t va = smem_u32(v_ring + vs * kTCTile);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_f16_ss(tmem + 128, tc_kdesc(pa + 32 * kk), tc_desc_sw128(va + 2048 * kk, kTCBox, 1024),
+                        kIdescPV, (jj > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bars->pv_done);
+        tc_commit(&bars->k_empty[jj % kTCKStages]);
+        tc_commit(&bars->v_empty[vs]);
+        return true;
+      };
+      uint32_t it = 0;
+      while (ok) {
+        const int ks = it % kTCKStages;
+        if (!mbar_wait(&bars->k_full[ks], (it / kTCKStages) & 1)) {
           ok = false;
           break;
         }
-        meta[slot] = make_int2(s0, min(kTileTokens, L - s0));
-        mbar_arrive_expect_tx(&full[slot], kPAStageBytes);
-        const int t = e * kTileTokens;
-        const int c1 = p.token_inner ? t : h, c2 = p.token_inner ? h : t;
-        uint8_t* st = ring + slot * kPAStageBytes;
-        tma_load_4d(st + 0 * kPAHalf, &tm_k, 0, c1, c2, (int)page, &full[slot], policy);
-        tma_load_4d(st + 1 * kPAHalf, &tm_k, 64, c1, c2, (int)page, &full[slot], policy);
-        tma_load_4d(st + 2 * kPAHalf, &tm_v, 0, c1, c2, (int)page, &full[slot], policy);
-        tma_load_4d(st + 3 * kPAHalf, &tm_v, 64, c1, c2, (int)page, &full[slot], policy);
-        ++issued;
+        if (bars->meta[ks].y < 0) break;  // no more key tiles
+        const int sb = it & 1;
+        if (it >= 2 && !mbar_wait(&bars->s_free[sb], ((it >> 1) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ka = smem_u32(k_ring + ks * kTCTile);
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const uint32_t off = (k8 >> 2) * (kTCQBytes / 2) + 32 * (k8 & 3);
+          const uint32_t koff = (k8 >> 2) * kTCBox + 32 * (k8 & 3);
+          tc_mma_f16_ss(tmem + 64 * sb, tc_kdesc(q_addr + off), tc_kdesc(ka + koff), kIdescS,
+                        k8 > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars->s_full[sb]);
+        if (it >= 1 && !issue_pv(it - 1)) {
+          ok = false;
+          break;
+        }
+        ++it;
       }
+      if (ok && it >= 1) ok = issue_pv(it - 1);
+      if (ok) {  // tell the softmax warps there is no tile `it`
+        const int sb = it & 1;
+        if (it >= 2) ok = mbar_wait(&bars->s_free[sb], ((it >> 1) & 1) ^ 1);
+        if (ok) mbar_arrive(&bars->s_full[sb]);
+      }
+      if (!ok) flag_status(p.status, SEER_DEV_TIMEOUT);
+      // every MMA this thread issued has finished before TMEM is freed
+      tc_commit(&bars->mma_done);
+      if (!mbar_wait(&bars->mma_done, 0)) flag_status(p.status, SEER_DEV_TIMEOUT);
     }
-    bool marked = false;
-    if (ok) {  // end marker: a stage with no data
-      const int slot = issued % kPAStages;
-      if (mbar_wait(&empty[slot], ((issued / kPAStages) & 1) ^ 1)) {
-        meta[slot] = make_int2(0, -1);
-        mbar_arrive(&full[slot]);
-        marked = true;
+  } else {
+    // ============================================================ softmax
+    const int quarter = warp & 3;               // TMEM lanes 32 * quarter ..
+    const int r = 32 * quarter + lane;          // this thread's row
+    const int tq = t0 + (r & 63);               // its query token
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint32_t it = 0;
+    for (;; ++it) {
+      const int sb = it & 1, ks = it % kTCKStages;
+      ok = mbar_wait(&bars->s_full[sb], (it >> 1) & 1);
+      ok = ok && mbar_wait(&bars->k_full[ks], (it / kTCKStages) & 1);  // meta of this tile
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int2 mt = bars->meta[ks];
+      if (mt.y < 0) break;  // no more key tiles
+      uint32_t sv[64];
+      __syncwarp();
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
+        tmem_ld32(lane_addr + 64 * sb, lo);
+        tmem_ld32(lane_addr + 64 * sb + 32, hi);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+      // visible keys of this row: c < lim (inside the sequence, not after tq)
+      const int lim = min(mt.y, tq - mt.x + 1);
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        x[c] = c < lim ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[c]);
+      }
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mx > m_ref + kTCRescale) {
+        if (m_ref != -INFINITY) {
+          alpha = fast_exp2(m_ref - mx);
+          rescale = true;
+        }
+        m_ref = mx;
+      }
+      const float ref = m_ref == -INFINITY ? 0.f : m_ref;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        x[c] = fast_exp2(x[c] - ref);  // exp2(-inf) = 0 for masked keys
+        sum += x[c];
+      }
+      l = l * alpha + sum;
+      // O is stable once the previous tile's P V has finished
+      if (it >= 1) ok = mbar_wait(&bars->pv_done, (it - 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t o[32];
+          __syncwarp();
+          tmem_ld32(lane_addr + 128 + 32 * c4, o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          __syncwarp();
+          tmem_st32(lane_addr + 128 + 32 * c4, o);
+        }
+      }
+      // key rows past the sequence may hold anything: zero them in V
+      if (mt.y < kTileTokens) {
+        const int vs = it % kTCVStages;
+        if (!mbar_wait(&bars->v_full[vs], (it / kTCVStages) & 1)) ok = false;
+        uint8_t* vd = v_ring + vs * kTCTile;
+        const int nz = (kTileTokens - mt.y) * 16;  // 16-byte pieces (2 boxes x 8 per row)
+        for (int i = r; i < nz && ok; i += kTCRows) {
+          const int key = mt.y + (i >> 4), piece = i & 15;
+          *reinterpret_cast<uint4*>(vd + (piece >> 3) * kTCBox + key * 128 + (piece & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      // P (bf16) into the K slot of this tile: row r, 128-byte swizzled
+      uint8_t* prow = k_ring + ks * kTCTile + r * 128;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint4 v;
+        v.x = pack_bf16x2(x[8 * c8 + 0], x[8 * c8 + 1]);
+        v.y = pack_bf16x2(x[8 * c8 + 2], x[8 * c8 + 3]);
+        v.z = pack_bf16x2(x[8 * c8 + 4], x[8 * c8 + 5]);
+        v.w = pack_bf16x2(x[8 * c8 + 6], x[8 * c8 + 7]);
+        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+    if (!ok) flag_status(p.status, SEER_DEV_TIMEOUT);
+    // ---- epilogue: the last P V, then normalise, bf16 out, natural-log lse
+    bool have_o = ok && it >= 1;
+    if (have_o) {
+      have_o = mbar_wait(&bars->pv_done, (it - 1) & 1);
+      have_o = __all_sync(0xffffffffu, have_o);
+      if (!have_o) flag_status(p.status, SEER_DEV_TIMEOUT);
+    }
+    tc_fence_after();
+    const int gs = r >> 6;
+    const int qh = h * p.G + g0 + gs;
+    const bool store = (gs == 0 || two) && tq < L;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint16_t* orow = p.out + (((int64_t)b * Lq + tq) * p.Hq + qh) * kHeadDim;
+#pragma unroll 1
+    for (int c4 = 0; c4 < 4; ++c4) {
+      uint32_t o[32];
+      if (have_o) {
+        __syncwarp();
+        tmem_ld32(lane_addr + 128 + 32 * c4, o);
       } else {
-        flag_status(p.status, SEER_DEV_TIMEOUT);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (store) {
+#pragma unroll
+        for (int e8 = 0; e8 < 4; ++e8) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[8 * e8 + 0]) * inv, __uint_as_float(o[8 * e8 + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(o[8 * e8 + 2]) * inv, __uint_as_float(o[8 * e8 + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(o[8 * e8 + 4]) * inv, __uint_as_float(o[8 * e8 + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(o[8 * e8 + 6]) * inv, __uint_as_float(o[8 * e8 + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * e8) = v;
+        }
       }
     }
-    // Let every copy this CTA started land before it retires.  With the end
-    // marker posted, the stage that last used the marker's slot was released
-    // by every math warp (so its copy landed), and its full barrier has moved
-    // on by the marker's phase: a parity wait on it could not tell the two
-    // apart, so it is left out.
-    const uint32_t in_flight = marked ? kPAStages - 1 : kPAStages;
-    for (uint32_t k = 0; k < in_flight && k < issued; ++k) {
-      const uint32_t s = issued - 1 - k;
-      if (!mbar_wait(&full[s % kPAStages], (s / kPAStages) & 1))
-        flag_status(p.status, SEER_DEV_TIMEOUT);
-    }
-    return;
+    if (store && p.lse != nullptr)
+      p.lse[((int64_t)b * p.Hq + qh) * Lq + tq] =
+          l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
   }
-
-  // ================================================================== math
-  const int r = lane >> 2, c = lane & 3;
-  const int ta = t0 + warp * 16 + r, tb = ta + 8;  // this thread's two query rows
-  // Q as the A operand (16 tokens x 128 dims), straight from global memory
-  uint32_t qa[8][4];
-  {
-    const uint16_t* qra = p.q + (((int64_t)b * Lq + ta) * p.Hq + qh) * kHeadDim + 2 * c;
-    const uint16_t* qrb = p.q + (((int64_t)b * Lq + tb) * p.Hq + qh) * kHeadDim + 2 * c;
-    const bool ina = ta < L, inb = tb < L;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      qa[ks][0] = ina ? ld_bf16x2(qra + 16 * ks) : 0u;
-      qa[ks][1] = inb ? ld_bf16x2(qrb + 16 * ks) : 0u;
-      qa[ks][2] = ina ? ld_bf16x2(qra + 16 * ks + 8) : 0u;
-      qa[ks][3] = inb ? ld_bf16x2(qrb + 16 * ks + 8) : 0u;
-    }
-  }
-  float o[16][4];
-#pragma unroll
-  for (int dt = 0; dt < 16; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
-
-  for (int k = 0;; ++k) {
-    const int slot = k % kPAStages;
-    if (!mbar_wait(&full[slot], (k / kPAStages) & 1)) {
-      flag_status(p.status, SEER_DEV_TIMEOUT);
-      break;
-    }
-    const int2 mt = meta[slot];
-    if (mt.y < 0) break;  // end marker
-    const int s0 = mt.x, valid = mt.y;
-    const uint32_t kbase = smem_u32(ring + slot * kPAStageBytes);
-    const uint32_t vbase = kbase + 2 * kPAHalf;
-
-    // ---- S = Q K^T (16 tokens x 64 keys), K rows as the B operand
-    float s[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-      for (int kp = 0; kp < 4; ++kp) {
-        const int key = nt * 8 + (lane & 7);
-        const int chunk = 4 * kp + (lane >> 3);
-        const uint32_t addr = kbase + (chunk >> 3) * kPAHalf + key * 128 +
-                              (((chunk & 7) ^ (key & 7)) << 4);
-        uint32_t x0, x1, x2, x3;
-        ldmatrix_x4(addr, x0, x1, x2, x3);
-        mma_bf16_16816(s[nt], qa[2 * kp], x0, x1);
-        mma_bf16_16816(s[nt], qa[2 * kp + 1], x2, x3);
-      }
-    }
-    // ---- causal and tail masks, online softmax in the exp2 domain
-    float mxa = -INFINITY, mxb = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = nt * 8 + 2 * c + (e & 1);
-        const int tq = e < 2 ? ta : tb;
-        const bool masked = col >= valid || s0 + col > tq;
-        s[nt][e] = masked ? -INFINITY : s[nt][e] * p.scale_log2;
-      }
-      mxa = fmaxf(mxa, fmaxf(s[nt][0], s[nt][1]));
-      mxb = fmaxf(mxb, fmaxf(s[nt][2], s[nt][3]));
-    }
-    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
-    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
-    mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
-    mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
-    const float na = fmaxf(ma, mxa), nbm = fmaxf(mb, mxb);
-    const float ua = na == -INFINITY ? 0.f : na, ub = nbm == -INFINITY ? 0.f : nbm;
-    const float alpha_a = fast_exp2(ma - ua), alpha_b = fast_exp2(mb - ub);
-    ma = na;
-    mb = nbm;
-    float suma = 0.f, sumb = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      s[nt][0] = fast_exp2(s[nt][0] - ua);
-      s[nt][1] = fast_exp2(s[nt][1] - ua);
-      s[nt][2] = fast_exp2(s[nt][2] - ub);
-      s[nt][3] = fast_exp2(s[nt][3] - ub);
-      suma += s[nt][0] + s[nt][1];
-      sumb += s[nt][2] + s[nt][3];
-    }
-    la = la * alpha_a + suma;
-    lb = lb * alpha_b + sumb;
-#pragma unroll
-    for (int dt = 0; dt < 16; ++dt) {
-      o[dt][0] *= alpha_a;
-      o[dt][1] *= alpha_a;
-      o[dt][2] *= alpha_b;
-      o[dt][3] *= alpha_b;
-    }
-    // ---- O += P V: P (from the S accumulators) rounded to bf16, V by ldmatrix.trans
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t ph[4];
-      ph[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-      ph[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-      ph[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      ph[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-      // tail keys (past the sequence) may hold anything: zero their V
-      const int k0 = 16 * kk + 2 * c;
-      const uint32_t m0 = (k0 < valid ? 0x0000ffffu : 0u) | (k0 + 1 < valid ? 0xffff0000u : 0u);
-      const uint32_t m1 =
-          (k0 + 8 < valid ? 0x0000ffffu : 0u) | (k0 + 9 < valid ? 0xffff0000u : 0u);
-#pragma unroll
-      for (int dp = 0; dp < 8; ++dp) {
-        const int key = 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int chunk = 2 * dp + (lane >> 4);
-        const uint32_t addr = vbase + (chunk >> 3) * kPAHalf + key * 128 +
-                              (((chunk & 7) ^ (key & 7)) << 4);
-        uint32_t v0, v1, v2, v3;
-        ldmatrix_x4_trans(addr, v0, v1, v2, v3);
-        v0 &= m0;
-        v1 &= m1;
-        v2 &= m0;
-        v3 &= m1;
-        mma_bf16_16816(o[2 * dp], ph, v0, v1);
-        mma_bf16_16816(o[2 * dp + 1], ph, v2, v3);
-      }
-    }
-    fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
-  }
-
-  // ---- epilogue: normalise, bf16 out, natural-log lse
-  la += __shfl_xor_sync(0xffffffffu, la, 1);
-  la += __shfl_xor_sync(0xffffffffu, la, 2);
-  lb += __shfl_xor_sync(0xffffffffu, lb, 1);
-  lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-  const float ia = la > 0.f ? 1.f / la : 0.f, ib = lb > 0.f ? 1.f / lb : 0.f;
-  if (ta < L) {
-    uint32_t* oa = reinterpret_cast<uint32_t*>(p.out + (((int64_t)b * Lq + ta) * p.Hq + qh) * kHeadDim);
-#pragma unroll
-    for (int dt = 0; dt < 16; ++dt) oa[(dt * 8 + 2 * c) / 2] = pack_bf16x2(o[dt][0] * ia, o[dt][1] * ia);
-    if (p.lse != nullptr && c == 0)
-      p.lse[((int64_t)b * p.Hq + qh) * Lq + ta] = la > 0.f ? (ma + log2f(la)) * kLn2 : -INFINITY;
-  }
-  if (tb < L) {
-    uint32_t* ob = reinterpret_cast<uint32_t*>(p.out + (((int64_t)b * Lq + tb) * p.Hq + qh) * kHeadDim);
-#pragma unroll
-    for (int dt = 0; dt < 16; ++dt) ob[(dt * 8 + 2 * c) / 2] = pack_bf16x2(o[dt][2] * ib, o[dt][3] * ib);
-    if (p.lse != nullptr && c == 0)
-      p.lse[((int64_t)b * p.Hq + qh) * Lq + tb] = lb > 0.f ? (mb + log2f(lb)) * kLn2 : -INFINITY;
+    tc_fence_after();
+    tmem_dealloc(tmem, kTCCols);
   }
 }
 
-cudaError_t run_prefill_attention(const CUtensorMap& tk, const CUtensorMap& tv,
-                                  const PrefillParams& p, cudaStream_t stream) {
+cudaError_t run_prefill_attention(const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const PrefillParams& p,
+                                  cudaStream_t stream) {
   static std::atomic<uint64_t> smem_set{0};
   cudaError_t e = ensure_smem_limit(prefill_attention_kernel, smem_set);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.max_blocks * p.bs / kTileTokens, p.Hq, p.B);
-  prefill_attention_kernel<<<grid, kPAThreads, kPASmem, stream>>>(tk, tv, p);
+  dim3 grid(p.max_blocks * p.bs / kTileTokens, p.Hkv * ((p.G + 1) / 2), p.B);
+  prefill_attention_kernel<<<grid, kTCThreads, kTCSmem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

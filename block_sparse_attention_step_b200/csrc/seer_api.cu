@@ -109,6 +109,25 @@ seer_status make_kv_map(const uint16_t* base, const seer_dims* d, int token_inne
   return r == CUDA_SUCCESS ? SEER_OK : SEER_ERR_UNSUPPORTED;
 }
 
+// Prompt-query tensor map over q [B][Lq][Hq][D] (Lq = max_blocks * bs): dims
+// (D, head, token, batch); box = 64 dims x 1 head x 64 tokens, 128-byte swizzle.
+seer_status make_q_map(const uint16_t* q, const seer_dims* d, CUtensorMap* map) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return SEER_ERR_CUDA;
+  const cuuint64_t lq = (cuuint64_t)d->max_blocks * d->block_size;
+  const cuuint64_t row = (cuuint64_t)d->head_dim * 2;
+  const cuuint64_t dims[4] = {(cuuint64_t)d->head_dim, (cuuint64_t)d->num_q_heads, lq,
+                              (cuuint64_t)d->batch};
+  const cuuint64_t strides[3] = {row, row * d->num_q_heads, row * d->num_q_heads * lq};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kTileTokens, 1};
+  const cuuint32_t elem[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(q), dims,
+                         strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SEER_OK : SEER_ERR_UNSUPPORTED;
+}
+
 seer_status check_dims(const seer_dims* d) {
   if (d == nullptr) return SEER_ERR_INVALID_ARG;
   if (d->batch < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1 || d->max_blocks < 1 ||
@@ -739,7 +758,8 @@ seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_st
   SEER_TRY(check_pool(d, a->k_pool));
   SEER_TRY(check_pool(d, a->v_pool));
   const int token_inner = d->stride_token < d->stride_head ? 1 : 0;
-  CUtensorMap tk, tv;
+  CUtensorMap tq, tk, tv;
+  SEER_TRY(make_q_map(a->q, d, &tq));
   SEER_TRY(make_kv_map(a->k_pool, d, token_inner, &tk));
   SEER_TRY(make_kv_map(a->v_pool, d, token_inner, &tv));
   const size_t rows = (size_t)d->batch * d->num_kv_heads * d->max_blocks;
@@ -777,7 +797,7 @@ seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_st
     SEER_CUDA(run_prefill_gate_select(p, stream));
   }
   NvtxRange r("prefill_attention");
-  SEER_CUDA(run_prefill_attention(tk, tv, p, stream));
+  SEER_CUDA(run_prefill_attention(tq, tk, tv, p, stream));
   return SEER_OK;
 }
 

@@ -112,8 +112,9 @@ struct PrefillParams {
 };
 
 cudaError_t run_prefill_gate_select(const PrefillParams& p, cudaStream_t stream);
-cudaError_t run_prefill_attention(const CUtensorMap& tk, const CUtensorMap& tv,
-                                  const PrefillParams& p, cudaStream_t stream);
+cudaError_t run_prefill_attention(const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const PrefillParams& p,
+                                  cudaStream_t stream);
 
 // The single-launch step: the decode kernel with the gate rows before it and
 // the combine after it, in one cooperative grid.  Control words (zero before

@@ -112,6 +112,42 @@ def test_prefill_dense_is_causal_attention():
     assert_out_close(f64(run.out[0, :L]), ref, "dense")
 
 
+@pytest.mark.parametrize("q_heads", [4, 3])
+def test_prefill_growing_scores_rescale_the_accumulator(q_heads):
+    """Keys whose scale grows block by block push every row's running maximum
+    up past the kernel's rescale threshold (a factor of 2^8) several times,
+    so the output accumulated in tensor memory is rescaled on the way; the
+    result must still be plain causal attention (torch's fp64 SDPA).  Three
+    query heads leave the last head pair with one real head."""
+    w = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"].replace(batch=1, q_heads=q_heads, kv_heads=1,
+                                                           seqlen=700)
+    data = W.generate(w, 67, DEV)
+    q = W.prefill_queries(w, 67, data["nb_max"], DEV)
+    kp = data["k_pool"]                                   # contiguous: page j = block j
+    grow = 1.0 + 0.75 * torch.arange(kp.shape[0], device=DEV, dtype=torch.float32)
+    data["k_pool"] = (kp.float() * grow[:, None, None, None]).to(torch.bfloat16)
+    run = PrefillBuffers(w, data, q, sparsity_permille=0, budget_tokens=0)
+    run.run(pool_keys=True)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    L, G = 700, q_heads
+    Q = q[0, :L].double().permute(1, 0, 2)[None]
+    K = W.gather_rows(data["k_pool"], data["page_table"], 0, 0, L, 64).double()
+    V = W.gather_rows(data["v_pool"], data["page_table"], 0, 0, L, 64).double()
+    x = torch.einsum("gtd,sd->gts", Q[0].cpu(), K.cpu()) * scale_of(w) * 1.4426950408889634
+    causal = torch.tril(torch.ones(L, L, dtype=torch.bool))
+    run_max = x.masked_fill(~causal, float("-inf")).amax(-1)      # each row's final maximum
+    first = x[:, :, :64].masked_fill(~causal[:, :64], float("-inf")).amax(-1)
+    grown = (run_max - first)[:, 320:]                            # rows from block 5 on
+    assert float((grown > 8.0).double().mean()) > 0.5             # most of them rescale
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.cpu(), K.cpu()[None, None].expand(1, G, L, 128), V.cpu()[None, None].expand(1, G, L, 128),
+        is_causal=True, scale=scale_of(w))[0].permute(1, 0, 2).numpy()
+    assert_out_close(f64(run.out[0, :L]), ref, "rescaled")
+    lse_ref = torch.logsumexp(x.masked_fill(~causal, float("-inf")) / 1.4426950408889634, -1)
+    np.testing.assert_allclose(f64(run.lse[0, :, :L]), lse_ref.numpy(), atol=1e-3, rtol=1e-5)
+
+
 def test_prefill_tail_garbage_never_matters():
     """NaN in the cache slots past each sequence's end changes nothing."""
     w, permille, budget = CASES["paged_bs64_s80"]
