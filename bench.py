@@ -525,6 +525,17 @@ def workload_config(w, num_splits, k_max, rep, layout, args):
     """The config object both arms print (the same keys and values for the
     same workload, split count and selection size)."""
     replicas, touched = rep
+    rotation = replicas * touched
+    l2_bytes = 126 * 1024 * 1024
+    if rotation > 4 * l2_bytes:
+        l2 = (f"inputs larger than L2: {replicas} rotating replicas, "
+              f"{touched / 1e6:.0f} MB read per step, L2 126 MB")
+    elif rotation > l2_bytes:
+        l2 = (f"partly L2-resident: {replicas} rotating replicas, {touched / 1e6:.0f} MB read "
+              f"per step, the rotation is less than 4x the 126 MB L2")
+    else:
+        l2 = (f"L2-hot: {replicas} replica(s), {touched / 1e6:.0f} MB read per step, the "
+              f"rotation fits in the 126 MB L2")
     cfg = {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
            "head_dim": w.head_dim, "block_size": w.block_size,
            "seq_len": w.seqlen if w.seqlen else f"U[{w.seqlen_range[0]},{w.seqlen_range[1]}]",
@@ -532,8 +543,7 @@ def workload_config(w, num_splits, k_max, rep, layout, args):
                          else f"sparsity {w.sparsity_permille / 10:g}%"),
            "force_newest": w.force_newest, "paged": w.paged, "kv_layout": layout,
            "num_splits": int(num_splits), "k_max": int(k_max),
-           "l2": (f"inputs larger than L2: {replicas} rotating replicas, "
-                  f"{touched / 1e6:.0f} MB read per step, L2 126 MB"),
+           "l2": l2,
            "block_mass": bool(args.mass),
            "selection_scope": ("one block set per sequence (all KV heads)" if args.unified
                                else "per KV head"),
@@ -796,7 +806,7 @@ def run_prefill(args):
     from block_sparse_attention_step_b200.runner import PrefillBuffers
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    w = W.WORKLOADS[W.HEADLINE].replace(batch=2, seqlen=16384)
+    w = W.WORKLOADS[W.HEADLINE].replace(batch=args.prefill_batch, seqlen=args.prefill_seqlen)
     if args.sparsity is not None:
         w = w.replace(sparsity_permille=args.sparsity)
     runs = []
@@ -826,9 +836,20 @@ def run_prefill(args):
 
     ms_full = timed(True)
     ms_attn_gate = timed(False)
+    # the dominant kernel alone: the attention over the selection in place
+    for i in range(args.warmup):
+        runs[i % 2].attention()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(args.steps):
+        runs[i % 2].attention()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_attn = a.elapsed_time(b) / args.steps
     clock_info = clocks.stop()
     peaks, kind = measured_peaks()
-    tflops = flops / (ms_attn_gate * 1e-3) / 1e12
+    tflops = flops / (ms_attn * 1e-3) / 1e12
     line = {
         "metric": "prefill prompt tokens/s (query-pooled block gate + causal block-sparse attention)",
         "value": w.batch * w.seqlen / (ms_full * 1e-3), "unit": "tokens/s", "n_gpus": 1,
@@ -840,11 +861,17 @@ def run_prefill(args):
                    "seq_len": w.seqlen, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
                    "block_size": w.block_size, "sparsity_permille": w.sparsity_permille,
                    "step": "seer_prefill with the full key pooling"},
-        "stage_ms": {"prefill_with_pooling": ms_full, "gate_select_attention": ms_attn_gate},
+        "stage_ms": {"prefill_with_pooling": ms_full, "gate_select_attention": ms_attn_gate,
+                     "attention_alone": ms_attn},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"], "traffic": None,
-                     "kernel": "prefill gate+select and attention (algorithmic attention FLOPs "
-                               "over both launches)", "flops_per_step": flops,
+                     "kernel": "prefill_attention_kernel (tcgen05), launched alone through "
+                               "seer_prefill_attention on the selection in place",
+                     "flops_per_launch": flops,
+                     "flops_note": "4 D per (query token, query head, attended key): real heads "
+                                   "only (a group of odd size also computes one padded head "
+                                   "per head pair that is not counted)",
+                     "gate_select_attention_tflops": flops / (ms_attn_gate * 1e-3) / 1e12,
                      "peak_source": f"{kind} bf16_tflops (burst)"},
         "gpu_launches": 3 * args.steps,
         "clocks": clock_info,
@@ -1072,7 +1099,7 @@ def main(argv=None):
                    help="KV pool page layout: token-major [P][bs][Hkv][D] or head-major [P][Hkv][bs][D]")
     p.add_argument("--seed", type=int, default=None,
                    help="seed of replica 0 (default: the workload's recorded seed)")
-    p.add_argument("--max-replicas", type=int, default=8)
+    p.add_argument("--max-replicas", type=int, default=24)
     p.add_argument("--cpu-budget", type=float, default=15.0,
                    help="seconds of timed oracle passes for the CPU baseline (at least one)")
     p.add_argument("--cpu-max-bytes", type=float, default=4e9,
@@ -1089,6 +1116,8 @@ def main(argv=None):
                    help="the whole step as one cooperative launch (seer_decode_step_fused)")
     p.add_argument("--prefill", action="store_true",
                    help="measure the prefill path with query pooling instead of the decode step")
+    p.add_argument("--prefill-batch", type=int, default=2)
+    p.add_argument("--prefill-seqlen", type=int, default=16384)
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be at least 3")

@@ -741,54 +741,66 @@ size_t seer_prefill_workspace_bytes(const seer_dims* d, int32_t k_max) {
   return round256(rows * k_max * sizeof(int32_t)) + round256(rows * sizeof(int32_t));
 }
 
-seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_stream stream) {
-  NvtxRange prefill_range("seer_prefill");
+// Checks, tensor maps and parameters shared by the whole prefill and its
+// attention stage (nothing is enqueued).  `gate`: the gate fields are used.
+static seer_status prefill_prepare(const seer_dims* d, const seer_prefill_args* a, bool gate,
+                                   PrefillParams* p, CUtensorMap* tq, CUtensorMap* tk,
+                                   CUtensorMap* tv) {
   SEER_TRY(check_dims(d));
-  if (a == nullptr || !a->q || !a->k_pool || !a->v_pool || !a->seqlens || !a->w_gate || !a->kbar ||
-      !a->out)
-    return SEER_ERR_INVALID_ARG;
-  if (a->sparsity_permille < 0 || a->sparsity_permille > 1000 || a->budget_tokens < 0)
+  if (a == nullptr || !a->q || !a->k_pool || !a->v_pool || !a->seqlens || !a->out)
     return SEER_ERR_INVALID_ARG;
   if (a->k_max < 1 || a->k_max > d->max_blocks) return SEER_ERR_INVALID_ARG;
-  if (a->workspace == nullptr || !aligned(a->workspace, 256) ||
-      a->workspace_bytes < seer_prefill_workspace_bytes(d, a->k_max))
-    return SEER_ERR_WORKSPACE;
-  if (!aligned(a->q, 16) || !aligned(a->out, 16) || !aligned(a->w_gate, 16) || !aligned(a->kbar, 16))
-    return SEER_ERR_UNSUPPORTED;
+  if (!aligned(a->q, 16) || !aligned(a->out, 16)) return SEER_ERR_UNSUPPORTED;
+  if (gate) {
+    if (!a->w_gate || !a->kbar) return SEER_ERR_INVALID_ARG;
+    if (a->sparsity_permille < 0 || a->sparsity_permille > 1000 || a->budget_tokens < 0)
+      return SEER_ERR_INVALID_ARG;
+    if (a->workspace == nullptr || !aligned(a->workspace, 256) ||
+        a->workspace_bytes < seer_prefill_workspace_bytes(d, a->k_max))
+      return SEER_ERR_WORKSPACE;
+    if (!aligned(a->w_gate, 16) || !aligned(a->kbar, 16)) return SEER_ERR_UNSUPPORTED;
+  }
   SEER_TRY(check_pool(d, a->k_pool));
   SEER_TRY(check_pool(d, a->v_pool));
   const int token_inner = d->stride_token < d->stride_head ? 1 : 0;
+  SEER_TRY(make_q_map(a->q, d, tq));
+  SEER_TRY(make_kv_map(a->k_pool, d, token_inner, tk));
+  SEER_TRY(make_kv_map(a->v_pool, d, token_inner, tv));
+  *p = PrefillParams{};
+  p->q = a->q;
+  p->w_gate = a->w_gate;
+  p->kbar = a->kbar;
+  p->page_table = a->page_table;
+  p->seqlens = a->seqlens;
+  p->scores = a->scores_out;
+  p->out = a->out;
+  p->lse = a->lse_out;
+  p->status = a->dev_status;
+  p->B = d->batch;
+  p->Hq = d->num_q_heads;
+  p->Hkv = d->num_kv_heads;
+  p->G = d->num_q_heads / d->num_kv_heads;
+  p->bs = d->block_size;
+  p->max_blocks = d->max_blocks;
+  p->k_max = a->k_max;
+  p->sparsity_permille = a->sparsity_permille;
+  p->budget_tokens = a->budget_tokens;
+  p->token_inner = token_inner;
+  p->num_pages = d->num_pages;
+  p->gate_scale = a->gate_scale;
+  p->scale_log2 = a->softmax_scale * kLog2e;
+  return SEER_OK;
+}
+
+seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_stream stream) {
+  NvtxRange prefill_range("seer_prefill");
+  PrefillParams p;
   CUtensorMap tq, tk, tv;
-  SEER_TRY(make_q_map(a->q, d, &tq));
-  SEER_TRY(make_kv_map(a->k_pool, d, token_inner, &tk));
-  SEER_TRY(make_kv_map(a->v_pool, d, token_inner, &tv));
+  SEER_TRY(prefill_prepare(d, a, true, &p, &tq, &tk, &tv));
   const size_t rows = (size_t)d->batch * d->num_kv_heads * d->max_blocks;
-  PrefillParams p = {};
-  p.q = a->q;
-  p.w_gate = a->w_gate;
-  p.kbar = a->kbar;
-  p.page_table = a->page_table;
-  p.seqlens = a->seqlens;
-  p.scores = a->scores_out;
   p.idx = reinterpret_cast<int32_t*>(a->workspace);
   p.n_sel = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a->workspace) +
                                        round256(rows * a->k_max * sizeof(int32_t)));
-  p.out = a->out;
-  p.lse = a->lse_out;
-  p.status = a->dev_status;
-  p.B = d->batch;
-  p.Hq = d->num_q_heads;
-  p.Hkv = d->num_kv_heads;
-  p.G = d->num_q_heads / d->num_kv_heads;
-  p.bs = d->block_size;
-  p.max_blocks = d->max_blocks;
-  p.k_max = a->k_max;
-  p.sparsity_permille = a->sparsity_permille;
-  p.budget_tokens = a->budget_tokens;
-  p.token_inner = token_inner;
-  p.num_pages = d->num_pages;
-  p.gate_scale = a->gate_scale;
-  p.scale_log2 = a->softmax_scale * kLog2e;
   if (a->pool_keys)
     SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
                             stream));
@@ -797,6 +809,20 @@ seer_status seer_prefill(const seer_dims* d, const seer_prefill_args* a, seer_st
     SEER_CUDA(run_prefill_gate_select(p, stream));
   }
   NvtxRange r("prefill_attention");
+  SEER_CUDA(run_prefill_attention(tq, tk, tv, p, stream));
+  return SEER_OK;
+}
+
+seer_status seer_prefill_attention(const seer_dims* d, const seer_prefill_args* a,
+                                   const int32_t* idx, const int32_t* n_sel,
+                                   seer_stream stream) {
+  NvtxRange r("seer_prefill_attention");
+  if (idx == nullptr || n_sel == nullptr) return SEER_ERR_INVALID_ARG;
+  PrefillParams p;
+  CUtensorMap tq, tk, tv;
+  SEER_TRY(prefill_prepare(d, a, false, &p, &tq, &tk, &tv));
+  p.idx = const_cast<int32_t*>(idx);
+  p.n_sel = const_cast<int32_t*>(n_sel);
   SEER_CUDA(run_prefill_attention(tq, tk, tv, p, stream));
   return SEER_OK;
 }

@@ -166,6 +166,18 @@ class PrefillBuffers:
             self.w.batch, self.w.kv_heads, self.nb_max)
         return idx, n_sel
 
+    def attention(self, out=None, lse=None, stream=None):
+        """The attention stage alone over the selection the last run() left
+        in the workspace (seer_prefill_attention)."""
+        idx, n_sel = self.selection()
+        d = self.data
+        seer.seer_prefill_attention(self.dims, self.q, d["k_pool"], d["v_pool"], self.page_table,
+                                    d["seqlens"], idx, n_sel, k_max=self.k_max,
+                                    softmax_scale=self.scale,
+                                    out=self.out if out is None else out,
+                                    lse_out=self.lse if lse is None else lse,
+                                    dev_status=self.status, stream=stream)
+
     def run(self, pool_keys: bool = True, stream=None):
         d = self.data
         seer.seer_prefill(self.dims, self.q, d["k_pool"], d["v_pool"], self.page_table,

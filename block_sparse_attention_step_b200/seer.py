@@ -38,6 +38,7 @@ EXPORTS = (
     "seer_decode_step_noalloc",
     "seer_decode_step_fused", "seer_step_workspace_init",
     "seer_prefill_k_max", "seer_prefill_workspace_bytes", "seer_prefill",
+    "seer_prefill_attention",
     "seer_block_lse_elems", "seer_sparse_decode_mass", "seer_block_mass",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -116,6 +117,7 @@ _SIGS = {
     "seer_prefill_k_max": (_I, [_D, _I, _I]),
     "seer_prefill_workspace_bytes": (ctypes.c_size_t, [_D, _I]),
     "seer_prefill": (_I, [_D, ctypes.POINTER(seer_prefill_args), _P]),
+    "seer_prefill_attention": (_I, [_D, ctypes.POINTER(seer_prefill_args), _P, _P, _P]),
     "seer_block_lse_elems": (ctypes.c_size_t, [_D]),
     "seer_sparse_decode_mass": (_I, [_D, _P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P,
                                      _P, _P, _P, _P]),
@@ -373,6 +375,24 @@ def seer_prefill_k_max(d, sparsity_permille, budget_tokens):
 
 def seer_prefill_workspace_bytes(d, k_max):
     return _lib().seer_prefill_workspace_bytes(ctypes.byref(d), int(k_max))
+
+
+def seer_prefill_attention(d, q, k_pool, v_pool, page_table, seqlens, idx, n_sel, *, k_max,
+                           softmax_scale, out, lse_out=None, dev_status=None, stream=None):
+    a = seer_prefill_args()
+    a.q = _ptr(q, torch.bfloat16, "q")
+    a.k_pool = _ptr(k_pool, torch.bfloat16, "k_pool")
+    a.v_pool = _ptr(v_pool, torch.bfloat16, "v_pool")
+    a.page_table = _ptr(page_table, torch.int32, "page_table", allow_none=True)
+    a.seqlens = _ptr(seqlens, torch.int32, "seqlens")
+    a.k_max = int(k_max)
+    a.softmax_scale = float(softmax_scale)
+    a.out = _ptr(out, torch.bfloat16, "out")
+    a.lse_out = _ptr(lse_out, torch.float32, "lse_out", allow_none=True)
+    a.dev_status = _ptr(dev_status, torch.int32, "dev_status", allow_none=True)
+    _check("seer_prefill_attention", _lib().seer_prefill_attention(
+        ctypes.byref(d), ctypes.byref(a), _ptr(idx, torch.int32, "idx"),
+        _ptr(n_sel, torch.int32, "n_sel"), _stream(stream)))
 
 
 def seer_prefill(d, q, k_pool, v_pool, page_table, seqlens, w_gate, kbar, *, pool_keys,

@@ -416,6 +416,21 @@ SEER_API size_t seer_prefill_workspace_bytes(const seer_dims *d, int32_t k_max);
 SEER_API seer_status seer_prefill(const seer_dims *d, const seer_prefill_args *a,
                                   seer_stream stream);
 
+/* The attention stage of seer_prefill alone, over a selection the caller
+ * gives (the causal masked softmax of the "Sparse Attention Reasoning" page,
+ * Step 4, per query block): idx [B][Hkv][max_blocks][a->k_max] ascending
+ * block indices (-1 padded) and n_sel [B][Hkv][max_blocks] their counts, the
+ * layout seer_prefill leaves in its workspace.  Every query token t of query
+ * block i attends the tokens s <= t (s < seqlens[b]) of the blocks listed for
+ * i; blocks after i, out of range, or on pages outside the pool are skipped
+ * and flagged (SEER_DEV_BAD_INDEX / SEER_DEV_BAD_PAGE).  Uses a->q, k_pool,
+ * v_pool, page_table, seqlens, k_max, softmax_scale, out, lse_out and
+ * dev_status; the gate fields and the workspace are not read.  Same kernel,
+ * same bits as the attention inside seer_prefill. */
+SEER_API seer_status seer_prefill_attention(const seer_dims *d, const seer_prefill_args *a,
+                                            const int32_t *idx, const int32_t *n_sel,
+                                            seer_stream stream);
+
 /* ------------------------------------------------------ single-launch step
  * The whole step in one cooperative launch (the persistent decode grid runs
  * the gate rows first and the LSE combine last; next to the per-stage path,

@@ -172,6 +172,26 @@ def test_prefill_tail_garbage_never_matters():
     assert torch.equal(out_a, b_run.out)
 
 
+@pytest.mark.parametrize("name", ["paged_bs64_s80", "contig_bs128_budget"])
+def test_prefill_attention_alone_gives_the_same_bits(name):
+    """seer_prefill_attention over the selection seer_prefill left in its
+    workspace writes exactly seer_prefill's output and lse."""
+    w, permille, budget = CASES[name]
+    data = W.generate(w, 69, DEV)
+    q = W.prefill_queries(w, 69, data["nb_max"], DEV)
+    run = PrefillBuffers(w, data, q, sparsity_permille=permille, budget_tokens=budget)
+    run.run(pool_keys=True)
+    out2 = torch.zeros_like(run.out)
+    lse2 = torch.full_like(run.lse, 7.0)
+    run.attention(out=out2, lse=lse2)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    for b in range(w.batch):
+        L = int(data["seqlens"][b])
+        assert torch.equal(out2[b, :L], run.out[b, :L])
+        assert torch.equal(lse2[b, :, :L], run.lse[b, :, :L])
+
+
 def test_prefill_full_size_sampled():
     """The prefill at the size and seeds the benchmark times (batch 2, 16K-token
     prompt, 40/8 heads, bs 64, 90 %): every pooled key, and for sampled query

@@ -130,6 +130,14 @@ def test_prefill_and_fused_host_checks(lib):
     null = None
     a = seer.seer_prefill_args()
     assert lib.seer_prefill(ctypes.byref(d), ctypes.byref(a), null) == 1      # no inputs
+    # the attention stage alone: no selection, then no inputs
+    assert lib.seer_prefill_attention(ctypes.byref(d), ctypes.byref(a), null, null, null) == 1
+    sel = ctypes.c_void_p(4096)
+    assert lib.seer_prefill_attention(ctypes.byref(d), ctypes.byref(a), sel, sel, null) == 1
+    a.q = a.k_pool = a.v_pool = a.seqlens = a.out = ctypes.cast(ctypes.c_void_p(4096 + 8),
+                                                                ctypes.c_void_p)
+    a.k_max = 4
+    assert lib.seer_prefill_attention(ctypes.byref(d), ctypes.byref(a), sel, sel, null) == 2
     fake = ctypes.c_void_p(4096)
     b = seer.seer_step_args()
     b.k_per_seq = b.kbar = fake
