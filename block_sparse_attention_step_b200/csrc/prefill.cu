@@ -195,7 +195,7 @@ struct TcBars {
   uint64_t k_full[kTCKStages], k_empty[kTCKStages];
   uint64_t v_full[kTCVStages], v_empty[kTCVStages];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, mma_done;
+  uint64_t p_full, pv_done[2], mma_done;  // P V of tile j completes on pv_done[j & 1]
   int2 meta[kTCKStages];  // per K stage: (first key token, valid keys) or (0, -1): no more
   uint32_t tmem_base;
 };
@@ -255,7 +255,8 @@ __global__ void __launch_bounds__(kTCThreads, 2)
       mbar_init(&bars->s_free[s], 4);
     }
     mbar_init(&bars->p_full, 4);
-    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->pv_done[0], 1);
+    mbar_init(&bars->pv_done[1], 1);
     mbar_init(&bars->mma_done, 1);
     fence_mbar_init();
   }
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(kTCThreads, 2)
         for (int kk = 0; kk < 4; ++kk)
           tc_mma_f16_ss(tmem + 128, tc_kdesc(pa + 32 * kk), tc_desc_sw128(va + 2048 * kk, kTCBox, 1024),
                         kIdescPV, (jj > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&bars->pv_done);
+        tc_commit(&bars->pv_done[jj & 1]);
         tc_commit(&bars->k_empty[jj % kTCKStages]);
         tc_commit(&bars->v_empty[vs]);
         return true;
@@ -424,6 +425,19 @@ __global__ void __launch_bounds__(kTCThreads, 2)
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    // P V of tile k completes on pv_done[k & 1], as that barrier's (k >> 1)-th
+    // phase.  Tile j waits for tile j - 2's (long finished) so that neither
+    // barrier ever runs two phases ahead of what this warp has seen; only an
+    // O rescale waits for tile j - 1's.
+    uint32_t pv_seen0 = 0u, pv_seen1 = 0u;  // phases observed on pv_done[0] / [1]
+    auto wait_pv = [&](uint32_t k) -> bool {
+      const uint32_t b = k & 1u, ph = k >> 1;
+      if ((b ? pv_seen1 : pv_seen0) > ph) return true;
+      const bool r = mbar_wait(&bars->pv_done[b], ph & 1u);
+      if (b) pv_seen1 = ph + 1u;
+      else pv_seen0 = ph + 1u;
+      return r;
+    };
     uint32_t it = 0;
     for (;; ++it) {
       const int sb = it & 1, ks = it % kTCKStages;
@@ -436,24 +450,25 @@ __global__ void __launch_bounds__(kTCThreads, 2)
       if (mt.y < 0) break;  // no more key tiles
       uint32_t sv[64];
       __syncwarp();
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-        tmem_ld32(lane_addr + 64 * sb, lo);
-        tmem_ld32(lane_addr + 64 * sb + 32, hi);
-      }
+      tmem_ld64(lane_addr + 64 * sb, sv);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free[sb]);
-      // visible keys of this row: c < lim (inside the sequence, not after tq)
+      // visible keys of this row: c < lim (inside the sequence, not after tq);
+      // eight independent partial maxima and sums keep the dependent chains
+      // short (two softmax warps per scheduler hide little latency)
       const int lim = min(mt.y, tq - mt.x + 1);
       float x[64];
-      float mx = -INFINITY;
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         x[c] = c < lim ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
+        m8[c & 7] = fmaxf(m8[c & 7], x[c]);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       float alpha = 1.f;
       bool rescale = false;
       if (mx > m_ref + kTCRescale) {
@@ -464,19 +479,25 @@ __global__ void __launch_bounds__(kTCThreads, 2)
         m_ref = mx;
       }
       const float ref = m_ref == -INFINITY ? 0.f : m_ref;
-      float sum = 0.f;
+      float s8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s8[i] = 0.f;
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         x[c] = fast_exp2(x[c] - ref);  // exp2(-inf) = 0 for masked keys
-        sum += x[c];
+        s8[c & 7] += x[c];
       }
+      const float sum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
       l = l * alpha + sum;
-      // O is stable once the previous tile's P V has finished
-      if (it >= 1) ok = mbar_wait(&bars->pv_done, (it - 1) & 1);
+      if (it >= 2) ok = wait_pv(it - 2);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      tc_fence_after();
       if (__any_sync(0xffffffffu, rescale)) {
+        // O is stable once the previous tile's P V has finished
+        if (it >= 1) ok = wait_pv(it - 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t o[32];
@@ -522,7 +543,8 @@ __global__ void __launch_bounds__(kTCThreads, 2)
     // ---- epilogue: the last P V, then normalise, bf16 out, natural-log lse
     bool have_o = ok && it >= 1;
     if (have_o) {
-      have_o = mbar_wait(&bars->pv_done, (it - 1) & 1);
+      if (it >= 2) have_o = wait_pv(it - 2);
+      have_o = wait_pv(it - 1) && have_o;
       have_o = __all_sync(0xffffffffu, have_o);
       if (!have_o) flag_status(p.status, SEER_DEV_TIMEOUT);
     }
@@ -533,24 +555,24 @@ __global__ void __launch_bounds__(kTCThreads, 2)
     const float inv = l > 0.f ? 1.f / l : 0.f;
     uint16_t* orow = p.out + (((int64_t)b * Lq + tq) * p.Hq + qh) * kHeadDim;
 #pragma unroll 1
-    for (int c4 = 0; c4 < 4; ++c4) {
-      uint32_t o[32];
+    for (int c2 = 0; c2 < 2; ++c2) {
+      uint32_t o[64];
       if (have_o) {
         __syncwarp();
-        tmem_ld32(lane_addr + 128 + 32 * c4, o);
+        tmem_ld64(lane_addr + 128 + 64 * c2, o);
       } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = 0u;
+        for (int e = 0; e < 64; ++e) o[e] = 0u;
       }
       if (store) {
 #pragma unroll
-        for (int e8 = 0; e8 < 4; ++e8) {
+        for (int e8 = 0; e8 < 8; ++e8) {
           uint4 v;
           v.x = pack_bf16x2(__uint_as_float(o[8 * e8 + 0]) * inv, __uint_as_float(o[8 * e8 + 1]) * inv);
           v.y = pack_bf16x2(__uint_as_float(o[8 * e8 + 2]) * inv, __uint_as_float(o[8 * e8 + 3]) * inv);
           v.z = pack_bf16x2(__uint_as_float(o[8 * e8 + 4]) * inv, __uint_as_float(o[8 * e8 + 5]) * inv);
           v.w = pack_bf16x2(__uint_as_float(o[8 * e8 + 6]) * inv, __uint_as_float(o[8 * e8 + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * e8) = v;
+          *reinterpret_cast<uint4*>(orow + 64 * c2 + 8 * e8) = v;
         }
       }
     }

@@ -369,17 +369,28 @@ def test_step_head_major_layout_is_bitwise_identical():
         assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("name", ["b16_h40_L32k_bs64_s90", "b64_ragged_h64_paged_bs64"])
-def test_step_fused_combine_equals_standalone_combine(name):
-    """The step merges the split partials inside the decode kernel; running the
-    standalone combine on the same partials gives the same bits."""
+@pytest.mark.parametrize("name,splits,q_heads", [
+    ("b16_h40_L32k_bs64_s90", 5, None),
+    ("b16_h40_L32k_bs64_s90", 20, None),       # more splits than one batch of loads
+    ("b64_ragged_h64_paged_bs64", 5, None),
+    ("b64_ragged_h64_paged_bs64", 3, 128),     # G = 16: the one-slot decode shape
+])
+def test_step_fused_combine_equals_standalone_combine(name, splits, q_heads):
+    """The step merges the split partials in its chained combine kernel;
+    running the standalone combine on the same partials gives the same bits
+    (more than one batch of 16 splits, and the group size whose decode shape
+    merges in its math warps, included)."""
     w = W.WORKLOADS[name].replace(batch=3)
+    if q_heads is not None:
+        w = w.replace(q_heads=q_heads)
     if w.seqlen is not None:
         w = w.replace(seqlen=4000)
     else:
         w = w.replace(seqlen_range=(64, 4000))
     data = W.generate(w, 31, DEV)
-    run = StepBuffers(w, data, num_splits=5)
+    run = StepBuffers(w, data, num_splits=splits)
+    run.out.fill_(0)
+    run.lse.fill_(0)
     run.step(update_kbar=2)
     v = run.workspace_views()
     out2 = torch.empty_like(run.out)
