@@ -45,6 +45,11 @@ constexpr int kStageBytes = 4 * kHalfTileBytes;       // K lo, K hi, V lo, V hi
 constexpr int kItemSlots = 3;
 constexpr int kOStride = kHeadDim + 4;                 // padded merge row (floats)
 constexpr int kEntries = 256;                          // stage entries in flight (power of 2)
+// Queued stages left when the scheduler claims a CTA's next item from the
+// shared counter (a build-time tuning constant).
+#ifndef SEER_DECODE_CLAIM_AHEAD
+#define SEER_DECODE_CLAIM_AHEAD 6
+#endif
 
 // The two-slot shapes hand each finished item's merge to warps of their own
 // (in the single-launch step they also take part in the gate phase and the
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(
     // hide the claim's round trips), so a CTA never sits on claimed items
     // while another runs dry and the CTAs finish together.
     const bool dyn = p.work_counter != nullptr;
-    constexpr uint32_t kClaimAhead = 4;
+    constexpr uint32_t kClaimAhead = SEER_DECODE_CLAIM_AHEAD;
     // single-launch step: a row's indices are read only once its gate row has
     // published them (bounded wait on the row flag, acquire)
     auto row_ready = [&](int bh) {
