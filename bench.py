@@ -498,6 +498,8 @@ def resolve_workload(args):
     w = W.WORKLOADS[args.workload]
     if args.sparsity is not None:
         w = w.replace(sparsity_permille=args.sparsity, budget_tokens=None)
+    if args.batch is not None:   # a smaller case of the same workload (profiler captures)
+        w = w.replace(batch=args.batch)
     return w
 
 
@@ -1094,6 +1096,8 @@ def main(argv=None):
     from block_sparse_attention_step_b200 import workloads as W
     p.add_argument("--workload", choices=sorted(W.WORKLOADS), default=W.HEADLINE)
     p.add_argument("--sparsity", type=int, default=None, help="override: sparsity in permille")
+    p.add_argument("--batch", type=int, default=None,
+                   help="override: batch size (a smaller case of the workload, e.g. for a capture)")
     p.add_argument("--splits", type=int, default=None)
     p.add_argument("--layout", choices=("nhd", "hnd"), default="nhd",
                    help="KV pool page layout: token-major [P][bs][Hkv][D] or head-major [P][Hkv][bs][D]")
