@@ -698,7 +698,10 @@ def run_ours(args):
         "step_us_percentiles": pct,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": recorded_traffic(w.name), "kernel": "sparse_decode_kernel",
+                     # the records are taken on each workload's own selection and batch
+                     "traffic": (recorded_traffic(w.name)
+                                 if args.sparsity is None and args.batch is None else None),
+                     "kernel": "sparse_decode_kernel",
                      "bytes_per_launch": dec_bytes, "peak_source": f"{peak_kind} hbm_gbs",
                      "peak_nominal": NOMINAL_HBM_GBS,
                      "frac_nominal": achieved / NOMINAL_HBM_GBS},
