@@ -4,12 +4,14 @@
 // fused step (rows of a persistent CTA, 320 threads):
 //   * optionally append the new token's K and V rows at position L - 1 of the
 //     paged cache (the step's KV append);
-//   * refresh the newest block's pooled key from K (the summation order of
-//     seer_pool_keys) and write it back to kbar;
 //   * g = gate_scale * W[h] qbar, qbar the mean of the group's queries;
+//   * refresh the newest block's pooled key from K (the summation order of
+//     seer_pool_keys; the appended token read from the new row itself) and
+//     write it back to kbar;
 //   * stream the kbar row through a ring of NBUF chunk buffers (bulk copies
-//     on mbarriers) and score every block, 8 rows per worker warp per chunk
-//     in one reduction that gives the same bits as warp_dot4 row by row;
+//     on mbarriers; the first goes out as soon as the row length is known)
+//     and score every block, 8 rows per worker warp per chunk in one
+//     reduction that gives the same bits as warp_dot4 row by row;
 //   * select the top-k with the exact value-binned select (or stop after the
 //     scores when the unified cross-head select follows).
 // Results are identical to seer_pool_keys (incremental), seer_gate_scores and
@@ -22,44 +24,21 @@
 
 namespace seer {
 
-// Shared-memory scratch of a gate row besides the chunk buffers.  part,
-// newest, qbar and gvec are read and written as float4: the struct and those
-// members sit on 16-byte boundaries.  The pooling partials are consumed
-// before the first score is written, so they share the scores' space.
+// Shared-memory scratch of a gate row besides the chunk buffers and the
+// pooling partials.  newest, qbar and gvec are read and written as float4:
+// the struct and those members sit on 16-byte boundaries.
 struct alignas(16) GateRowScratch {
-  union {
-    float scores[kMaxBlocks];
-    float part[kPoolWarps * kHeadDim];
-  };
+  float scores[kMaxBlocks];
   float newest[kHeadDim];
   float qbar[kHeadDim];
   float gvec[kHeadDim];
   SelectSmem sel;
 };
-static_assert(offsetof(GateRowScratch, part) % 16 == 0 &&
-                  offsetof(GateRowScratch, newest) % 16 == 0 &&
+static_assert(offsetof(GateRowScratch, newest) % 16 == 0 &&
                   offsetof(GateRowScratch, qbar) % 16 == 0 &&
                   offsetof(GateRowScratch, gvec) % 16 == 0 &&
                   offsetof(GateRowScratch, sel) % 8 == 0,
               "float4 members of the gate scratch on 16-byte boundaries");
-
-// Same rows and summation order as pool_warp_partial, through L2 (the row
-// appended by this CTA a moment ago must not come from a stale read-only
-// cache line).
-__device__ __forceinline__ float4 pool_warp_partial_l2(const uint16_t* base_lane,
-                                                       int64_t stride_token, int valid,
-                                                       int warp) {
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 16
-  for (int t = warp; t < valid; t += kPoolWarps) {
-    const uint2 v = __ldcg(reinterpret_cast<const uint2*>(base_lane + (int64_t)t * stride_token));
-    a0 += __uint_as_float(v.x << 16);
-    a1 += __uint_as_float(v.x & 0xffff0000u);
-    a2 += __uint_as_float(v.y << 16);
-    a3 += __uint_as_float(v.y & 0xffff0000u);
-  }
-  return make_float4(a0, a1, a2, a3);
-}
 
 // The kbar chunk buffers of a gate row: NBUF slots of CHUNK_ROWS rows each,
 // anywhere in shared memory (16-byte aligned).
@@ -83,33 +62,44 @@ struct ChunkRing {
 // Returns false when a wait ran out (SEER_DEV_TIMEOUT is flagged).
 template <int THREADS, int WORKERS, int NBUF, int QFIRST, int QTHREADS, int R8 = 1>
 __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRing<NBUF>& ring,
-                         uint64_t* bars, uint32_t& seq, GateRowScratch& gs, int next_b = -1,
-                         int next_h = 0, uint32_t* ahead = nullptr) {
+                         uint64_t* bars, uint32_t& seq, GateRowScratch& gs, float* part,
+                         int next_b = -1, int next_h = 0, uint32_t* ahead = nullptr) {
   constexpr int CHUNK_ROWS = 8 * R8 * WORKERS;
   constexpr int kWRows = kHeadDim / WORKERS;  // W rows per worker warp
+  constexpr int kPoolRows = 128 / kPoolWarps;  // newest-block tokens per pooling warp (bs <= 128)
+  // With 16 or more warps each newest-block token row is split between two
+  // warps (dims 0..63 and 64..127), so each lane holds half as many words.
+  constexpr int kPoolSplit = THREADS / 32 >= 2 * kPoolWarps ? 2 : 1;
+  constexpr int kPoolWords = 2 / kPoolSplit;  // 32-bit words (bf16 pairs) per lane per token
   static_assert(THREADS % 32 == 0 && THREADS / 32 >= kPoolWarps, "pooling uses 8 warps");
   static_assert(WORKERS * 32 <= THREADS && kWRows % 8 == 0, "8 W rows per reduction");
   static_assert(kHeadDim % QTHREADS == 0 && QFIRST + QTHREADS <= THREADS, "mean query threads");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t bh = (int64_t)b * p.Hkv + h;
+  // Loads that need nothing else go out first: the row lengths, this warp's
+  // rows of W[h] (rows warp + WORKERS * i) and, below, the group's queries.
   int L = __ldg(p.seqlens + b);
+  const int Ln = next_b >= 0 ? __ldg(p.seqlens + next_b) : 0;
+  const int k_row = __ldg(p.k_per_seq + b);
+  float4 wrow[kWRows];
+  if (warp < WORKERS) {
+    const float* W = p.w_gate + (int64_t)h * kHeadDim * kHeadDim;
+#pragma unroll
+    for (int r = 0; r < kWRows; ++r)
+      wrow[r] = __ldg(reinterpret_cast<const float4*>(W + (warp + r * WORKERS) * kHeadDim +
+                                                      4 * lane));
+  }
   L = max(0, min(L, p.max_blocks * p.bs));
   const int nb = ceil_div_i(L, p.bs);
   const int nchunks = ceil_div_i(nb, CHUNK_ROWS);
   float* kb_row = p.kbar + bh * p.max_blocks * kHeadDim;
-  const int k_row = __ldg(p.k_per_seq + b);
   bool ok = true;
   // the chunk stream: this row's chunks, then the next row's
-  int next_nb = 0;
-  const float* next_kb = nullptr;
-  if (next_b >= 0) {
-    const int Ln = max(0, min(__ldg(p.seqlens + next_b), p.max_blocks * p.bs));
-    next_nb = ceil_div_i(Ln, p.bs);
-    next_kb = p.kbar + ((int64_t)next_b * p.Hkv + next_h) * p.max_blocks * kHeadDim;
-  }
+  const int next_nb = next_b >= 0 ? ceil_div_i(max(0, min(Ln, p.max_blocks * p.bs)), p.bs) : 0;
+  const float* next_kb =
+      next_b >= 0 ? p.kbar + ((int64_t)next_b * p.Hkv + next_h) * p.max_blocks * kHeadDim : nullptr;
   const int stream_len = nchunks + ceil_div_i(next_nb, CHUNK_ROWS);
   const uint32_t first = ahead != nullptr ? *ahead : 0u;  // already issued
-  uint32_t issued = first;
   auto issue = [&](int u) {  // position u of the stream into slot (seq + u) % NBUF
     const uint32_t slot = (seq + u) % NBUF;
     const bool own = u < nchunks;
@@ -120,57 +110,35 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
     bulk_copy_g2s(ring.slot[slot], (own ? kb_row : next_kb) + (int64_t)c * CHUNK_ROWS * kHeadDim,
                   bytes, &bars[slot]);
   };
-
-  // The first chunk goes out before anything else; the other free slots
-  // (this row's own chunks, then, if the row is short, the next row's) are
-  // filled once the loads that form g below have returned.  One chunk per
-  // row already keeps HBM busy across the grid, and the few loads that g
-  // needs would otherwise queue behind every row's whole first burst.
+  // One chunk goes out as soon as the lengths are in; the other free slots
+  // are filled once the newest block's K loads below are on their way, so
+  // that those loads queue behind one chunk per row, not behind the whole
+  // burst (g's own loads left before any of it).
   constexpr int kBurst = 1;
   if (tid == 0)
     for (int u = (int)first; u < kBurst && u < stream_len; ++u) issue(u);
+  uint32_t issued = (uint32_t)max((int)first, min(NBUF, stream_len));
 
-  // KV append: the new token's K and V rows of head h at position L - 1
+  // The newest block's page: the KV append writes the new token's K and V
+  // rows of head h into it (position L - 1), and its pooled key is
+  // refreshed from K below.
   const bool append = p.k_new != nullptr && L > 0;
+  const bool refresh = p.incremental && nb > 0;
+  const int valid_new = refresh ? L - (nb - 1) * p.bs : 0;
+  int64_t new_page = 0;
   bool bad_page = false;
-  if (append) {
-    const int64_t page = page_of(p.page_table, b, (L - 1) / p.bs, p.max_blocks);
-    bad_page = page < 0 || page >= p.num_pages;
-    if (warp == 0 && !bad_page) {
-      const int64_t off = page * p.stride_page + (int64_t)((L - 1) % p.bs) * p.stride_token +
-                          (int64_t)h * p.stride_head + 4 * lane;
-      const int64_t src = ((int64_t)b * p.Hkv + h) * kHeadDim + 4 * lane;
-      *reinterpret_cast<uint2*>(p.k_pool_w + off) = __ldg(reinterpret_cast<const uint2*>(p.k_new + src));
-      *reinterpret_cast<uint2*>(p.v_pool_w + off) = __ldg(reinterpret_cast<const uint2*>(p.v_new + src));
-    }
-    __syncthreads();  // the pooled-key refresh below reads the appended row
+  if (append || refresh) {
+    new_page = page_of(p.page_table, b, nb - 1, p.max_blocks);
+    bad_page = new_page < 0 || new_page >= p.num_pages;
+  }
+  if (append && warp == 0 && !bad_page) {
+    const int64_t off = new_page * p.stride_page + (int64_t)((L - 1) % p.bs) * p.stride_token +
+                        (int64_t)h * p.stride_head + 4 * lane;
+    const int64_t src = bh * kHeadDim + 4 * lane;
+    *reinterpret_cast<uint2*>(p.k_pool_w + off) = __ldg(reinterpret_cast<const uint2*>(p.k_new + src));
+    *reinterpret_cast<uint2*>(p.v_pool_w + off) = __ldg(reinterpret_cast<const uint2*>(p.v_new + src));
   }
 
-  // newest block's pooled key (incremental update), warps 0..7
-  const bool refresh = p.incremental && nb > 0;
-  int valid_new = 0;
-  if (refresh) {
-    valid_new = L - (nb - 1) * p.bs;
-    const int64_t page = page_of(p.page_table, b, nb - 1, p.max_blocks);
-    const bool bad = page < 0 || page >= p.num_pages;
-    bad_page |= bad;
-    if (warp < kPoolWarps && !bad) {
-      const uint16_t* base =
-          p.k_pool + page * p.stride_page + (int64_t)h * p.stride_head + 4 * lane;
-      const float4 a = append ? pool_warp_partial_l2(base, p.stride_token, valid_new, warp)
-                              : pool_warp_partial(base, p.stride_token, valid_new, warp);
-      *reinterpret_cast<float4*>(&gs.part[warp * kHeadDim + 4 * lane]) = a;
-    }
-  }
-  // this warp's rows of W[h] (rows warp + WORKERS * i), in flight meanwhile
-  float4 wrow[kWRows];
-  if (warp < WORKERS) {
-    const float* W = p.w_gate + (int64_t)h * kHeadDim * kHeadDim;
-#pragma unroll
-    for (int r = 0; r < kWRows; ++r)
-      wrow[r] = __ldg(reinterpret_cast<const float4*>(W + (warp + r * WORKERS) * kHeadDim +
-                                                      4 * lane));
-  }
   // mean query of the group (q in mapped host memory: read through L2 and
   // copied to q_copy for the decode)
   if (tid >= QFIRST && tid < QFIRST + QTHREADS) {
@@ -193,16 +161,60 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
       gs.qbar[d] = s / (float)p.G;
     }
   }
-  __syncthreads();
+  // The newest block's K rows go out now, behind one chunk per row: token t
+  // to warp t % 8 (+ 8 for the upper half of the dims when split), lane l to
+  // dims 4l .. 4l+3 (2l, 2l+1 of its half when split).  The appended token is
+  // read from k_new itself, so no barrier has to order the append before
+  // these loads.
+  const int pool_warp = warp % kPoolWarps;
+  const int pool_dim = (warp / kPoolWarps) * (kHeadDim / kPoolSplit) + 2 * kPoolWords * lane;
+  const bool pooler = refresh && warp < kPoolWarps * kPoolSplit && !bad_page;
+  uint32_t knew[kPoolRows][kPoolWords];
+  if (pooler) {
+    const uint16_t* base = p.k_pool + new_page * p.stride_page + (int64_t)h * p.stride_head + pool_dim;
+    const uint16_t* appended = append ? p.k_new + bh * kHeadDim + pool_dim : nullptr;
+#pragma unroll
+    for (int i = 0; i < kPoolRows; ++i) {
+      const int t = pool_warp + i * kPoolWarps;
+      const uint16_t* src =
+          (append && t == valid_new - 1) ? appended : base + (int64_t)t * p.stride_token;
+      if constexpr (kPoolWords == 2) {
+        const uint2 v = t < valid_new ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0u, 0u);
+        knew[i][0] = v.x;
+        knew[i][1] = v.y;
+      } else {
+        knew[i][0] = t < valid_new ? __ldg(reinterpret_cast<const uint32_t*>(src)) : 0u;
+      }
+    }
+  }
+  // the newest block's mean over its valid tokens, summed in the order of
+  // seer_pool_keys (per dim: the tokens of each residue mod 8 in order, then
+  // the 8 partials in order), and written back to kbar
+  auto pool_sum = [&]() {
+    if (!pooler) return;
+    float a[2 * kPoolWords] = {};
+#pragma unroll
+    for (int i = 0; i < kPoolRows; ++i) {
+      if (pool_warp + i * kPoolWarps < valid_new) {
+#pragma unroll
+        for (int w = 0; w < kPoolWords; ++w) {
+          a[2 * w] += __uint_as_float(knew[i][w] << 16);
+          a[2 * w + 1] += __uint_as_float(knew[i][w] & 0xffff0000u);
+        }
+      }
+    }
+    float* dst = &part[pool_warp * kHeadDim + pool_dim];
+    if constexpr (kPoolWords == 2)
+      *reinterpret_cast<float4*>(dst) = make_float4(a[0], a[1], a[2], a[3]);
+    else
+      *reinterpret_cast<float2*>(dst) = make_float2(a[0], a[1]);
+  };
+  // Without the split the words would stay live across the projection: the
+  // warps sum them as soon as they arrive instead.
+  if constexpr (kPoolSplit == 1) pool_sum();
+  __syncthreads();  // qbar
   if (tid == 0)
     for (int u = max((int)first, kBurst); u < NBUF && u < stream_len; ++u) issue(u);
-  issued = (uint32_t)max((int)first, min(NBUF, stream_len));
-  if (refresh && tid < kHeadDim) {
-    float v = 0.f;
-    if (!bad_page) v = pool_finish(gs.part, tid, valid_new);
-    gs.newest[tid] = v;
-    kb_row[(int64_t)(nb - 1) * kHeadDim + tid] = v;
-  }
   if (bad_page && tid == 0) flag_status(p.status, SEER_DEV_BAD_PAGE);
   // g = gate_scale * W[h] qbar, 8 rows per reduction
   if (warp < WORKERS) {
@@ -217,7 +229,16 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
         gs.gvec[warp + (g8 * 8 + ((lane >> 2) & 7)) * WORKERS] = __fmul_rn(v, p.gate_scale);
     }
   }
+  if constexpr (kPoolSplit == 2) pool_sum();
   __syncthreads();
+  if (refresh) {
+    if (tid < kHeadDim) {
+      const float v = bad_page ? 0.f : pool_finish(part, tid, valid_new);
+      gs.newest[tid] = v;
+      kb_row[(int64_t)(nb - 1) * kHeadDim + tid] = v;
+    }
+    __syncthreads();
+  }
 
   // scores, chunk by chunk; thread 0 refills each buffer once it is read
   const float4 gv = *reinterpret_cast<const float4*>(&gs.gvec[4 * lane]);

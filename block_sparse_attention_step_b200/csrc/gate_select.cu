@@ -4,9 +4,10 @@
 // the scores through HBM and without two of the step's launches.
 //
 // Each CTA (512 threads, one per SM) streams its kbar row (NB x 512 bytes)
-// through three 64 KB shared-memory buffers with bulk copies, issued before
-// the gate projection g = W qbar is formed so the projection hides under the
-// first copies.  (Measured and dropped: 256-thread CTAs with 24 KB buffers,
+// through three 64 KB shared-memory buffers with bulk copies: the first as
+// soon as the row length is in, the others right after the newest block's K
+// loads (so those queue behind one chunk, not three), all before the gate
+// projection g = W qbar is formed, which hides under the copies.  (Measured and dropped: 256-thread CTAs with 24 KB buffers,
 // two per SM, for batches with more rows than SMs -- 5 % slower on the
 // ragged batch, 60 % slower on the headline one; and each 64 KB chunk cut
 // into 4-16 KB bulk copies -- slower at every size.)  The
@@ -27,9 +28,11 @@ constexpr int kGSBuffers = 3;
 struct GateSelectSmem {
   float buf[kGSBuffers][kGSChunkRows * kHeadDim];  // kbar rows in flight
   GateRowScratch row;                              // 16-byte aligned (float4 members)
+  float part[kPoolWarps * kHeadDim];               // newest-block pooling partials
   uint64_t bar[kGSBuffers];
 };
-static_assert(offsetof(GateSelectSmem, row) % 16 == 0 && offsetof(GateSelectSmem, bar) % 8 == 0,
+static_assert(offsetof(GateSelectSmem, row) % 16 == 0 && offsetof(GateSelectSmem, part) % 16 == 0 &&
+                  offsetof(GateSelectSmem, bar) % 8 == 0,
               "gate kernel shared-memory carve alignment");
 
 __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSelectParams p) {
@@ -51,7 +54,8 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
     p.work_counter[threadIdx.x] = 0u;
   uint32_t seq = 0;
   const ChunkRing<kGSBuffers> ring = {{sm.buf[0], sm.buf[1], sm.buf[2]}};
-  gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(p, b, h, ring, sm.bar, seq, sm.row);
+  gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(p, b, h, ring, sm.bar, seq, sm.row,
+                                                              sm.part);
 }
 
 // The same rows for batches with more (b, h) rows than SMs: one persistent
@@ -87,7 +91,7 @@ __global__ void __launch_bounds__(kGSThreads, 1)
     __syncthreads();
     const int nxt = next_row;
     gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(
-        p, row / p.Hkv, row % p.Hkv, ring, sm.bar, seq, sm.row, nxt >= 0 ? nxt / p.Hkv : -1,
+        p, row / p.Hkv, row % p.Hkv, ring, sm.bar, seq, sm.row, sm.part, nxt >= 0 ? nxt / p.Hkv : -1,
         nxt >= 0 ? nxt % p.Hkv : 0, &ahead);
     __syncthreads();  // next_row is rewritten for the following row
     row = nxt >= 0 ? nxt : rows;

@@ -360,6 +360,11 @@ __global__ void __launch_bounds__(
     uint64_t* gbar = reinterpret_cast<uint64_t*>(smem + Shape::kGateBars);
     constexpr int kR8 = Shape::kGateR8;
     constexpr size_t kChunkBytes = (size_t)kR8 * kStageBytes;  // 8 * R8 * 8 warps rows
+    // the pooling partials of the newest block go to the query-row slots,
+    // which the scheduler fills only once the decode starts
+    static_assert((size_t)kItemSlots * Shape::kQSlotBytes >= (size_t)kPoolWarps * kHeadDim * 4,
+                  "pooling partials fit in the query-row slots");
+    float* gpart = reinterpret_cast<float*>(smem + Shape::kQBuf);
     ChunkRing<kSlots> gring;
 #pragma unroll
     for (int i = 0; i < kSlots - 1; ++i)
@@ -376,7 +381,8 @@ __global__ void __launch_bounds__(
     for (int row = blockIdx.x; row < rows; row += gridDim.x) {
       const int nxt = row + (int)gridDim.x;  // this CTA's next row: its kbar streams in early
       gate_row<Shape::kThreads, kMathWarps, kSlots, kMathThreads, 64, kR8>(
-          f.gate, row / p.Hkv, row % p.Hkv, gring, gbar, gseq, gs, nxt < rows ? nxt / p.Hkv : -1,
+          f.gate, row / p.Hkv, row % p.Hkv, gring, gbar, gseq, gs, gpart,
+          nxt < rows ? nxt / p.Hkv : -1,
           nxt < rows ? nxt % p.Hkv : 0, &gahead);
       __syncthreads();  // the row's indices, kbar row and appended K/V are written
       if (threadIdx.x == 0) {
