@@ -35,6 +35,19 @@ static_assert(offsetof(GateSelectSmem, row) % 16 == 0 && offsetof(GateSelectSmem
                   offsetof(GateSelectSmem, bar) % 8 == 0,
               "gate kernel shared-memory carve alignment");
 
+// Publishes row bh (after a barrier that follows its gate row): its indices,
+// kbar row, appended K/V row and query copy are visible to the decode grid,
+// whose TMA and bulk copies read the last two, once the flag is.  The epoch
+// does not move before every row is out (the decode grid's last CTA
+// advances it).
+__device__ __forceinline__ void publish_row(const GateSelectParams& p, int bh) {
+  if (p.row_flag == nullptr || threadIdx.x != 0) return;
+  const uint32_t value = *reinterpret_cast<const volatile uint32_t*>(p.epoch) + 1u;
+  __threadfence();
+  fence_proxy_async_global();
+  st_release_gpu(p.row_flag + bh, value);
+}
+
 __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSelectParams p) {
   extern __shared__ uint8_t gs_raw[];
   GateSelectSmem& sm = *reinterpret_cast<GateSelectSmem*>(
@@ -56,11 +69,15 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
   const ChunkRing<kGSBuffers> ring = {{sm.buf[0], sm.buf[1], sm.buf[2]}};
   gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(p, b, h, ring, sm.bar, seq, sm.row,
                                                               sm.part);
+  if (p.row_flag != nullptr) {
+    __syncthreads();  // every thread's writes of the row come before the flag
+    publish_row(p, b * p.Hkv + h);
+  }
 }
 
 // The same rows for batches with more (b, h) rows than SMs: one persistent
-// CTA per SM gates row after row, claiming the next row (a counter zeroed
-// before the launch) while it starts the current one, and keeps one kbar
+// CTA per SM gates row after row, claiming the next row (a counter at zero
+// when the launch starts) while it starts the current one, and keeps one kbar
 // chunk stream across its rows -- the next row's first chunks are in flight
 // while this one finishes and selects, and no CTA start-up or drain sits
 // between rows.
@@ -93,8 +110,18 @@ __global__ void __launch_bounds__(kGSThreads, 1)
     gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(
         p, row / p.Hkv, row % p.Hkv, ring, sm.bar, seq, sm.row, sm.part, nxt >= 0 ? nxt / p.Hkv : -1,
         nxt >= 0 ? nxt % p.Hkv : 0, &ahead);
-    __syncthreads();  // next_row is rewritten for the following row
+    __syncthreads();  // next_row is rewritten for the following row; the row is out
+    publish_row(p, row);
     row = nxt >= 0 ? nxt : rows;
+  }
+  // the last CTA past its final claim puts the claiming words back to zero
+  // for the next launch that shares them
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.row_done, 1u) == gridDim.x - 1) {
+      atomicExch(p.row_counter, 0u);
+      atomicExch(p.row_done, 0u);
+    }
   }
 }
 

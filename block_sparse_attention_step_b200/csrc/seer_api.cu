@@ -582,16 +582,28 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
   g.k_max = a->k_max;
   g.force_newest = a->force_newest ? 1 : 0;
   g.gate_scale = a->gate_scale;
-  g.work_counter = w.work_counter;  // zeroed by the gate grid for the decode grid
   g.scores_only = a->unified_heads ? 1 : 0;
   g.B = d->batch;
-  g.row_counter = w.work_counter + 5;
   const int num_sms = num_sms_current();
+  // More rows than SMs: a persistent row-claiming gate grid, whose rows finish
+  // one after another over the whole gate phase.  Each row then publishes a
+  // flag and the decode grid starts on it at once instead of waiting for the
+  // whole gate grid (the unified select, a grid of its own, keeps the wait).
+  // With one row per CTA the rows finish within a few microseconds of each
+  // other and the grid-wide wait is cheaper than the per-row protocol.
+  const bool rows_grid = (int64_t)d->batch * d->num_kv_heads > num_sms;
+  const bool row_flags = rows_grid && !a->unified_heads;
+  // the decode's item counter: at rest from the last launch (or
+  // seer_step_workspace_init); without row flags the gate grid also zeroes
+  // it, before the decode grid reads it
+  g.work_counter = row_flags ? nullptr : w.work_counter;
+  g.row_flag = row_flags ? w.row_flag : nullptr;
+  g.epoch = w.work_counter + 2;
+  g.row_counter = w.work_counter + 5;  // the row-claiming grid's counter and
+  g.row_done = w.work_counter + 6;     // its CTAs done (the last resets both)
   {
     NvtxRange r("gate_select");
-    if ((int64_t)d->batch * d->num_kv_heads > num_sms) {
-      // more rows than SMs: persistent row-claiming gate (its counter starts at 0)
-      SEER_CUDA(cudaMemsetAsync(g.row_counter, 0, sizeof(uint32_t), stream));
+    if (rows_grid) {
       SEER_CUDA(run_gate_select_rows(g, num_sms, stream, true));
     } else {
       SEER_CUDA(run_gate_select(g, d->batch, stream, true));
@@ -616,7 +628,9 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
   // a3, then a4; each grid launches early and waits for its predecessor
   {
     NvtxRange r("sparse_decode");
-    SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, true));
+    SEER_CUDA(run_sparse_decode(L.tk, L.tv, L.p, num_sms_current(), stream, true,
+                                row_flags ? w.work_counter : nullptr,
+                                row_flags ? w.row_flag : nullptr));
   }
   CombineParams c = {};
   c.o_part = w.o_part;

@@ -60,10 +60,16 @@ struct GateSelectParams {
   uint32_t* work_counter;  // optional: zeroed for the decode grid that follows
   int B;
   uint32_t* row_counter;   // the row-claiming gate grid's counter (zero before it starts)
+  uint32_t* row_done;      // its CTAs done; the last one puts both back to zero
   // optional: q is then host memory mapped into the device's address space,
   // and each gate row copies its group's query rows into q_copy (device) for
   // the decode grid
   uint16_t* q_copy;
+  // optional: each row publishes row_flag[bh] = epoch[0] + 1 once its
+  // selection, appended K/V row and query copy are out (the decode grid that
+  // follows then waits per row, not for the whole gate grid)
+  uint32_t* row_flag;
+  const uint32_t* epoch;
 };
 
 struct DecodeParams {
@@ -117,11 +123,14 @@ cudaError_t run_prefill_attention(const CUtensorMap& tq, const CUtensorMap& tk,
                                   cudaStream_t stream);
 
 // The single-launch step: the decode kernel with the gate rows before it and
-// the combine after it, in one cooperative grid.  Control words (zero before
-// the first launch; every completed launch leaves them ready for the next):
+// the combine after it, in one cooperative grid.  Control words of a step
+// workspace (zero before the first launch; every completed launch leaves
+// them ready for the next):
 //   ctl[0] next item, ctl[1] schedulers done (the decode's item counter),
 //   ctl[2] launch epoch, ctl[3] CTAs done decoding, ctl[4] CTAs done
-//   combining; row_flag[bh] = epoch + 1 once row bh's selection is out.
+//   combining, ctl[5] next row and ctl[6] CTAs done of the row-claiming gate
+//   grid; row_flag[bh] = epoch + 1 once row bh's selection is out (this
+//   step, or a per-stage step whose gate grid publishes rows).
 struct FusedParams {
   GateSelectParams gate;
   uint32_t* ctl;
@@ -160,8 +169,12 @@ cudaError_t run_fill_k(const int32_t* seqlens, int B, int bs, int permille, int 
                        int32_t* k_out, cudaStream_t stream);
 cudaError_t run_fused_step(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                            const FusedParams& f, int num_sms, cudaStream_t stream);
+// ctl / row_flag (optional): the step workspace's control words and row
+// flags published by the gate grid before it; nullptr: wait for the whole
+// preceding grid.
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
-                              int num_sms, cudaStream_t stream, bool pdl);
+                              int num_sms, cudaStream_t stream, bool pdl,
+                              uint32_t* ctl = nullptr, uint32_t* row_flag = nullptr);
 cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream, bool pdl);
 cudaError_t run_block_mass(const MassParams& p, int B, cudaStream_t stream);
 

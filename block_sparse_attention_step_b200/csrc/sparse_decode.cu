@@ -38,6 +38,8 @@
 #include "gate_row.cuh"
 #include "combine_core.cuh"
 
+#include <type_traits>
+
 namespace seer {
 
 constexpr int kHalfTileBytes = kTileTokens * 64 * 2;  // 64 tokens x 64 dims bf16
@@ -147,14 +149,18 @@ __device__ __forceinline__ ItemCoord item_coord(const DecodeParams& p, int item,
   return c;
 }
 
-template <bool FUSED>
+// Index rows written while this grid runs (by its own gate rows, or by a
+// gate grid that publishes each row) must come through L2.
+template <bool CONCURRENT>
 __device__ __forceinline__ int ld_row_data(const int32_t* ptr) {
-  // rows written by other CTAs of the same grid must come through L2
-  if constexpr (FUSED) return __ldcg(ptr);
+  if constexpr (CONCURRENT) return __ldcg(ptr);
   else return __ldg(ptr);
 }
 
-template <int NT, int STAGES, int MSLOTS, bool MASS, bool FUSED>
+// ROWFLAGS: the per-stage decode after a gate grid that publishes each row
+// (f.ctl and f.row_flag set); the single-launch step (FUSED) always works
+// with row flags.
+template <int NT, int STAGES, int MSLOTS, bool MASS, bool FUSED, bool ROWFLAGS>
 __global__ void __launch_bounds__(
     DecodeShape<NT, STAGES, MSLOTS, merge_warps(MSLOTS, FUSED)>::kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -347,12 +353,22 @@ __global__ void __launch_bounds__(
   __syncthreads();
   // Everything above touches only shared memory; from here on the kernel reads
   // what the preceding kernel wrote (the index rows) and writes what it may
-  // still read (the partials), so wait for it, then let the next one launch.
-  pdl_wait();
+  // still read (the partials).  Without row flags it waits for the whole
+  // preceding grid.  With them (a gate grid that publishes each row) each
+  // row's indices are read after its flag, and the partials are safe as they
+  // are: the gate grid let this grid launch only after its own wait for the
+  // kernel before it, the previous step's combine.  Then let the next one
+  // launch.
+  constexpr bool kRowFlags = FUSED || ROWFLAGS;
+  if constexpr (!kRowFlags || FUSED) pdl_wait();
   pdl_launch_dependents();
 
-  // ---- single-launch step, phase A: the gate rows of this CTA (all threads)
   __shared__ uint32_t epoch_next;  // this launch's row-flag value
+  if constexpr (!FUSED && kRowFlags) {
+    if (threadIdx.x == 0) epoch_next = ld_volatile(f.ctl + 2) + 1u;
+    __syncthreads();
+  }
+  // ---- single-launch step, phase A: the gate rows of this CTA (all threads)
   if constexpr (FUSED) {
     constexpr int kSlots = Shape::kGateSlots;
     static_assert(kStageBytes == 8 * kMathWarps * kHeadDim * 4, "a stage holds one kbar chunk");
@@ -429,10 +445,10 @@ __global__ void __launch_bounds__(
     // while another runs dry and the CTAs finish together.
     const bool dyn = p.work_counter != nullptr;
     constexpr uint32_t kClaimAhead = SEER_DECODE_CLAIM_AHEAD;
-    // single-launch step: a row's indices are read only once its gate row has
+    // with row flags a row's indices are read only once its gate row has
     // published them (bounded wait on the row flag, acquire)
     auto row_ready = [&](int bh) {
-      if constexpr (FUSED) {
+      if constexpr (kRowFlags) {
         if (lane == 0 && ok) {
           const long long t0 = clock64();
           while (ld_acquire_gpu(f.row_flag + bh) != epoch_next) {
@@ -452,7 +468,7 @@ __global__ void __launch_bounds__(
       const int bh = item_bh(p, item);
       row_ready(bh);
       L_cur = __ldg(p.seqlens + bh / p.Hkv);
-      n_cur = ld_row_data<FUSED>(p.n_sel + bh);
+      n_cur = ld_row_data<kRowFlags>(p.n_sel + bh);
     }
     int it_no = 0;
     for (; item < p.num_items && ok; ++it_no) {
@@ -462,7 +478,7 @@ __global__ void __launch_bounds__(
         const int bh = item_bh(p, nxt);
         row_ready(bh);
         L_nxt = __ldg(p.seqlens + bh / p.Hkv);
-        n_nxt = ld_row_data<FUSED>(p.n_sel + bh);
+        n_nxt = ld_row_data<kRowFlags>(p.n_sel + bh);
       }
       const ItemCoord ic = item_coord(p, item, L_cur, n_cur);
 
@@ -472,7 +488,7 @@ __global__ void __launch_bounds__(
         const int i = base + lane;
         int cnt = 0;
         if (i < ic.hi) {
-          const int j = ld_row_data<FUSED>(p.idx + ic.row + i);
+          const int j = ld_row_data<kRowFlags>(p.idx + ic.row + i);
           if (j >= 0 && j < ic.nb) cnt = ceil_div_i(min(p.bs, ic.L - j * p.bs), kTileTokens);
           if (base == ic.lo) j0 = j;
         }
@@ -502,7 +518,7 @@ __global__ void __launch_bounds__(
         const int i = base + lane;
         int j = -1, pg = 0, ne = 0;
         if (i < ic.hi) {
-          j = (base == ic.lo) ? j0 : ld_row_data<FUSED>(p.idx + ic.row + i);
+          j = (base == ic.lo) ? j0 : ld_row_data<kRowFlags>(p.idx + ic.row + i);
           if (j < 0 || j >= ic.nb) {
             flag_status(p.status, SEER_DEV_BAD_INDEX);
             j = -1;
@@ -570,7 +586,7 @@ __global__ void __launch_bounds__(
           const int bh = item_bh(p, nxt);
           row_ready(bh);
           L_nxt = __ldg(p.seqlens + bh / p.Hkv);
-          n_nxt = ld_row_data<FUSED>(p.n_sel + bh);
+          n_nxt = ld_row_data<kRowFlags>(p.n_sel + bh);
         }
       }
       item = nxt;
@@ -594,9 +610,9 @@ __global__ void __launch_bounds__(
       if (atomicAdd(p.work_counter + 1, 1u) == gridDim.x - 1) {
         atomicExch(p.work_counter, 0u);
         atomicExch(p.work_counter + 1, 0u);
-        // every CTA read the epoch before its gate rows: the next launch's
+        // every CTA read the epoch before its first row: the next launch's
         // flags use the next value
-        if constexpr (FUSED) atomicAdd(f.ctl + 2, 1u);
+        if constexpr (kRowFlags) atomicAdd(f.ctl + 2, 1u);
       }
     }
     // terminator (the copy thread stops on a negative page)
@@ -966,13 +982,13 @@ __global__ void __launch_bounds__(
 }
 
 // ------------------------------------------------------------------ launcher
-template <int NT, int STAGES, int MSLOTS, bool MASS, bool FUSED>
+template <int NT, int STAGES, int MSLOTS, bool MASS, bool FUSED, bool ROWFLAGS = false>
 static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
                                  const DecodeParams& p, const FusedParams& f, int num_sms,
                                  cudaStream_t stream, bool pdl) {
   using Shape = DecodeShape<NT, STAGES, MSLOTS, merge_warps(MSLOTS, FUSED)>;
   const size_t smem = FUSED ? Shape::smem_bytes_fused(p.G) : Shape::smem_bytes(p.G);
-  auto kern = sparse_decode_kernel<NT, STAGES, MSLOTS, MASS, FUSED>;
+  auto kern = sparse_decode_kernel<NT, STAGES, MSLOTS, MASS, FUSED, ROWFLAGS>;
   static std::atomic<uint64_t> smem_set{0};
   cudaError_t e = ensure_smem_limit(kern, smem_set);
   if (e != cudaSuccess) return e;
@@ -1001,25 +1017,46 @@ static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
   return cudaGetLastError();
 }
 
+template <int NT_, int MSLOTS_>
+struct ShapeTag {
+  static constexpr int kNT = NT_;
+  static constexpr int kMSlots = MSLOTS_;
+};
+
 // Two merge slots (no per-item rendezvous of the math warps) when shared
 // memory allows, else one.
 cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
-                              int num_sms, cudaStream_t stream, bool pdl) {
+                              int num_sms, cudaStream_t stream, bool pdl, uint32_t* ctl,
+                              uint32_t* row_flag) {
   int dev = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     optin = 227 * 1024;
   const bool mass = p.block_lse != nullptr;
-  const FusedParams none = {};
+  FusedParams fl = {};  // row flags only (and the epoch word they count from)
+  const bool flags = row_flag != nullptr && ctl != nullptr;
+  if (flags) {
+    fl.ctl = ctl;
+    fl.row_flag = row_flag;
+  }
+  auto go = [&](auto shape_tag, auto mass_tag, auto flags_tag) {
+    using T = decltype(shape_tag);
+    return launch_decode<T::kNT, 4, T::kMSlots, decltype(mass_tag)::value, false,
+                         decltype(flags_tag)::value>(tk, tv, p, fl, num_sms, stream, pdl);
+  };
+  auto pick = [&](auto shape_tag) {
+    if (mass)
+      return flags ? go(shape_tag, std::true_type{}, std::true_type{})
+                   : go(shape_tag, std::true_type{}, std::false_type{});
+    return flags ? go(shape_tag, std::false_type{}, std::true_type{})
+                 : go(shape_tag, std::false_type{}, std::false_type{});
+  };
   if (p.G <= 8) {
     if (DecodeShape<1, 4, 2>::smem_bytes(p.G) + 256 <= (size_t)optin)  // + static shared
-      return mass ? launch_decode<1, 4, 2, true, false>(tk, tv, p, none, num_sms, stream, pdl)
-                  : launch_decode<1, 4, 2, false, false>(tk, tv, p, none, num_sms, stream, pdl);
-    return mass ? launch_decode<1, 4, 1, true, false>(tk, tv, p, none, num_sms, stream, pdl)
-                : launch_decode<1, 4, 1, false, false>(tk, tv, p, none, num_sms, stream, pdl);
+      return pick(ShapeTag<1, 2>{});
+    return pick(ShapeTag<1, 1>{});
   }
-  return mass ? launch_decode<2, 4, 1, true, false>(tk, tv, p, none, num_sms, stream, pdl)
-              : launch_decode<2, 4, 1, false, false>(tk, tv, p, none, num_sms, stream, pdl);
+  return pick(ShapeTag<2, 1>{});
 }
 
 // The single-launch step (gate rows, decode, combine in one cooperative grid).

@@ -48,6 +48,12 @@ seer_status seer_decode_step_noalloc(const seer_dims* d, const seer_step_args* a
   seer_step_args b = *a;
   b.workspace = scratch;
   b.workspace_bytes = kScratchBytes;
+  // The control words sit at an offset that depends on the shape, k_max and
+  // split count, so a call after a differently shaped one would find other
+  // data there: zero them on the stream first.
+  const seer_status z =
+      seer_step_workspace_init(d, a->k_max, a->num_splits, scratch, kScratchBytes, stream);
+  if (z != SEER_OK) return z;
   return seer_decode_step(d, &b, stream);
 }
 

@@ -153,10 +153,10 @@ SEER_API int32_t seer_default_splits(const seer_dims *d, int32_t k_max,
 
 /* Bytes of caller workspace seer_decode_step needs (scores, idx, n_sel,
  * o_part, lse_part, then the control words: the decode grid's item counter,
- * the single-launch step's epoch and phase counters, and its [B][Hkv] u32
- * row flags;
- * each part 256-byte aligned).  seer_decode_step initialises what it uses;
- * seer_decode_step_fused needs seer_step_workspace_init once. */
+ * the row flags' epoch, the single-launch step's phase counters, the
+ * row-claiming gate grid's counters, and the [B][Hkv] u32 row flags;
+ * each part 256-byte aligned).  seer_decode_step and seer_decode_step_fused
+ * need seer_step_workspace_init once before a workspace's first use. */
 SEER_API size_t seer_step_workspace_bytes(const seer_dims *d, int32_t k_max,
                                  int32_t num_splits);
 
@@ -280,6 +280,18 @@ typedef struct seer_step_args {
   const uint16_t *v_new;
 } seer_step_args;
 
+/* The step: a0 (incremental when update_kbar = 1) + a1 + a2 in one gate grid
+ * (or a gate grid and the unified select), a3, a4.
+ *   - The workspace's control words must be zero before the first call:
+ *     seer_step_workspace_init once after allocating it (and again after a
+ *     call that flagged SEER_DEV_TIMEOUT).  Every completed call leaves them
+ *     ready for the next; calls that share a workspace must not overlap.
+ *   - With more (b, KV head) rows than SMs the gate grid is persistent and
+ *     claims rows one after another; then (without unified_heads) each row
+ *     publishes a flag in the workspace once its selection and KV append are
+ *     out, and the decode grid starts on that row at once instead of
+ *     waiting for the whole gate grid (bounded waits; SEER_DEV_TIMEOUT when
+ *     one runs out). */
 SEER_API seer_status seer_decode_step(const seer_dims *d, const seer_step_args *a,
                              seer_stream stream);
 
@@ -344,7 +356,8 @@ SEER_API seer_status seer_block_mass(const seer_dims *d, const int32_t *idx,
  * that must never enter the CUDA allocator (cudaMalloc can serialise against
  * other work and can fail under memory pressure mid-generation).
  *
- * It runs exactly seer_decode_step, but its workspace is a file-scope device
+ * It runs exactly seer_decode_step (its control words zeroed on the stream
+ * first), but its workspace is a file-scope device
  * array of SEER_NOALLOC_SCRATCH_BYTES (16 MiB) inside this library: every GPU
  * that loads the library holds those 16 MiB until the process exits.
  * a->workspace and a->workspace_bytes are ignored; the caller still passes
@@ -453,8 +466,8 @@ SEER_API seer_status seer_decode_step_fused(const seer_dims *d,
 
 /* Zeroes the control words of a step workspace (bytes from
  * seer_step_workspace_bytes with the same k_max and num_splits); enqueued on
- * `stream`.  Needed once before seer_decode_step_fused uses the workspace;
- * seer_decode_step itself needs no initialised workspace. */
+ * `stream`.  Needed once before seer_decode_step or seer_decode_step_fused
+ * uses the workspace. */
 SEER_API seer_status seer_step_workspace_init(const seer_dims *d, int32_t k_max,
                                               int32_t num_splits, void *workspace,
                                               size_t workspace_bytes,

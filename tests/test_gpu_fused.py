@@ -60,6 +60,8 @@ def test_fused_step_equals_per_stage_step(name, update_kbar):
     run.step(update_kbar=update_kbar)
     torch.cuda.synchronize()
     ref = _snapshot(run)
+    # the per-stage step advances the epoch too when its gate grid publishes rows
+    e0 = run.workspace_views()["ctl"].tolist()[2]
     for rep in range(3):  # successive launches on one workspace
         run.kbar.copy_(kbar0)
         run.out.zero_()
@@ -70,9 +72,9 @@ def test_fused_step_equals_per_stage_step(name, update_kbar):
         _assert_same(ref, _snapshot(run))
         v = run.workspace_views()
         ctl = v["ctl"].tolist()
-        assert ctl[:2] == [0, 0] and ctl[3:5] == [0, 0]    # counters at rest
-        assert ctl[2] == rep + 1                           # one epoch per launch
-        assert (v["row_flag"] == rep + 1).all()
+        assert ctl[:2] == [0, 0] and ctl[3:7] == [0, 0, 0, 0]   # counters at rest
+        assert ctl[2] == e0 + rep + 1                           # one epoch per launch
+        assert (v["row_flag"] == e0 + rep + 1).all()
 
 
 def _append_inputs(w, seed):

@@ -180,6 +180,40 @@ def test_step_many_rows_matches_standalone_stages(update_kbar):
     check_rows(w, data, run, rows, report)
 
 
+def test_step_row_flags_rest_and_repeat():
+    """More (b, h) rows than SMs: the persistent gate grid publishes each row
+    and the decode grid starts on it without waiting for the whole gate grid.
+    Over successive steps on one workspace the control words come back to
+    rest, the epoch advances by one per step, every row flag holds it, and the
+    output equals the standalone decode + combine over the step's own
+    indices, bit for bit (the decode read every row after it was out)."""
+    w = W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(
+        batch=80, q_heads=8, kv_heads=2, seqlen_range=(1, 45000), sparsity_permille=800)
+    data = W.generate(w, 29, DEV)
+    run = StepBuffers(w, data)
+    run.pool_full()
+    for rep in range(3):
+        run.step(update_kbar=1)
+        torch.cuda.synchronize()
+        assert run.status.item() == 0
+        v = run.workspace_views()
+        ctl = v["ctl"].tolist()
+        assert ctl[:2] == [0, 0] and ctl[3:7] == [0, 0, 0, 0]   # counters at rest
+        assert ctl[2] == rep + 1                                # one epoch per step
+        assert (v["row_flag"] == rep + 1).all()
+    o_part = torch.empty_like(v["o_part"])
+    lse_part = torch.empty_like(v["lse_part"])
+    out = torch.empty_like(run.out)
+    lse = torch.empty_like(run.lse)
+    seer.seer_sparse_decode(run.dims, data["q"], data["k_pool"], data["v_pool"], run.page_table,
+                            data["seqlens"], v["idx"], v["n_sel"], run.k_max, run.num_splits,
+                            run.scale, o_part, lse_part, run.status)
+    seer.seer_combine(run.dims, o_part, lse_part, run.num_splits, out, lse)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    assert torch.equal(out, run.out) and torch.equal(lse, run.lse)
+
+
 def test_step_incremental_kbar_matches_full_rebuild():
     """Run at L - 1 with a full rebuild, append the token at L - 1 (its K/V
     rows are already in the pool) with the incremental update, and compare
