@@ -41,7 +41,7 @@ static_assert(offsetof(GateSelectSmem, row) % 16 == 0 && offsetof(GateSelectSmem
 // does not move before every row is out (the decode grid's last CTA
 // advances it).
 __device__ __forceinline__ void publish_row(const GateSelectParams& p, int bh) {
-  if (p.row_flag == nullptr || threadIdx.x != 0) return;
+  if (p.row_flag == nullptr || bh < 0) return;
   const uint32_t value = *reinterpret_cast<const volatile uint32_t*>(p.epoch) + 1u;
   __threadfence();
   fence_proxy_async_global();
@@ -71,22 +71,21 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
                                                               sm.part);
   if (p.row_flag != nullptr) {
     __syncthreads();  // every thread's writes of the row come before the flag
-    publish_row(p, b * p.Hkv + h);
+    if (threadIdx.x == 0) publish_row(p, b * p.Hkv + h);
   }
 }
 
 // The same rows for batches with more (b, h) rows than SMs: one persistent
-// CTA per SM gates row after row, claiming the next row (a counter at zero
-// when the launch starts) while it starts the current one, and keeps one kbar
-// chunk stream across its rows -- the next row's first chunks are in flight
-// while this one finishes and selects, and no CTA start-up or drain sits
-// between rows.
+// CTA per SM gates row after row, claiming rows two ahead (a counter at zero
+// when the launch starts), and keeps one kbar chunk stream across its rows --
+// the next row's first chunks are in flight while this one finishes and
+// selects, and no CTA start-up or drain sits between rows.
 __global__ void __launch_bounds__(kGSThreads, 1)
     gate_select_rows_kernel(const GateSelectParams p) {
   extern __shared__ uint8_t gs_raw[];
   GateSelectSmem& sm = *reinterpret_cast<GateSelectSmem*>(
       (reinterpret_cast<uintptr_t>(gs_raw) + 127) & ~uintptr_t(127));
-  __shared__ int next_row;
+  __shared__ int next_rows[2];
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGSBuffers; ++i) mbar_init(&sm.bar[i], 1);
     fence_mbar_init();
@@ -99,21 +98,35 @@ __global__ void __launch_bounds__(kGSThreads, 1)
   const int rows = p.B * p.Hkv;
   const ChunkRing<kGSBuffers> ring = {{sm.buf[0], sm.buf[1], sm.buf[2]}};
   uint32_t seq = 0, ahead = 0;
-  int row = blockIdx.x;
-  while (row < rows) {
-    if (threadIdx.x == 0) {
-      const unsigned v = atomicAdd(p.row_counter, 1u) + gridDim.x;
-      next_row = v < (unsigned)rows ? (int)v : -1;
+  // Rows are claimed two ahead: the claim of the row after next goes out as a
+  // row starts and is read when the next one starts, so its round trip hides
+  // under a whole row (thread 0 holds it in `pending`).
+  unsigned pending = 0xffffffffu;
+  if (threadIdx.x == 0) {
+    const unsigned v = atomicAdd(p.row_counter, 1u) + gridDim.x;
+    next_rows[0] = v < (unsigned)rows ? (int)v : -1;
+    if (v < (unsigned)rows) pending = atomicAdd(p.row_counter, 1u) + gridDim.x;
+  }
+  __syncthreads();
+  int row = blockIdx.x, prev = -1;
+  for (int it = 0; row < rows; ++it) {
+    const int nxt = next_rows[it & 1];
+    if (threadIdx.x == 0) {  // the row after nxt, and the claim after that one
+      const bool more = nxt >= 0 && pending < (unsigned)rows;
+      next_rows[(it + 1) & 1] = more ? (int)pending : -1;
+      pending = more ? atomicAdd(p.row_counter, 1u) + gridDim.x : 0xffffffffu;
     }
-    __syncthreads();
-    const int nxt = next_row;
+    // the previous row, out since the barrier that ended it; its fences run
+    // on warp 1 while the other warps start this row
+    if (threadIdx.x == 32) publish_row(p, prev);
     gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(
         p, row / p.Hkv, row % p.Hkv, ring, sm.bar, seq, sm.row, sm.part, nxt >= 0 ? nxt / p.Hkv : -1,
         nxt >= 0 ? nxt % p.Hkv : 0, &ahead);
-    __syncthreads();  // next_row is rewritten for the following row; the row is out
-    publish_row(p, row);
+    __syncthreads();  // the row is out; next_rows[(it + 1) & 1] is written
+    prev = row;
     row = nxt >= 0 ? nxt : rows;
   }
+  if (threadIdx.x == 32) publish_row(p, prev);
   // the last CTA past its final claim puts the claiming words back to zero
   // for the next launch that shares them
   if (threadIdx.x == 0) {
