@@ -148,6 +148,53 @@ def test_step_zero_query_ties_every_score(seqlen, force):
     check_rows(w, data, run, [(b, h) for b in range(2) for h in range(2)], report)
 
 
+KBAR_PATTERNS = ("periodic_ties", "all_equal", "nan_rows", "overflow", "signed_zero")
+
+
+@pytest.mark.parametrize("pattern", KBAR_PATTERNS)
+@pytest.mark.parametrize("rows_grid,force", [(False, False), (False, True), (True, True)])
+def test_step_select_on_adversarial_scores_matches_block_select(pattern, rows_grid, force):
+    """The gate row's select (one warp for rows of up to 512 blocks, the whole
+    CTA beyond) against the standalone block-wide select over the step's own
+    scores, bit for bit, on pooled keys crafted so that the scores tie
+    (periodic rows, every row equal), hold NaN, overflow to +-inf or NaN, or
+    are +-0; row lengths span 1 .. 600 blocks (both select forms), through the
+    one-row-per-CTA gate grid and the row-claiming one."""
+    batch = 40 if rows_grid else 6  # 40 x 4 = 160 (b, h) rows, more than the SMs
+    w = W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(
+        batch=batch, q_heads=16, kv_heads=4, seqlen_range=(1, 600 * 64), sparsity_permille=800,
+        force_newest=force)
+    data = W.generate(w, 31, DEV)
+    run = StepBuffers(w, data)
+    kb = run.kbar  # [B][Hkv][NBmax][D], used as is with update_kbar = 0
+    g = torch.Generator(device="cpu").manual_seed(3)
+    base = torch.randn(tuple(kb.shape), generator=g).to(DEV)
+    nbm = kb.shape[2]
+    if pattern == "periodic_ties":
+        kb.copy_(base[:, :, :7].repeat(1, 1, -(-nbm // 7), 1)[:, :, :nbm])
+    elif pattern == "all_equal":
+        kb.copy_(base[:, :, :1].expand_as(kb))
+    elif pattern == "nan_rows":
+        kb.copy_(base)
+        kb[:, :, ::5] = float("nan")
+    elif pattern == "overflow":
+        kb.copy_(base * 3e38)
+    else:
+        kb.copy_(torch.where(base > 0, torch.zeros_like(base), torch.full_like(base, -0.0)))
+    run.step(update_kbar=0)
+    torch.cuda.synchronize()
+    assert run.status.item() & seer.DEV_TIMEOUT == 0
+    v = run.workspace_views()
+    idx = torch.full_like(v["idx"], 77)
+    n_sel = torch.full_like(v["n_sel"], 77)
+    seer.seer_block_select(run.dims, v["scores"], data["seqlens"], run.k_per_seq, force,
+                           run.k_max, idx, n_sel, run.status)
+    torch.cuda.synchronize()
+    assert torch.equal(n_sel, v["n_sel"]) and torch.equal(idx, v["idx"])
+    nb = -(-data["seqlens"].cpu() // 64)
+    assert (nb > 512).any() and (nb <= 512).any()
+
+
 @pytest.mark.parametrize("update_kbar", [1, 2])
 def test_step_many_rows_matches_standalone_stages(update_kbar):
     """More (b, h) rows than SMs (the fused gate kernel runs in several waves):
