@@ -60,7 +60,12 @@ struct ChunkRing {
 // < 0: no next row), so the next row's data is on its way while this row
 // finishes and selects.
 // Returns false when a wait ran out (SEER_DEV_TIMEOUT is flagged).
-template <int THREADS, int WORKERS, int NBUF, int QFIRST, int QTHREADS, int R8 = 1>
+// SPEC_FIRST (a CTA that gates one row, nothing issued ahead): the first
+// chunk goes out before the row length is known -- min(CHUNK_ROWS, NBmax)
+// rows of the kbar row, all inside the kbar buffer, of which the row scores
+// its first nb -- and an empty row waits for it before returning.
+template <int THREADS, int WORKERS, int NBUF, int QFIRST, int QTHREADS, int R8 = 1,
+          bool SPEC_FIRST = false>
 __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRing<NBUF>& ring,
                          uint64_t* bars, uint32_t& seq, GateRowScratch& gs, float* part,
                          int next_b = -1, int next_h = 0, uint32_t* ahead = nullptr) {
@@ -76,6 +81,12 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
   static_assert(kHeadDim % QTHREADS == 0 && QFIRST + QTHREADS <= THREADS, "mean query threads");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t bh = (int64_t)b * p.Hkv + h;
+  if (SPEC_FIRST && tid == 0) {
+    const uint32_t bytes = (uint32_t)min(CHUNK_ROWS, p.max_blocks) * kHeadDim * 4;
+    mbar_arrive_expect_tx(&bars[seq % NBUF], bytes);
+    bulk_copy_g2s(ring.slot[seq % NBUF], p.kbar + bh * p.max_blocks * kHeadDim, bytes,
+                  &bars[seq % NBUF]);
+  }
   // Loads that need nothing else go out first: the row lengths, this warp's
   // rows of W[h] (rows warp + WORKERS * i) and, below, the group's queries.
   int L = __ldg(p.seqlens + b);
@@ -115,7 +126,7 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
   // that those loads queue behind one chunk per row, not behind the whole
   // burst (g's own loads left before any of it).
   constexpr int kBurst = 1;
-  if (tid == 0)
+  if (tid == 0 && !SPEC_FIRST)
     for (int u = (int)first; u < kBurst && u < stream_len; ++u) issue(u);
   uint32_t issued = (uint32_t)max((int)first, min(NBUF, stream_len));
 
@@ -281,6 +292,13 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
       if (tid == 0 && ok) issue(c + NBUF);
       issued = max(issued, (uint32_t)(c + NBUF + 1));
     }
+  }
+  if (SPEC_FIRST && nchunks == 0) {  // the early chunk of an empty row
+    if (ok && !mbar_wait(&bars[seq % NBUF], (seq / NBUF) & 1)) {
+      flag_status(p.status, SEER_DEV_TIMEOUT);
+      ok = false;
+    }
+    seq += 1;
   }
   seq += (uint32_t)nchunks;
   if (ahead != nullptr) *ahead = issued > (uint32_t)nchunks ? issued - (uint32_t)nchunks : 0u;

@@ -67,8 +67,8 @@ __global__ void __launch_bounds__(kGSThreads, 1) gate_select_kernel(const GateSe
     p.work_counter[threadIdx.x] = 0u;
   uint32_t seq = 0;
   const ChunkRing<kGSBuffers> ring = {{sm.buf[0], sm.buf[1], sm.buf[2]}};
-  gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim>(p, b, h, ring, sm.bar, seq, sm.row,
-                                                              sm.part);
+  gate_row<kGSThreads, kGSWorkers, kGSBuffers, 256, kHeadDim, 1, true>(p, b, h, ring, sm.bar, seq,
+                                                                       sm.row, sm.part);
   if (p.row_flag != nullptr) {
     __syncthreads();  // every thread's writes of the row come before the flag
     if (threadIdx.x == 0) publish_row(p, b * p.Hkv + h);
