@@ -25,6 +25,38 @@ __global__ void __launch_bounds__(kHeadDim) combine_kernel(const CombineParams p
   if (p.lse_out != nullptr && d == 0) p.lse_out[row] = lse;
 }
 
+// The step's chained combine: one warp per (b, query head) row
+// (combine_row_warp: the same bits as combine_kernel), four rows per CTA,
+// for partials on 16-byte boundaries.
+constexpr int kCombineRowsPerCta = 4;
+
+__global__ void __launch_bounds__(kCombineRowsPerCta * 32)
+    combine_rows_kernel(const CombineParams p, int rows) {
+  pdl_wait();  // the partials come from the preceding decode grid
+  const int row = blockIdx.x * kCombineRowsPerCta + (threadIdx.x >> 5);
+  if (row >= rows) return;  // the whole warp
+  combine_row_warp(p.lse_part + (int64_t)row * p.S, p.o_part + (int64_t)row * p.S * kHeadDim, p.S,
+                   p.out + (int64_t)row * kHeadDim, p.lse_out != nullptr ? p.lse_out + row : nullptr,
+                   Load4L2{}, p.out_host != nullptr ? p.out_host + (int64_t)row * kHeadDim : nullptr);
+}
+
+cudaError_t run_combine_rows(const CombineParams& p, int B, int Hq, cudaStream_t stream,
+                             bool pdl) {
+  const int rows = B * Hq;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((rows + kCombineRowsPerCta - 1) / kCombineRowsPerCta);
+  cfg.blockDim = dim3(kCombineRowsPerCta * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, combine_rows_kernel, p, rows);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(Hq, B);

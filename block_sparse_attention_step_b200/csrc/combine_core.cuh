@@ -65,10 +65,12 @@ __device__ __forceinline__ float combine_element(const float* lse_row, const flo
 // The same merge for one whole (b, query head) row by one warp: lane l takes
 // dims 4l .. 4l+3 and every split's 4 values in one 16-byte load; the split
 // weights come from the lse values through shuffles.  Same arithmetic in the
-// same order as combine_element, so the same bits.  S <= 64.
+// same order as combine_element, so the same bits.  S <= 64; o_row 16-byte
+// aligned.  out_row2 (optional) receives the same bf16 row.
 template <typename LOAD4>
 __device__ __forceinline__ void combine_row_warp(const float* lse_row, const float* o_row, int S,
-                                                 uint16_t* out_row, float* lse_out, LOAD4 load4) {
+                                                 uint16_t* out_row, float* lse_out, LOAD4 load4,
+                                                 uint16_t* out_row2 = nullptr) {
   const int lane = threadIdx.x & 31;
   const float la = lane < S ? __ldcg(lse_row + lane) : -INFINITY;
   const float lb = lane + 32 < S ? __ldcg(lse_row + lane + 32) : -INFINITY;
@@ -91,10 +93,20 @@ __device__ __forceinline__ void combine_row_warp(const float* lse_row, const flo
     }
   }
   const float r = tot > 0.f ? 1.f / tot : 0.f;
-  out_row[4 * lane + 0] = to_bf16_bits(tot > 0.f ? __fmul_rn(acc0, r) : 0.f);
-  out_row[4 * lane + 1] = to_bf16_bits(tot > 0.f ? __fmul_rn(acc1, r) : 0.f);
-  out_row[4 * lane + 2] = to_bf16_bits(tot > 0.f ? __fmul_rn(acc2, r) : 0.f);
-  out_row[4 * lane + 3] = to_bf16_bits(tot > 0.f ? __fmul_rn(acc3, r) : 0.f);
+  const uint16_t v0 = to_bf16_bits(tot > 0.f ? __fmul_rn(acc0, r) : 0.f);
+  const uint16_t v1 = to_bf16_bits(tot > 0.f ? __fmul_rn(acc1, r) : 0.f);
+  const uint16_t v2 = to_bf16_bits(tot > 0.f ? __fmul_rn(acc2, r) : 0.f);
+  const uint16_t v3 = to_bf16_bits(tot > 0.f ? __fmul_rn(acc3, r) : 0.f);
+  out_row[4 * lane + 0] = v0;
+  out_row[4 * lane + 1] = v1;
+  out_row[4 * lane + 2] = v2;
+  out_row[4 * lane + 3] = v3;
+  if (out_row2 != nullptr) {
+    out_row2[4 * lane + 0] = v0;
+    out_row2[4 * lane + 1] = v1;
+    out_row2[4 * lane + 2] = v2;
+    out_row2[4 * lane + 3] = v3;
+  }
   if (lse_out != nullptr && lane == 0) *lse_out = tot > 0.f ? m + logf(tot) : -INFINITY;
 }
 

@@ -641,7 +641,14 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
   c.out_host = out_mapped;
   {
     NvtxRange r("combine");
-    SEER_CUDA(run_combine(c, d->batch, d->num_q_heads, stream, true));
+    // One CTA of 128 threads per (b, query head) row while those fit on the
+    // GPU at once (2048 resident threads per SM); past that, one warp per row
+    // (the same bits), which needs a quarter of the threads.
+    const int64_t rows = (int64_t)d->batch * d->num_q_heads;
+    if (rows * kHeadDim > (int64_t)num_sms * 2048)
+      SEER_CUDA(run_combine_rows(c, d->batch, d->num_q_heads, stream, true));
+    else
+      SEER_CUDA(run_combine(c, d->batch, d->num_q_heads, stream, true));
   }
   if (mass) {
     MassParams m;

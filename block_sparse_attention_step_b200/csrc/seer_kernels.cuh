@@ -176,6 +176,9 @@ cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, cons
                               int num_sms, cudaStream_t stream, bool pdl,
                               uint32_t* ctl = nullptr, uint32_t* row_flag = nullptr);
 cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream, bool pdl);
+// one warp per row; o_part on 16-byte boundaries
+cudaError_t run_combine_rows(const CombineParams& p, int B, int Hq, cudaStream_t stream,
+                             bool pdl);
 cudaError_t run_block_mass(const MassParams& p, int B, cudaStream_t stream);
 
 }  // namespace seer

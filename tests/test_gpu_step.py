@@ -450,18 +450,20 @@ def test_step_head_major_layout_is_bitwise_identical():
         assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("name,splits,q_heads", [
-    ("b16_h40_L32k_bs64_s90", 5, None),
-    ("b16_h40_L32k_bs64_s90", 20, None),       # more splits than one batch of loads
-    ("b64_ragged_h64_paged_bs64", 5, None),
-    ("b64_ragged_h64_paged_bs64", 3, 128),     # G = 16: the one-slot decode shape
+@pytest.mark.parametrize("name,splits,q_heads,batch", [
+    ("b16_h40_L32k_bs64_s90", 5, None, 3),
+    ("b16_h40_L32k_bs64_s90", 20, None, 3),       # more splits than one batch of loads
+    ("b64_ragged_h64_paged_bs64", 5, None, 3),
+    ("b64_ragged_h64_paged_bs64", 3, 128, 3),     # G = 16: the one-slot decode shape
+    ("b64_ragged_h64_paged_bs64", 5, None, 40),   # 2560 rows: the warp-per-row combine
 ])
-def test_step_fused_combine_equals_standalone_combine(name, splits, q_heads):
-    """The step merges the split partials in its chained combine kernel;
-    running the standalone combine on the same partials gives the same bits
-    (more than one batch of 16 splits, and the group size whose decode shape
-    merges in its math warps, included)."""
-    w = W.WORKLOADS[name].replace(batch=3)
+def test_step_fused_combine_equals_standalone_combine(name, splits, q_heads, batch):
+    """The step merges the split partials in its chained combine kernel (one
+    CTA per row, or one warp per row once the rows outnumber what the GPU
+    holds at once); running the standalone combine (one CTA per row) on the
+    same partials gives the same bits (more than one batch of 16 splits, and
+    the group size whose decode shape merges in its math warps, included)."""
+    w = W.WORKLOADS[name].replace(batch=batch)
     if q_heads is not None:
         w = w.replace(q_heads=q_heads)
     if w.seqlen is not None:
