@@ -4,13 +4,14 @@
 // the scores through HBM and without two of the step's launches.
 //
 // Each CTA (512 threads, one per SM) streams its kbar row (NB x 512 bytes)
-// through three 64 KB shared-memory buffers with bulk copies: the first as
-// soon as the row length is in, the others right after the newest block's K
-// loads (so those queue behind one chunk, not three), all before the gate
-// projection g = W qbar is formed, which hides under the copies.  (Measured and dropped: 256-thread CTAs with 24 KB buffers,
-// two per SM, for batches with more rows than SMs -- 5 % slower on the
-// ragged batch, 60 % slower on the headline one; and each 64 KB chunk cut
-// into 4-16 KB bulk copies -- slower at every size.)  The
+// through three 64 KB shared-memory buffers with bulk copies: the first at
+// once (128 rows, before the row length is known), the others right after
+// the newest block's K loads (so those queue behind one chunk, not three),
+// all before the gate projection g = W qbar is formed, which hides under the
+// copies.  (Measured and dropped: 256-thread CTAs with 24 KB buffers, two per
+// SM, for batches with more rows than SMs -- 5 % slower on the ragged batch,
+// 60 % slower on the headline one; and each 64 KB chunk cut into 4-16 KB bulk
+// copies -- slower at every size.)  The
 // newest block's mean is recomputed from K with the same summation order as
 // seer_pool_keys and written back; the scores (also written to the caller's
 // scores buffer) stay in shared memory for the exact value-binned top-k.

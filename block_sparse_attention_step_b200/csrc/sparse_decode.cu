@@ -34,6 +34,9 @@
 //     the item's head rows into o_part / lse_part and free the slot, so the
 //     math warps never stop at item boundaries (the one-slot shapes merge in
 //     the math warps instead, one item later).
+// After the persistent row-claiming gate grid, which publishes each row's
+// flag as it finishes, the scheduler reads a row's indices once its flag is
+// out instead of waiting for the whole gate grid (the ROWFLAGS instantiation).
 // Every mbarrier wait is bounded (SEER_DEV_TIMEOUT); nothing traps.
 #include "gate_row.cuh"
 #include "combine_core.cuh"
