@@ -7,7 +7,8 @@ One step = one pass of the whole hot path over one batch: incremental pooled-
 key update of the newest block, gate scores, top-k block selection, split-KV
 sparse decode and LSE combine (one ``seer_decode_step`` call: the fused
 pool+gate+select kernel, the decode kernel and the combine kernel, chained by
-programmatic dependent launch; the step is replayed as a CUDA graph).
+programmatic dependent launch; the timed steps are replayed as CUDA graphs of
+one whole rotation of the replicas each, so consecutive steps chain too).
 Inputs are seeded synthetic tensors already resident in HBM; the timed loop
 rotates over R independent replicas whose combined footprint exceeds four
 times the L2, so every step reads its K/V, pooled keys and weights from HBM.
@@ -550,7 +551,11 @@ def workload_config(w, num_splits, k_max, rep, layout, args):
            "selection_scope": ("one block set per sequence (all KV heads)" if args.unified
                                else "per KV head"),
            "step_launch": ("single cooperative launch" if args.fused
-                           else "per stage, PDL-chained")}
+                           else "per stage, PDL-chained"),
+           "timed_launches": ("direct C-ABI calls" if args.no_graph
+                              else "one CUDA graph per step" if args.graph_per_step
+                              else "one CUDA graph per rotation of the replicas (PDL between "
+                                   "steps inside it)")}
     return cfg
 
 
@@ -604,10 +609,14 @@ def run_ours(args):
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    # One step per replica captured as a CUDA graph (the step is two kernels
-    # chained by programmatic dependent launch); replaying it keeps host launch
-    # cost out of the device time.  --no-graph launches the C-ABI call directly.
-    graphs = []
+    # CUDA graphs keep host launch cost out of the device time: one graph per
+    # replica holding its step (single steps: warm-up and the per-step
+    # spread), and one graph holding a whole rotation, the replicas' steps one
+    # after another, so that inside it every step's first kernel is chained to
+    # the previous step's last by programmatic dependent launch just as on a
+    # stream (between two graph launches it is not).  --no-graph launches the
+    # C-ABI call directly; --graph-per-step replays the per-replica graphs only.
+    graphs, rotation = [], None
     if not args.no_graph:
         side = torch.cuda.Stream(dev)
         side.wait_stream(stream)
@@ -621,6 +630,11 @@ def run_ours(args):
             with torch.cuda.graph(g):
                 step_call(runs[i].dims, step_args[i], torch.cuda.current_stream())
             graphs.append(g)
+        if not args.graph_per_step:
+            rotation = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(rotation):
+                for i in range(replicas):
+                    step_call(runs[i].dims, step_args[i], torch.cuda.current_stream())
         torch.cuda.synchronize()
 
     def one_step(i):
@@ -628,6 +642,16 @@ def run_ours(args):
             graphs[i % replicas].replay()
         else:
             step_call(runs[i % replicas].dims, step_args[i % replicas], stream)
+
+    def steps_from_zero(k):
+        """Exactly k steps, replicas in turn from replica 0."""
+        i = 0
+        if rotation is not None:
+            for _ in range(k // replicas):
+                rotation.replay()
+            i = k - k % replicas
+        for j in range(i, k):
+            one_step(j)
 
     clocks = ClockSampler(local) if rank == 0 else None
     for i in range(args.warmup):
@@ -639,8 +663,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for i in range(args.steps):
-        one_step(i)
+    steps_from_zero(args.steps)
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -1113,6 +1136,8 @@ def main(argv=None):
                    help="host bytes of oracle inputs (K and V rows); a batch above it is sampled")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-graph", action="store_true", help="launch each step directly, no CUDA graph")
+    p.add_argument("--graph-per-step", action="store_true",
+                   help="replay one graph per step (no whole-rotation graph)")
     p.add_argument("--mass", action="store_true",
                    help="also emit every block's attention mass (dense-mode gate target)")
     p.add_argument("--recall", action="store_true",
