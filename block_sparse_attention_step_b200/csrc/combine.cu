@@ -27,21 +27,23 @@ __global__ void __launch_bounds__(kHeadDim) combine_kernel(const CombineParams p
 
 // The step's chained combine: one warp per (b, query head) row
 // (combine_row_warp: the same bits as combine_kernel), four rows per CTA,
-// for partials on 16-byte boundaries.
+// for partials on 16-byte boundaries; PACKED for 8-byte aligned outputs.
 constexpr int kCombineRowsPerCta = 4;
 
+template <bool PACKED>
 __global__ void __launch_bounds__(kCombineRowsPerCta * 32)
     combine_rows_kernel(const CombineParams p, int rows) {
   pdl_wait();  // the partials come from the preceding decode grid
   const int row = blockIdx.x * kCombineRowsPerCta + (threadIdx.x >> 5);
   if (row >= rows) return;  // the whole warp
-  combine_row_warp(p.lse_part + (int64_t)row * p.S, p.o_part + (int64_t)row * p.S * kHeadDim, p.S,
-                   p.out + (int64_t)row * kHeadDim, p.lse_out != nullptr ? p.lse_out + row : nullptr,
-                   Load4L2{}, p.out_host != nullptr ? p.out_host + (int64_t)row * kHeadDim : nullptr);
+  combine_row_warp<Load4L2, PACKED>(
+      p.lse_part + (int64_t)row * p.S, p.o_part + (int64_t)row * p.S * kHeadDim, p.S,
+      p.out + (int64_t)row * kHeadDim, p.lse_out != nullptr ? p.lse_out + row : nullptr, Load4L2{},
+      p.out_host != nullptr ? p.out_host + (int64_t)row * kHeadDim : nullptr);
 }
 
 cudaError_t run_combine_rows(const CombineParams& p, int B, int Hq, cudaStream_t stream,
-                             bool pdl) {
+                             bool pdl, bool packed) {
   const int rows = B * Hq;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((rows + kCombineRowsPerCta - 1) / kCombineRowsPerCta);
@@ -52,7 +54,8 @@ cudaError_t run_combine_rows(const CombineParams& p, int B, int Hq, cudaStream_t
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, combine_rows_kernel, p, rows);
+  cudaError_t e = packed ? cudaLaunchKernelEx(&cfg, combine_rows_kernel<true>, p, rows)
+                         : cudaLaunchKernelEx(&cfg, combine_rows_kernel<false>, p, rows);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -66,8 +66,10 @@ __device__ __forceinline__ float combine_element(const float* lse_row, const flo
 // dims 4l .. 4l+3 and every split's 4 values in one 16-byte load; the split
 // weights come from the lse values through shuffles.  Same arithmetic in the
 // same order as combine_element, so the same bits.  S <= 64; o_row 16-byte
-// aligned.  out_row2 (optional) receives the same bf16 row.
-template <typename LOAD4>
+// aligned.  out_row2 (optional) receives the same bf16 row.  PACKED: each
+// lane stores its four values as one 8-byte word (both rows 8-byte aligned),
+// so a warp writes a row in one contiguous 256-byte store.
+template <typename LOAD4, bool PACKED = false>
 __device__ __forceinline__ void combine_row_warp(const float* lse_row, const float* o_row, int S,
                                                  uint16_t* out_row, float* lse_out, LOAD4 load4,
                                                  uint16_t* out_row2 = nullptr) {
@@ -97,15 +99,21 @@ __device__ __forceinline__ void combine_row_warp(const float* lse_row, const flo
   const uint16_t v1 = to_bf16_bits(tot > 0.f ? __fmul_rn(acc1, r) : 0.f);
   const uint16_t v2 = to_bf16_bits(tot > 0.f ? __fmul_rn(acc2, r) : 0.f);
   const uint16_t v3 = to_bf16_bits(tot > 0.f ? __fmul_rn(acc3, r) : 0.f);
-  out_row[4 * lane + 0] = v0;
-  out_row[4 * lane + 1] = v1;
-  out_row[4 * lane + 2] = v2;
-  out_row[4 * lane + 3] = v3;
-  if (out_row2 != nullptr) {
-    out_row2[4 * lane + 0] = v0;
-    out_row2[4 * lane + 1] = v1;
-    out_row2[4 * lane + 2] = v2;
-    out_row2[4 * lane + 3] = v3;
+  if constexpr (PACKED) {
+    const uint2 w = make_uint2((uint32_t)v0 | ((uint32_t)v1 << 16), (uint32_t)v2 | ((uint32_t)v3 << 16));
+    *reinterpret_cast<uint2*>(out_row + 4 * lane) = w;
+    if (out_row2 != nullptr) *reinterpret_cast<uint2*>(out_row2 + 4 * lane) = w;
+  } else {
+    out_row[4 * lane + 0] = v0;
+    out_row[4 * lane + 1] = v1;
+    out_row[4 * lane + 2] = v2;
+    out_row[4 * lane + 3] = v3;
+    if (out_row2 != nullptr) {
+      out_row2[4 * lane + 0] = v0;
+      out_row2[4 * lane + 1] = v1;
+      out_row2[4 * lane + 2] = v2;
+      out_row2[4 * lane + 3] = v3;
+    }
   }
   if (lse_out != nullptr && lane == 0) *lse_out = tot > 0.f ? m + logf(tot) : -INFINITY;
 }

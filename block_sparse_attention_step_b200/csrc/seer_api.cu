@@ -644,9 +644,12 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
     // One CTA of 128 threads per (b, query head) row while those fit on the
     // GPU at once (2048 resident threads per SM); past that, one warp per row
     // (the same bits), which needs a quarter of the threads.
+    // Output in mapped host memory: one warp per row with 8-byte stores when
+    // both outputs allow them, so each row crosses PCIe as one 256-byte write.
     const int64_t rows = (int64_t)d->batch * d->num_q_heads;
-    if (rows * kHeadDim > (int64_t)num_sms * 2048)
-      SEER_CUDA(run_combine_rows(c, d->batch, d->num_q_heads, stream, true));
+    const bool packed = aligned(a->out, 8) && (out_mapped == nullptr || aligned(out_mapped, 8));
+    if (rows * kHeadDim > (int64_t)num_sms * 2048 || (out_mapped != nullptr && packed))
+      SEER_CUDA(run_combine_rows(c, d->batch, d->num_q_heads, stream, true, packed));
     else
       SEER_CUDA(run_combine(c, d->batch, d->num_q_heads, stream, true));
   }

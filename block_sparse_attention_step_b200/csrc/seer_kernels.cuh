@@ -176,9 +176,10 @@ cudaError_t run_sparse_decode(const CUtensorMap& tk, const CUtensorMap& tv, cons
                               int num_sms, cudaStream_t stream, bool pdl,
                               uint32_t* ctl = nullptr, uint32_t* row_flag = nullptr);
 cudaError_t run_combine(const CombineParams& p, int B, int Hq, cudaStream_t stream, bool pdl);
-// one warp per row; o_part on 16-byte boundaries
+// one warp per row; o_part on 16-byte boundaries; packed: out (and out_host)
+// on 8-byte boundaries, written 8 bytes per lane
 cudaError_t run_combine_rows(const CombineParams& p, int B, int Hq, cudaStream_t stream,
-                             bool pdl);
+                             bool pdl, bool packed);
 cudaError_t run_block_mass(const MassParams& p, int B, cudaStream_t stream);
 
 }  // namespace seer
