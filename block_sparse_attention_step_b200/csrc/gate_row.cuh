@@ -150,24 +150,36 @@ __device__ bool gate_row(const GateSelectParams& p, int b, int h, const ChunkRin
     *reinterpret_cast<uint2*>(p.v_pool_w + off) = __ldg(reinterpret_cast<const uint2*>(p.v_new + src));
   }
 
-  // mean query of the group (q in mapped host memory: read through L2 and
-  // copied to q_copy for the decode)
+  // mean query of the group
   if (tid >= QFIRST && tid < QFIRST + QTHREADS) {
+    const int64_t row0 = ((int64_t)b * p.Hq + (int64_t)h * p.G) * kHeadDim;
+    if (p.q_copy != nullptr) {
+      // q in mapped host memory (16-byte aligned): the group's G rows, one
+      // contiguous G x 256 bytes, cross PCIe as 16-byte words in one round
+      // trip, are copied to q_copy for the decode and staged in the score
+      // buffer (free until the chunk loop) for the mean below
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + row0);
+      uint4* dst = reinterpret_cast<uint4*>(p.q_copy + row0);
+      uint4* stage = reinterpret_cast<uint4*>(gs.scores);
+      const int words = p.G * kHeadDim * 2 / 16;
+      for (int w = tid - QFIRST; w < words; w += QTHREADS) {
+        const uint4 v = __ldcg(src + w);
+        stage[w] = v;
+        dst[w] = v;
+      }
+      named_barrier_sync(2, QTHREADS);  // the mean-query threads only
+    }
+    const uint16_t* staged = reinterpret_cast<const uint16_t*>(gs.scores);
 #pragma unroll
     for (int m = 0; m < kHeadDim / QTHREADS; ++m) {
       const int d = tid - QFIRST + m * QTHREADS;
-      const int64_t off = ((int64_t)b * p.Hq + (int64_t)h * p.G) * kHeadDim + d;
       float s = 0.f;
       if (p.q_copy != nullptr) {
-        for (int g = 0; g < p.G; ++g) {
-          const unsigned short v = __ldcg(reinterpret_cast<const unsigned short*>(p.q) + off +
-                                          g * kHeadDim);
-          p.q_copy[off + g * kHeadDim] = v;
-          s += __uint_as_float((uint32_t)v << 16);
-        }
+        for (int g = 0; g < p.G; ++g)
+          s += __uint_as_float((uint32_t)staged[g * kHeadDim + d] << 16);
       } else {
         for (int g = 0; g < p.G; ++g)
-          s += __uint_as_float((uint32_t)__ldg(p.q + off + g * kHeadDim) << 16);
+          s += __uint_as_float((uint32_t)__ldg(p.q + row0 + d + g * kHeadDim) << 16);
       }
       gs.qbar[d] = s / (float)p.G;
     }

@@ -876,7 +876,9 @@ seer_status seer_decode_step_host(const seer_dims* d, const seer_step_args* a,
   const size_t bytes = (size_t)d->batch * d->num_q_heads * d->head_dim * sizeof(uint16_t);
   // mapped buffers are read and written by the step's own kernels; others
   // go through a copy on the stream
+  // (the gate reads mapped q as 16-byte words: a q_host off that boundary is copied)
   const uint16_t* q_map = static_cast<const uint16_t*>(mapped_host_ptr(q_host));
+  if (q_map != nullptr && !aligned(q_map, 16)) q_map = nullptr;
   uint16_t* out_map = static_cast<uint16_t*>(mapped_host_ptr(out_host));
   if (q_map == nullptr)
     SEER_CUDA(cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, stream));

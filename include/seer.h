@@ -301,8 +301,8 @@ SEER_API seer_status seer_decode_step(const seer_dims *d, const seer_step_args *
  * is pinned and mapped into the device's address space (cudaHostAlloc /
  * cudaMallocHost memory, or cudaHostRegister'ed with the mapped flag; see
  * seer_host_ptr_mapped) is accessed by the step's kernels directly: the gate
- * reads q_host and fills q_dev, the combine writes out_host, and no copy is
- * enqueued.  Any other host buffer goes through cudaMemcpyAsync on `stream`
+ * reads q_host (when it is also 16-byte aligned) and fills q_dev, the combine
+ * writes out_host, and no copy is enqueued.  Any other host buffer goes through cudaMemcpyAsync on `stream`
  * (before the step for q, after it for out).  Asynchronous either way: q_host
  * must stay unchanged and out_host is valid only once the stream is
  * synchronised. */
