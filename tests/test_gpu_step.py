@@ -324,6 +324,41 @@ def test_step_host_entry_point_matches_device_step(name, pinned_q, pinned_out):
     assert torch.equal(run.out, dev_out)
 
 
+@pytest.mark.parametrize("name", list(HOST_CASES) + ["many_query_rows"])
+def test_step_host_entry_point_off_boundary_buffers(name):
+    """Pinned (mapped) host buffers that start one element into their
+    allocation: q off a 16-byte boundary goes through the copy instead of the
+    gate's 16-byte reads, and out off an 8-byte boundary is written by the
+    combine element by element (per-row CTAs, or one warp per row with 2-byte
+    stores once the rows outnumber one wave); the same bits as the device
+    step either way."""
+    w = (W.WORKLOADS["b64_ragged_h64_paged_bs64"].replace(batch=40, seqlen_range=(64, 3000))
+         if name == "many_query_rows" else HOST_CASES[name])
+    data = W.generate(w, 5, DEV)
+    run = StepBuffers(w, data)
+    run.pool_full()
+    kbar0 = run.kbar.clone()
+    run.step(update_kbar=1)
+    torch.cuda.synchronize()
+    dev_out = run.out.clone()
+    n = data["q"].numel()
+    q_buf = torch.zeros(n + 8, dtype=torch.bfloat16).pin_memory()
+    q_host = q_buf[1:1 + n].view(data["q"].shape)
+    q_host.copy_(data["q"].cpu())
+    out_buf = torch.zeros(dev_out.numel() + 8, dtype=torch.bfloat16).pin_memory()
+    out_host = out_buf[1:1 + dev_out.numel()].view(dev_out.shape)
+    assert q_host.data_ptr() % 16 != 0 and out_host.data_ptr() % 8 != 0
+    q_dev = torch.zeros_like(data["q"])
+    run.kbar.copy_(kbar0)
+    run.out.zero_()
+    seer.seer_decode_step_host(run.dims, run.args(1, q=q_dev), q_host, q_dev, out_host)
+    torch.cuda.synchronize()
+    assert run.status.item() == 0
+    assert torch.equal(q_dev.cpu(), q_host)
+    assert torch.equal(out_host, dev_out.cpu())
+    assert torch.equal(run.out, dev_out)
+
+
 # --------------------------------------------------------- full-size, sampled
 
 FULL = [
