@@ -57,3 +57,36 @@ def test_noalloc_step_matches_workspace_step_twice():
     with pytest.raises(seer.SeerError) as e:
         seer.seer_decode_step_noalloc(big, args)
     assert e.value.status == 4          # SEER_ERR_WORKSPACE
+
+
+def test_noalloc_steps_of_different_shapes_in_turn():
+    """Differently shaped steps through the one fixed array, in turn.  The control words
+    and row flags sit at an offset that depends on the shape, so each call lands on what
+    the call before it left in the array (partials, indices, or its own flags at another
+    offset); every call must still give the caller-workspace step's bits."""
+    require_gpu()
+    base = W.WORKLOADS["b8_h32_L8k_bs64_s90_newest"]
+    shapes = [
+        base.replace(batch=20, seqlen=2000),   # 160 rows: the row-claiming gate, row flags on
+        base.replace(batch=3, seqlen=5000),    # 24 rows: one gate CTA per row
+        W.WORKLOADS["b16_h40_L32k_bs128_budget4k_newest"].replace(batch=2, seqlen=4000),
+    ]
+    runs = []
+    for i, w in enumerate(shapes):
+        run = StepBuffers(w, W.generate(w, 30 + i, "cuda"))
+        run.pool_full()
+        run.step(update_kbar=0)
+        torch.cuda.synchronize()
+        assert run.status.item() == 0, i
+        assert seer.seer_step_workspace_bytes(run.dims, run.k_max, run.num_splits) \
+            <= seer.NOALLOC_SCRATCH_BYTES
+        runs.append((run, run.out.clone(), run.lse.clone()))
+    for rep in range(2):
+        for i, (run, ref_out, ref_lse) in enumerate(runs):
+            run.out.fill_(0)
+            run.lse.fill_(0)
+            seer.seer_decode_step_noalloc(run.dims, run.args(update_kbar=0))
+            torch.cuda.synchronize()
+            assert run.status.item() == 0, (rep, i)
+            assert torch.equal(run.out, ref_out), (rep, i)
+            assert torch.equal(run.lse, ref_lse), (rep, i)
