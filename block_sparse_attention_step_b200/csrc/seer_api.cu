@@ -516,12 +516,21 @@ seer_status seer_combine(const seer_dims* d, const float* o_part, const float* l
   return SEER_OK;
 }
 
-// The step; q_mapped / out_mapped (optional): host memory mapped into the
-// device, read by the gate (which fills a->q for the decode) / written by the
-// combine besides a->out.
+// What an entry point adds around the step's kernels, enqueued only once
+// every check has passed.
+struct StepExtras {
+  const uint16_t* q_mapped = nullptr;     // host q mapped into the device: the gate reads
+                                          // it and fills a->q for the decode
+  uint16_t* out_mapped = nullptr;         // host out mapped into the device: the combine
+                                          // writes it besides a->out
+  const uint16_t* q_host_copy = nullptr;  // host q copied into a->q before the kernels
+  bool zero_ctl = false;                  // control words and row flags zeroed first
+};
+
 static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
-                                    seer_stream stream, const uint16_t* q_mapped,
-                                    uint16_t* out_mapped) {
+                                    seer_stream stream, const StepExtras& x) {
+  const uint16_t* q_mapped = x.q_mapped;
+  uint16_t* out_mapped = x.out_mapped;
   NvtxRange step_range("seer_decode_step");
   SEER_TRY(check_dims(d));
   if (a == nullptr || a->k_per_seq == nullptr || a->kbar == nullptr) return SEER_ERR_INVALID_ARG;
@@ -544,6 +553,11 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
   if (mass && (!a->block_mass || !a->block_lse || !a->lse_out)) return SEER_ERR_INVALID_ARG;
   L.p.block_lse = mass ? a->block_lse : nullptr;
 
+  if (x.zero_ctl) SEER_CUDA(cudaMemsetAsync(w.work_counter, 0, w.ctl_bytes, stream));
+  if (x.q_host_copy != nullptr)
+    SEER_CUDA(cudaMemcpyAsync(const_cast<uint16_t*>(a->q), x.q_host_copy,
+                              (size_t)d->batch * d->num_q_heads * kHeadDim * sizeof(uint16_t),
+                              cudaMemcpyHostToDevice, stream));
   if (a->update_kbar == 2) {
     NvtxRange r("pool_keys (full rebuild)");
     SEER_TRY(seer_pool_keys(d, a->k_pool, a->page_table, a->seqlens, 0, a->kbar, a->dev_status,
@@ -674,7 +688,17 @@ static seer_status decode_step_impl(const seer_dims* d, const seer_step_args* a,
 }
 
 seer_status seer_decode_step(const seer_dims* d, const seer_step_args* a, seer_stream stream) {
-  return decode_step_impl(d, a, stream, nullptr, nullptr);
+  return decode_step_impl(d, a, stream, StepExtras{});
+}
+
+// The step with its control words zeroed on the stream first, after every
+// check (the no-allocation entry point, whose workspace is shared by calls
+// of any shape).
+seer_status decode_step_zeroed_ctl(const seer_dims* d, const seer_step_args* a,
+                                   seer_stream stream) {
+  StepExtras x;
+  x.zero_ctl = true;
+  return decode_step_impl(d, a, stream, x);
 }
 
 seer_status seer_step_workspace_init(const seer_dims* d, int32_t k_max, int32_t num_splits,
@@ -877,15 +901,15 @@ seer_status seer_decode_step_host(const seer_dims* d, const seer_step_args* a,
   // mapped buffers are read and written by the step's own kernels; others
   // go through a copy on the stream
   // (the gate reads mapped q as 16-byte words: a q_host off that boundary is copied)
-  const uint16_t* q_map = static_cast<const uint16_t*>(mapped_host_ptr(q_host));
-  if (q_map != nullptr && !aligned(q_map, 16)) q_map = nullptr;
-  uint16_t* out_map = static_cast<uint16_t*>(mapped_host_ptr(out_host));
-  if (q_map == nullptr)
-    SEER_CUDA(cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, stream));
+  StepExtras x;
+  x.q_mapped = static_cast<const uint16_t*>(mapped_host_ptr(q_host));
+  if (x.q_mapped != nullptr && !aligned(x.q_mapped, 16)) x.q_mapped = nullptr;
+  x.out_mapped = static_cast<uint16_t*>(mapped_host_ptr(out_host));
+  if (x.q_mapped == nullptr) x.q_host_copy = q_host;  // copied after the step's checks
   seer_step_args b = *a;
   b.q = q_dev;
-  SEER_TRY(decode_step_impl(d, &b, stream, q_map, out_map));
-  if (out_map == nullptr)
+  SEER_TRY(decode_step_impl(d, &b, stream, x));
+  if (x.out_mapped == nullptr)
     SEER_CUDA(cudaMemcpyAsync(out_host, a->out, bytes, cudaMemcpyDeviceToHost, stream));
   return SEER_OK;
 }

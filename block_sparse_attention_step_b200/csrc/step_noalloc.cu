@@ -33,6 +33,12 @@ void* scratch_address(int device) {
 
 }  // namespace
 
+// seer_decode_step with the control words and row flags zeroed on the stream
+// after every check and before the kernels (defined with the other step
+// entry points; C linkage, hidden like every symbol outside the header).
+extern "C" seer_status decode_step_zeroed_ctl(const seer_dims* d, const seer_step_args* a,
+                                              seer_stream stream);
+
 extern "C" {
 
 seer_status seer_decode_step_noalloc(const seer_dims* d, const seer_step_args* a,
@@ -50,11 +56,8 @@ seer_status seer_decode_step_noalloc(const seer_dims* d, const seer_step_args* a
   b.workspace_bytes = kScratchBytes;
   // The control words sit at an offset that depends on the shape, k_max and
   // split count, so a call after a differently shaped one would find other
-  // data there: zero them on the stream first.
-  const seer_status z =
-      seer_step_workspace_init(d, a->k_max, a->num_splits, scratch, kScratchBytes, stream);
-  if (z != SEER_OK) return z;
-  return seer_decode_step(d, &b, stream);
+  // data there: the step zeroes them on the stream first.
+  return decode_step_zeroed_ctl(d, &b, stream);
 }
 
 }  // extern "C"

@@ -102,6 +102,11 @@ def test_invalid_arguments_fail_before_any_launch(lib):
     a.k_max = 4
     a.num_splits = 1
     assert lib.seer_decode_step(ctypes.byref(d), ctypes.byref(a), null) == 4
+    # the host-buffer form checks the step before it enqueues q's copy (a copy
+    # enqueued first would fail here with a CUDA error, or land on a GPU)
+    a.out = fake
+    assert lib.seer_decode_step_host(ctypes.byref(d), ctypes.byref(a), fake, fake, fake,
+                                     null) == 4
 
 
 def test_workspace_and_default_splits(lib):
